@@ -1,0 +1,243 @@
+"""ctypes wrapper for the CPU oracle (oracle.c).
+
+TEST INFRASTRUCTURE ONLY. The test suite, the smoke check and the bench's
+CPU-baseline leg use it. The product path never imports it.
+
+Every function takes and returns numpy arrays. The C library is built on
+first use with gcc (-O2 -ffp-contract=off, no fast-math), or ahead of time by
+build().
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so in place. Returns its path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < max(
+            os.path.getmtime(_SRC), os.path.getmtime(os.path.join(_HERE, "oracle.h"))):
+        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+               "-fPIC", "-shared", "-o", _LIB + ".tmp", _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    build()
+    lib = ctypes.CDLL(_LIB)
+    P = ctypes.c_void_p
+    i64, i32, u64 = ctypes.c_int64, ctypes.c_int, ctypes.c_uint64
+    lib.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
+    lib.orc_bf16_to_f32.restype = ctypes.c_float
+    lib.orc_f32_to_bf16.argtypes = [ctypes.c_float]
+    lib.orc_f32_to_bf16.restype = ctypes.c_uint16
+    lib.orc_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.orc_e4m3_encode.restype = ctypes.c_uint8
+    lib.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+    lib.orc_e4m3_decode.restype = ctypes.c_float
+    lib.orc_splitmix64.argtypes = [u64]
+    lib.orc_splitmix64.restype = u64
+    lib.orc_route_softmax.argtypes = [P, i64, i32, i32, i32, P, P]
+    lib.orc_route_softmax.restype = None
+    lib.orc_route_group_sigmoid.argtypes = [P, i64, i32, i32, i32, i32, P, P, P]
+    lib.orc_route_group_sigmoid.restype = None
+    lib.orc_apply_mask.argtypes = [P, P, i64, i32, u64, u64]
+    lib.orc_apply_mask.restype = None
+    lib.orc_layout.argtypes = [P, i32, i32, i32, i32, P, P, P, P, P, P, P, P]
+    lib.orc_layout.restype = i32
+    lib.orc_quant_fp8_row.argtypes = [P, i32, P, P]
+    lib.orc_quant_fp8_row.restype = None
+    lib.orc_dispatch.argtypes = [P, P, P, i64, i32, i32, i32, P, P, P, P]
+    lib.orc_dispatch.restype = None
+    lib.orc_identity_expert_fp8.argtypes = [P, P, i64, i32, P]
+    lib.orc_identity_expert_fp8.restype = None
+    lib.orc_combine.argtypes = [P, P, P, P, i64, i32, i32, P, i64, P]
+    lib.orc_combine.restype = None
+    _lib = lib
+    return lib
+
+
+def _p(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# ---- number formats --------------------------------------------------------
+
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    lib = _load()
+    flat = np.ascontiguousarray(bits, dtype=np.uint16).ravel()
+    return np.array([lib.orc_bf16_to_f32(int(b)) for b in flat], dtype=np.float32).reshape(np.shape(bits))
+
+
+def f32_to_bf16(x: np.ndarray) -> np.ndarray:
+    lib = _load()
+    flat = np.ascontiguousarray(x, dtype=np.float32).ravel()
+    return np.array([lib.orc_f32_to_bf16(float(v)) for v in flat], dtype=np.uint16).reshape(np.shape(x))
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    lib = _load()
+    flat = np.ascontiguousarray(x, dtype=np.float32).ravel()
+    return np.array([lib.orc_e4m3_encode(float(v)) for v in flat], dtype=np.uint8).reshape(np.shape(x))
+
+
+def e4m3_decode(c: np.ndarray) -> np.ndarray:
+    lib = _load()
+    flat = np.ascontiguousarray(c, dtype=np.uint8).ravel()
+    return np.array([lib.orc_e4m3_decode(int(v)) for v in flat], dtype=np.float32).reshape(np.shape(c))
+
+
+def splitmix64(counter: int) -> int:
+    return int(_load().orc_splitmix64(counter & 0xFFFF_FFFF_FFFF_FFFF))
+
+
+def mask_threshold(frac: float) -> int:
+    """Threshold on the high 32 bits of the hash: floor(frac * 2^32), taken on
+    the fp32 value of frac."""
+    f = float(np.float32(frac))
+    return int(min(max(np.floor(f * 4294967296.0), 0.0), 4294967296.0))
+
+
+# ---- routing ---------------------------------------------------------------
+
+def route(logits: np.ndarray, K: int, route_kind: int, G: int = 1, KG: int = 1):
+    """Returns (topk_idx int32 [N,K], topk_w fp32 [N,K], margin fp64 [N] or None)."""
+    lib = _load()
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    N, E = logits.shape
+    idx = np.empty((N, K), dtype=np.int32)
+    w = np.empty((N, K), dtype=np.float32)
+    if route_kind == 2:
+        margin = np.empty(N, dtype=np.float64)
+        lib.orc_route_group_sigmoid(_p(logits), N, E, K, G, KG, _p(idx), _p(w), _p(margin))
+        return idx, w, margin
+    lib.orc_route_softmax(_p(logits), N, E, K, 1 if route_kind == 1 else 0, _p(idx), _p(w))
+    return idx, w, None
+
+
+def apply_mask(idx: np.ndarray, w: np.ndarray, seed: int, frac: float) -> None:
+    """In place: masks slots to -1 / weight 0."""
+    N, K = idx.shape
+    _load().orc_apply_mask(_p(idx), _p(w), N, K, seed & 0xFFFF_FFFF_FFFF_FFFF, mask_threshold(frac))
+
+
+# ---- layout ----------------------------------------------------------------
+
+def layout(idx: np.ndarray, R: int, T: int, E: int) -> dict:
+    lib = _load()
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    N, K = idx.shape
+    assert N == R * T
+    out = dict(
+        is_token_in_rank=np.empty((N, R), dtype=np.uint8),
+        num_tokens_per_rank=np.empty((R, R), dtype=np.int32),
+        cnt=np.empty((R, E), dtype=np.int32),
+        num_tokens_per_expert=np.empty(E, dtype=np.int32),
+        expert_off=np.empty(E + 1, dtype=np.int32),
+        rank_off=np.empty(R + 1, dtype=np.int32),
+        src_off=np.empty((E, R), dtype=np.int32),
+        dst_row=np.empty((N, K), dtype=np.int32),
+    )
+    err = lib.orc_layout(_p(idx), R, T, E, K, _p(out["is_token_in_rank"]),
+                         _p(out["num_tokens_per_rank"]), _p(out["cnt"]),
+                         _p(out["num_tokens_per_expert"]), _p(out["expert_off"]),
+                         _p(out["rank_off"]), _p(out["src_off"]), _p(out["dst_row"]))
+    out["error"] = int(err)
+    return out
+
+
+# ---- dispatch / combine ----------------------------------------------------
+
+def quant_fp8_row(x_row: np.ndarray):
+    x_row = np.ascontiguousarray(x_row, dtype=np.uint16)
+    H = x_row.shape[0]
+    q = np.empty(H, dtype=np.uint8)
+    s = np.empty(H // 128, dtype=np.float32)
+    _load().orc_quant_fp8_row(_p(x_row), H, _p(q), _p(s))
+    return q, s
+
+
+def dispatch(x: np.ndarray, dst_row: np.ndarray, topk_w: np.ndarray, M: int, fp8: bool):
+    """Returns (recv_x, recv_scale or None, recv_src, recv_w) with M rows."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    dst_row = np.ascontiguousarray(dst_row, dtype=np.int32)
+    topk_w = np.ascontiguousarray(topk_w, dtype=np.float32)
+    N, H = x.shape
+    K = dst_row.shape[1]
+    recv_x = np.zeros((M, H), dtype=np.uint8 if fp8 else np.uint16)
+    recv_scale = np.zeros((M, H // 128), dtype=np.float32) if fp8 else None
+    recv_src = np.full(M, -1, dtype=np.int32)
+    recv_w = np.zeros(M, dtype=np.float32)
+    _load().orc_dispatch(_p(x), _p(dst_row), _p(topk_w), N, H, K, 1 if fp8 else 0,
+                         _p(recv_x), _p(recv_scale), _p(recv_src), _p(recv_w))
+    return recv_x, recv_scale, recv_src, recv_w
+
+
+def identity_expert_fp8(q: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    scale = np.ascontiguousarray(scale, dtype=np.float32)
+    M, H = q.shape
+    y = np.empty((M, H), dtype=np.uint16)
+    _load().orc_identity_expert_fp8(_p(q), _p(scale), M, H, _p(y))
+    return y
+
+
+def combine(y: np.ndarray, y_scale: np.ndarray | None, dst_row: np.ndarray, topk_w: np.ndarray,
+            tokens: np.ndarray | None = None) -> np.ndarray:
+    """Returns bf16 bits [n_tokens, H] (all N tokens when tokens is None).
+
+    y is bf16 bits [M,H] (y_scale None) or e4m3 codes [M,H] with fp32 scales
+    [M,H/128]."""
+    y = np.ascontiguousarray(y)
+    dst_row = np.ascontiguousarray(dst_row, dtype=np.int32)
+    topk_w = np.ascontiguousarray(topk_w, dtype=np.float32)
+    N, K = dst_row.shape
+    H = y.shape[1]
+    if tokens is not None:
+        tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+        n = tokens.shape[0]
+    else:
+        n = N
+    out = np.empty((n, H), dtype=np.uint16)
+    _load().orc_combine(_p(y), _p(y_scale), _p(dst_row), _p(topk_w), N, H, K,
+                        _p(tokens), n, _p(out))
+    return out
+
+
+def run_path(x: np.ndarray, logits: np.ndarray | None, w, topk_idx=None, topk_w=None,
+             combine_tokens=None, fp8_combine_fused: bool = False):
+    """Whole path on the CPU for workload w: routing (or the given top-k),
+    mask, layout, dispatch, identity expert and combine. Returns a dict."""
+    if topk_idx is None:
+        idx, tw, margin = route(logits, w.K, w.route, w.G, w.KG)
+        if w.mask_frac:
+            apply_mask(idx, tw, w.mask_seed, w.mask_frac)
+    else:
+        idx, tw, margin = np.array(topk_idx, dtype=np.int32), np.array(topk_w, dtype=np.float32), None
+    lay = layout(idx, w.R, w.T, w.E)
+    M = int(lay["expert_off"][-1])
+    recv_x, recv_scale, recv_src, recv_w = dispatch(x, lay["dst_row"], tw, M, w.fp8)
+    if w.fp8 and not fp8_combine_fused:
+        y, ys = identity_expert_fp8(recv_x, recv_scale), None
+    else:
+        y, ys = recv_x, recv_scale
+    out = combine(y, ys, lay["dst_row"], tw, combine_tokens)
+    return dict(topk_idx=idx, topk_w=tw, margin=margin, M=M, recv_x=recv_x,
+                recv_scale=recv_scale, recv_src=recv_src, recv_w=recv_w, y=y, out=out, **lay)

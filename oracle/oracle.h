@@ -1,0 +1,91 @@
+/*
+ * CPU oracle for MoE expert-parallel dispatch / combine with group-limited top-k.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the test suite, the smoke check and the
+ * bench's CPU-baseline leg may load this library. The product path (the CUDA
+ * library and its Python binding) never calls it and shares no code with it.
+ *
+ * Plain single-threaded C11. Each function states the definition it writes out.
+ * Floating point is IEEE binary64 wherever the method leaves the precision
+ * open (routing scores and weights). It is binary32 where the method fixes
+ * binary32:
+ *  - the FP8 scale arithmetic;
+ *  - the top-k weighted combine, accumulated in fp32 with one rounding to bf16.
+ *
+ * Parity unpinned (conventions, not results; no independent pin exists):
+ *  - the group-limited weight normalisation w_k = s_k / sum_j s_j, with no
+ *    extra routed scaling factor;
+ *  - the amax floor 1e-4 used by the FP8 quantiser for all-zero blocks.
+ */
+#ifndef COMBINE_TOP_GROUP_ORACLE_H
+#define COMBINE_TOP_GROUP_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- number formats ---------------------------------------------------- */
+float    orc_bf16_to_f32(uint16_t b);
+uint16_t orc_f32_to_bf16(float f);           /* round to nearest even */
+uint8_t  orc_e4m3_encode(float v);           /* OCP e4m3fn, RNE, saturate to +-448 */
+float    orc_e4m3_decode(uint8_t c);
+uint64_t orc_splitmix64(uint64_t counter);   /* first output of SplitMix64 seeded with counter */
+
+/* ---- routing ----------------------------------------------------------- */
+/* Softmax top-K. idx [N,K] int32, w [N,K] fp32. renorm != 0 rescales the K
+ * selected probabilities to sum 1. */
+void orc_route_softmax(const float *logits, int64_t N, int E, int K, int renorm,
+                       int32_t *idx, float *w);
+
+/* Group-limited sigmoid gating. margin [N] (may be NULL) receives, per token,
+ * the fp64 gap between the last kept group score and the best dropped one
+ * (+inf when every group is kept). */
+void orc_route_group_sigmoid(const float *logits, int64_t N, int E, int K, int G, int KG,
+                             int32_t *idx, float *w, double *margin);
+
+/* Mask slot (g,k) to -1 (weight 0) when the high 32 bits of
+ * splitmix64(seed ^ (g*K + k)) are below threshold. */
+void orc_apply_mask(int32_t *idx, float *w, int64_t N, int K, uint64_t seed, uint64_t threshold);
+
+/* ---- layout ------------------------------------------------------------ */
+/* Returns a bitmask of data errors: bit 0 = expert id outside [-1, E) (the slot
+ * is then treated as masked). Output shapes:
+ *   is_token_in_rank u8 [N,R], num_tokens_per_rank i32 [R,R], cnt i32 [R,E],
+ *   num_tokens_per_expert i32 [E], expert_off i32 [E+1], rank_off i32 [R+1],
+ *   src_off i32 [E,R], dst_row i32 [N,K]. */
+int orc_layout(const int32_t *idx, int R, int T, int E, int K,
+               uint8_t *is_token_in_rank, int32_t *num_tokens_per_rank, int32_t *cnt,
+               int32_t *num_tokens_per_expert, int32_t *expert_off, int32_t *rank_off,
+               int32_t *src_off, int32_t *dst_row);
+
+/* ---- dispatch ---------------------------------------------------------- */
+/* Quantise one bf16 row of H channels (H % 128 == 0) to e4m3 with one fp32
+ * scale per 128-channel block. */
+void orc_quant_fp8_row(const uint16_t *x, int H, uint8_t *q, float *scale);
+
+/* Full dispatch. fp8 == 0: recv_x is bf16 [M,H]; fp8 != 0: recv_x is e4m3
+ * [M,H] and recv_scale fp32 [M,H/128]. recv_src i32 [M], recv_w fp32 [M]. */
+void orc_dispatch(const uint16_t *x, const int32_t *dst_row, const float *topk_w,
+                  int64_t N, int H, int K, int fp8,
+                  void *recv_x, float *recv_scale, int32_t *recv_src, float *recv_w);
+
+/* Identity expert for FP8 receive rows: y = bf16(e4m3_decode(q) * scale). */
+void orc_identity_expert_fp8(const uint8_t *q, const float *scale, int64_t M, int H,
+                             uint16_t *y);
+
+/* ---- combine ----------------------------------------------------------- */
+/* out[g] = bf16( sum_k w[g,k] * y[dst_row[g,k]] ), k ascending, fp32 fma.
+ * y_scale == NULL: y is bf16 [M,H]. Otherwise y is e4m3 [M,H] and each value is
+ * dequantised as e4m3_decode(q) * y_scale[row, h/128] before the fma.
+ * Computes the listed tokens only (tokens == NULL: all N in order); out has one
+ * row per computed token. */
+void orc_combine(const void *y, const float *y_scale, const int32_t *dst_row,
+                 const float *topk_w, int64_t N, int H, int K,
+                 const int64_t *tokens, int64_t n_tokens, uint16_t *out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
