@@ -1,0 +1,304 @@
+"""Bench: MoE expert-parallel routing + layout -> dispatch -> combine on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--config prefill] [--impl ours|reference]
+
+A step is one pass of the whole path over one batch: ep_get_layout (routing +
+layout), ep_dispatch and ep_combine, with an identity expert in between.
+The default workload is the prefill shape:
+- 8 emulated ranks x 4096 tokens, H = 7168;
+- 256 experts, group-limited top-8 (8 groups, keep 4);
+- bf16 dispatch.
+Its inputs (x 470 MB, receive rows 3.76 GB) exceed the 126 MB L2, so steps
+run back to back with no flush. For workloads that fit in L2 (--config tiny
+or decode) a 512 MB buffer is written between steps.
+
+value = the step's algorithmic HBM bytes (layout + dispatch + combine) / step
+time, in GB/s, summed over ranks. N > 1 runs N independent replicas (weak
+scaling), with no data-path collective. The timed region is K steps
+bracketed by a barrier and a device sync, and the time is the max over
+ranks. Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (the only reference this path has)
+on rank 0, on a bounded sample of the same workload. Other ranks exit 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+import time
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+from combine_top_group_b200 import metrics  # noqa: E402
+from combine_top_group_b200 import workloads as wl  # noqa: E402
+
+ORACLE_SAMPLE_T = 128  # tokens per rank in the CPU oracle's bounded sample
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="prefill", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="tokens per rank (0 = the workload's own); smaller cases for profiling")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--num-sms", type=int, default=0, help="SM cap for dispatch (0 = all)")
+    ap.add_argument("--fused-fp8-combine", action="store_true",
+                    help="FP8 workloads: combine straight from the e4m3 rows (fused dequant)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+def workload_desc(w: wl.Workload) -> dict:
+    return {"workload": w.describe(), "ranks_emulated": w.R, "tokens_per_rank": w.T, "hidden": w.H,
+            "experts": w.E, "topk": w.K, "groups": w.G, "topk_groups": w.KG,
+            "route": wl.ROUTE_NAMES[w.route], "dispatch": "fp8_e4m3" if w.fp8 else "bf16",
+            "mask_frac": w.mask_frac}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (test infrastructure) as the timed baseline
+# ---------------------------------------------------------------------------
+
+def oracle_step_sample(w: wl.Workload, seed: int = 0):
+    """One oracle pass over a bounded sample of the workload: the same shape,
+    with ORACLE_SAMPLE_T tokens per rank. Returns (seconds, algorithmic
+    bytes)."""
+    import oracle  # test infrastructure: only this leg of the bench runs it
+    ws = w.with_tokens(min(w.T, ORACLE_SAMPLE_T))
+    x = wl.make_x(ws, seed)
+    logits = wl.make_logits(ws, seed)
+    t0 = time.perf_counter()
+    res = oracle.run_path(x, logits, ws)
+    dt = time.perf_counter() - t0
+    M = res["M"]
+    nbytes = metrics.layout_bytes(ws) + metrics.dispatch_bytes(ws, M) + metrics.combine_bytes(ws, M)
+    return dt, nbytes, ws
+
+
+def cpu_baseline(w: wl.Workload) -> dict:
+    dt, nbytes, ws = oracle_step_sample(w)
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"one full path (route, layout, dispatch, identity expert, combine) over "
+                      f"{ws.R}x{ws.T} tokens of the same shape; {dt:.2f} s single-threaded C"}
+
+
+def run_reference(args, w: wl.Workload, rank: int, world: int):
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_step_sample(w)
+    tot_t, tot_b = 0.0, 0
+    for _ in range(args.steps):
+        dt, nb, ws = oracle_step_sample(w)
+        tot_t += dt
+        tot_b += nb
+    value = tot_b / tot_t / 1e9
+    line = {
+        "impl": "reference", "metric": "routing+layout+dispatch+combine achieved HBM GB/s (algorithmic bytes / time)",
+        "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if not w.fp8 else "fp8_e4m3", "data": "synthetic",
+        "config": workload_desc(w),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: the whole path over {ws.R}x{ws.T} tokens of the same shape"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU path
+# ---------------------------------------------------------------------------
+
+def run_ours(args, w: wl.Workload, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    from combine_top_group_b200 import ep, runner
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    pipe = runner.Pipeline(w, seed=rank, device=dev, num_sms=args.num_sms)
+    fused = w.fp8 and args.fused_fp8_combine
+    # identity expert for FP8 rows: y depends only on the (fixed) inputs, so it
+    # is made once here, outside the timed region
+    pipe.step(fused=True)
+    if w.fp8 and not fused:
+        pipe.identity_expert()
+    if pipe.check_errors() != 0:
+        raise RuntimeError("device error word set during set-up")
+    M = pipe.num_rows()
+    bytes_layout = metrics.layout_bytes(w)
+    bytes_dispatch = metrics.dispatch_bytes(w, M)
+    bytes_combine = metrics.combine_bytes(w, M, fused_fp8=fused)
+    bytes_step = bytes_layout + bytes_dispatch + bytes_combine
+
+    fits_l2 = (w.N * w.H * 2 + M * w.H * (1 if w.fp8 else 2)) < 2 * 126 * 2 ** 20
+    flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev) if fits_l2 else None
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.fill_(1)
+        pipe.step(fused=fused)
+    torch.cuda.synchronize(dev)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    props = torch.cuda.get_device_properties(dev)
+    bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+    clk = metrics.ClockSampler(pci_bus_id=bus).start()
+    barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        if flush is not None:
+            flush.fill_(1)
+        e = ev[i]
+        e[0].record(stream)
+        pipe.layout(stream)
+        e[1].record(stream)
+        pipe.dispatch(stream)
+        e[2].record(stream)
+        pipe.combine(fused=fused, stream=stream)
+        e[3].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = clk.stop()
+    if pipe.check_errors() != 0:
+        raise RuntimeError("device error word set during the timed steps")
+
+    t_layout = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+    t_disp = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    t_comb = sum(e[2].elapsed_time(e[3]) for e in ev) / 1e3
+    t_total = t_layout + t_disp + t_comb
+    if world > 1:
+        t = torch.tensor([t_total, t_layout, t_disp, t_comb], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_total, t_layout, t_disp, t_comb = t.tolist()
+    K = args.steps
+    value = world * bytes_step * K / t_total / 1e9
+
+    # end to end through the C ABI from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps=min(K, 5), world=world)
+
+    peak, peak_src = metrics.hbm_peak()
+    d_avg, c_avg = t_disp / K, t_comb / K
+    kern, k_bytes, k_time = (("dispatch", bytes_dispatch, d_avg) if d_avg >= c_avg
+                             else ("combine", bytes_combine, c_avg))
+    achieved = k_bytes / k_time / 1e9
+    traffic = metrics.stored_traffic(kern, w.name)
+    out = {
+        "metric": "routing+layout+dispatch+combine achieved HBM GB/s (algorithmic bytes / device time)",
+        "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": t_total / K * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8_e4m3" if w.fp8 else "bf16", "data": "synthetic",
+        "config": {**workload_desc(w), "parallelism": f"replicas{world}" if world > 1 else "1gpu",
+                   "num_sms": args.num_sms or "all", "combine_input": "fp8_fused" if fused else "bf16",
+                   "l2": "512 MB flush between steps" if flush is not None else
+                         "inputs larger than L2 (no flush)"},
+        "layout_us": t_layout / K * 1e6, "dispatch_us": d_avg * 1e6, "combine_us": c_avg * 1e6,
+        "dispatch_plus_combine_us": (d_avg + c_avg) * 1e6,
+        "dispatch_gbs": bytes_dispatch / d_avg / 1e9, "combine_gbs": bytes_combine / c_avg / 1e9,
+        "dispatch_frac_of_peak": bytes_dispatch / d_avg / 1e9 / peak,
+        "combine_frac_of_peak": bytes_combine / c_avg / 1e9 / peak,
+        "receive_rows": M,
+        "algorithmic_bytes": {"layout": bytes_layout, "dispatch": bytes_dispatch, "combine": bytes_combine},
+        "roofline": {"bound": "hbm", "kernel": kern, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": f"{peak_src} (hbm_gbs copy)"},
+        "gpu_launches": 5 * K,
+        "clocks": clocks,
+    }
+    why = metrics.clocks_rejected(clocks)
+    if why:
+        out["clocks_rejected"] = why
+    if e2e is not None:
+        out["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps, world):
+    """Same metric, through the C ABI, with the step's inputs copied in from
+    pinned host memory and its result copied back, inside the timed region."""
+    import torch
+    import torch.distributed as dist
+    x_h = pipe.x.cpu().pin_memory()
+    l_h = pipe.logits.cpu().pin_memory()
+    out_h = torch.empty(pipe.out.shape, dtype=pipe.out.dtype).pin_memory()
+    h2d = x_h.numel() * x_h.element_size() + l_h.numel() * l_h.element_size()
+    d2h = out_h.numel() * out_h.element_size()
+
+    def one():
+        pipe.x.copy_(x_h, non_blocking=True)
+        pipe.logits.copy_(l_h, non_blocking=True)
+        pipe.layout(stream)
+        pipe.dispatch(stream)
+        if w.fp8 and not fused:
+            pipe.combine(fused=False, stream=stream)  # y made once from the same inputs
+        else:
+            pipe.combine(fused=fused, stream=stream)
+        out_h.copy_(pipe.out, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        one()
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    t = s.elapsed_time(e) / 1e3
+    if world > 1:
+        tt = torch.tensor([t], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t = tt.item()
+    return {"value": world * bytes_step * steps / t / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": t / steps * 1e3}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = wl.WORKLOADS[args.config]
+    if args.tokens:
+        w = w.with_tokens(args.tokens)
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,325 @@
+// C ABI of libep (declared in include/ep.h): argument validation, worst-case
+// buffer sizing and partitioning, and the launches. Host code only. Every
+// device computation happens in layout.cu, dispatch.cu and combine.cu.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <new>
+
+#include "ep.h"
+#include "internal.h"
+
+namespace {
+
+thread_local char g_msg[256] = "";
+
+ep_status_t fail(ep_status_t st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+ep_status_t cuda_fail(cudaError_t e, const char* what) {
+    return fail(EP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+ep_status_t ok() {
+    g_msg[0] = '\0';
+    return EP_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+ep_status_t validate(const ep_config_t* c) {
+    if (!c) return fail(EP_ERR_INVALID, "config is NULL");
+    if (c->num_ranks < 1 || c->num_ranks > 32) return fail(EP_ERR_UNSUPPORTED, "num_ranks must be in [1, 32]");
+    if (c->max_tokens_per_rank < 1) return fail(EP_ERR_INVALID, "max_tokens_per_rank must be >= 1");
+    if (c->hidden < 128 || c->hidden % 128 != 0) return fail(EP_ERR_UNSUPPORTED, "hidden must be a positive multiple of 128");
+    if (c->hidden > 65536) return fail(EP_ERR_UNSUPPORTED, "hidden must be <= 65536");
+    if (c->num_experts < 1 || c->num_experts > 1024) return fail(EP_ERR_UNSUPPORTED, "num_experts must be in [1, 1024]");
+    if (c->num_experts % c->num_ranks != 0) return fail(EP_ERR_INVALID, "num_experts must be a multiple of num_ranks");
+    if (c->topk < 1 || c->topk > 32 || c->topk > c->num_experts)
+        return fail(EP_ERR_INVALID, "topk must be in [1, min(32, num_experts)]");
+    if (c->num_groups < 1 || c->num_groups > 32 || c->num_experts % c->num_groups != 0)
+        return fail(EP_ERR_INVALID, "num_groups must be in [1, 32] and divide num_experts");
+    if (c->topk_groups < 1 || c->topk_groups > c->num_groups)
+        return fail(EP_ERR_INVALID, "topk_groups must be in [1, num_groups]");
+    if (c->num_groups > 1) {
+        const int gs = c->num_experts / c->num_groups;
+        if (gs < 2) return fail(EP_ERR_INVALID, "group-limited gating needs >= 2 experts per group");
+        if (c->topk > c->topk_groups * gs) return fail(EP_ERR_INVALID, "topk exceeds the experts of the kept groups");
+    }
+    if (c->num_sms < 0) return fail(EP_ERR_INVALID, "num_sms must be >= 0");
+    if (c->flags & ~EP_FLAG_FP8) return fail(EP_ERR_INVALID, "unknown flag bits");
+    const int64_t m_max = (int64_t)c->num_ranks * c->max_tokens_per_rank * c->topk;
+    if (m_max >= (int64_t)1 << 31) return fail(EP_ERR_UNSUPPORTED, "R*T_max*K must be < 2^31 (int32 row ids)");
+    return EP_OK;
+}
+
+struct Plan {
+    size_t off[20];
+    size_t total;
+};
+
+// Region order inside the workspace; every region is 256-byte aligned.
+enum {
+    R_TOPK_IDX, R_TOPK_W, R_ITR, R_NTPR, R_CNT, R_NTPE, R_EOFF, R_ROFF, R_SOFF, R_DST,
+    R_CHUNK, R_PREF, R_ERR, R_RECV_X, R_RECV_SCALE, R_RECV_SRC, R_RECV_W, R_COUNT
+};
+
+Plan plan_of(const ep_config_t* c, int64_t* n_max, int64_t* m_max, int64_t* nc_max) {
+    const int64_t R = c->num_ranks, T = c->max_tokens_per_rank, H = c->hidden, E = c->num_experts,
+                  K = c->topk;
+    const int64_t N = R * T, M = N * K;
+    const int64_t nc = R * ((T + 31) / 32);  // most chunks: 32 tokens each
+    const bool fp8 = (c->flags & EP_FLAG_FP8) != 0;
+    size_t sz[R_COUNT];
+    sz[R_TOPK_IDX] = 4 * N * K;
+    sz[R_TOPK_W] = 4 * N * K;
+    sz[R_ITR] = N * R;
+    sz[R_NTPR] = 4 * R * R;
+    sz[R_CNT] = 4 * R * E;
+    sz[R_NTPE] = 4 * E;
+    sz[R_EOFF] = 4 * (E + 1);
+    sz[R_ROFF] = 4 * (R + 1);
+    sz[R_SOFF] = 4 * E * R;
+    sz[R_DST] = 4 * N * K;
+    sz[R_CHUNK] = 4 * nc * (E + R);
+    sz[R_PREF] = 4 * (E + R) * (R + 1);
+    sz[R_ERR] = 16;
+    sz[R_RECV_X] = (size_t)M * H * (fp8 ? 1 : 2);
+    sz[R_RECV_SCALE] = fp8 ? (size_t)M * (H / 128) * 4 : 0;
+    sz[R_RECV_SRC] = 4 * M;
+    sz[R_RECV_W] = 4 * M;
+    Plan p{};
+    size_t cur = 0;
+    for (int i = 0; i < R_COUNT; ++i) {
+        p.off[i] = cur;
+        cur += align256(sz[i]);
+    }
+    p.total = cur;
+    *n_max = N;
+    *m_max = M;
+    *nc_max = nc;
+    return p;
+}
+
+ep_status_t check_buf(const ep_buffer_t* b) {
+    if (!b) return fail(EP_ERR_INVALID, "buffer is NULL");
+    return EP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ep_abi_version(void) { return EP_ABI_VERSION; }
+
+const char* ep_status_string(ep_status_t s) {
+    switch (s) {
+        case EP_OK: return "EP_OK";
+        case EP_ERR_INVALID: return "EP_ERR_INVALID";
+        case EP_ERR_CAPACITY: return "EP_ERR_CAPACITY";
+        case EP_ERR_OOM: return "EP_ERR_OOM";
+        case EP_ERR_CUDA: return "EP_ERR_CUDA";
+        case EP_ERR_UNSUPPORTED: return "EP_ERR_UNSUPPORTED";
+        case EP_ERR_DEVICE: return "EP_ERR_DEVICE";
+    }
+    return "EP_ERR_UNKNOWN";
+}
+
+const char* ep_last_error_message(void) { return g_msg; }
+
+ep_config_t ep_default_config(int num_ranks, int max_tokens_per_rank, int hidden, int num_experts, int topk) {
+    ep_config_t c;
+    memset(&c, 0, sizeof c);
+    c.num_ranks = num_ranks;
+    c.max_tokens_per_rank = max_tokens_per_rank;
+    c.hidden = hidden;
+    c.num_experts = num_experts;
+    c.topk = topk;
+    c.num_groups = 1;
+    c.topk_groups = 1;
+    c.num_sms = 0;
+    c.flags = 0;
+    return c;
+}
+
+ep_status_t ep_buffer_workspace_bytes(const ep_config_t* cfg, size_t* bytes) {
+    ep_status_t st = validate(cfg);
+    if (st != EP_OK) return st;
+    if (!bytes) return fail(EP_ERR_INVALID, "bytes is NULL");
+    int64_t n, m, nc;
+    *bytes = plan_of(cfg, &n, &m, &nc).total;
+    return ok();
+}
+
+ep_status_t ep_buffer_create(const ep_config_t* cfg, void* d_workspace, size_t bytes, ep_buffer_t** out) {
+    ep_status_t st = validate(cfg);
+    if (st != EP_OK) return st;
+    if (!out) return fail(EP_ERR_INVALID, "out is NULL");
+    *out = nullptr;
+    if (!d_workspace) return fail(EP_ERR_INVALID, "workspace is NULL");
+    if ((uintptr_t)d_workspace % 256 != 0) return fail(EP_ERR_INVALID, "workspace must be 256-byte aligned");
+    int64_t n, m, nc;
+    const Plan p = plan_of(cfg, &n, &m, &nc);
+    if (bytes < p.total)
+        return fail(EP_ERR_OOM, "workspace has %zu bytes, the worst case needs %zu", bytes, p.total);
+    cudaPointerAttributes attr;
+    cudaError_t e = cudaPointerGetAttributes(&attr, d_workspace);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaPointerGetAttributes");
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+        return fail(EP_ERR_INVALID, "workspace is not device memory");
+    int dev = attr.device, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return cuda_fail(e, "cudaDeviceGetAttribute");
+    ep_buffer_t* b = new (std::nothrow) ep_buffer_t();
+    if (!b) return fail(EP_ERR_OOM, "host allocation of the buffer struct failed");
+    uint8_t* w = static_cast<uint8_t*>(d_workspace);
+    b->cfg = *cfg;
+    b->n_max = n;
+    b->m_max = m;
+    b->nc_max = nc;
+    b->device = dev;
+    b->sm_count = sms;
+    b->last_T = -1;
+    b->topk_idx = reinterpret_cast<int32_t*>(w + p.off[R_TOPK_IDX]);
+    b->topk_w = reinterpret_cast<float*>(w + p.off[R_TOPK_W]);
+    b->is_token_in_rank = w + p.off[R_ITR];
+    b->num_tokens_per_rank = reinterpret_cast<int32_t*>(w + p.off[R_NTPR]);
+    b->cnt = reinterpret_cast<int32_t*>(w + p.off[R_CNT]);
+    b->num_tokens_per_expert = reinterpret_cast<int32_t*>(w + p.off[R_NTPE]);
+    b->expert_off = reinterpret_cast<int32_t*>(w + p.off[R_EOFF]);
+    b->rank_off = reinterpret_cast<int32_t*>(w + p.off[R_ROFF]);
+    b->src_off = reinterpret_cast<int32_t*>(w + p.off[R_SOFF]);
+    b->dst_row = reinterpret_cast<int32_t*>(w + p.off[R_DST]);
+    b->chunk = reinterpret_cast<int32_t*>(w + p.off[R_CHUNK]);
+    b->pref = reinterpret_cast<int32_t*>(w + p.off[R_PREF]);
+    b->err = reinterpret_cast<uint32_t*>(w + p.off[R_ERR]);
+    b->recv_x = w + p.off[R_RECV_X];
+    b->recv_scale = (cfg->flags & EP_FLAG_FP8) ? reinterpret_cast<float*>(w + p.off[R_RECV_SCALE]) : nullptr;
+    b->recv_src = reinterpret_cast<int32_t*>(w + p.off[R_RECV_SRC]);
+    b->recv_w = reinterpret_cast<float*>(w + p.off[R_RECV_W]);
+    int prev = 0;
+    cudaGetDevice(&prev);
+    if (prev != dev) cudaSetDevice(dev);
+    // legacy-stream memset, then wait for it: callers' streams may be
+    // non-blocking and would not be ordered after it otherwise
+    e = cudaMemset(b->err, 0, 16);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(nullptr);
+    if (prev != dev) cudaSetDevice(prev);
+    if (e != cudaSuccess) {
+        delete b;
+        return cuda_fail(e, "cudaMemset(error word)");
+    }
+    *out = b;
+    return ok();
+}
+
+ep_status_t ep_buffer_destroy(ep_buffer_t* buf) {
+    delete buf;
+    return ok();
+}
+
+ep_status_t ep_buffer_layout(const ep_buffer_t* b, ep_layout_t* out) {
+    if (ep_status_t st = check_buf(b)) return st;
+    if (!out) return fail(EP_ERR_INVALID, "out is NULL");
+    out->topk_idx = b->topk_idx;
+    out->topk_w = b->topk_w;
+    out->is_token_in_rank = b->is_token_in_rank;
+    out->num_tokens_per_rank = b->num_tokens_per_rank;
+    out->cnt_src_expert = b->cnt;
+    out->num_tokens_per_expert = b->num_tokens_per_expert;
+    out->expert_off = b->expert_off;
+    out->rank_off = b->rank_off;
+    out->src_off = b->src_off;
+    out->dst_row = b->dst_row;
+    return ok();
+}
+
+ep_status_t ep_buffer_recv(const ep_buffer_t* b, void** recv_x, float** recv_scale, int32_t** recv_src,
+                           float** recv_w, int64_t* max_rows) {
+    if (ep_status_t st = check_buf(b)) return st;
+    if (recv_x) *recv_x = b->recv_x;
+    if (recv_scale) *recv_scale = b->recv_scale;
+    if (recv_src) *recv_src = b->recv_src;
+    if (recv_w) *recv_w = b->recv_w;
+    if (max_rows) *max_rows = b->m_max;
+    return ok();
+}
+
+ep_status_t ep_get_layout(ep_buffer_t* b, int T, const float* d_logits, const int32_t* d_topk_idx,
+                          const float* d_topk_w, int route, uint64_t mask_seed, float mask_frac, void* stream) {
+    if (ep_status_t st = check_buf(b)) return st;
+    if (T < 0) return fail(EP_ERR_INVALID, "T must be >= 0");
+    if (T > b->cfg.max_tokens_per_rank)
+        return fail(EP_ERR_CAPACITY, "T=%d exceeds max_tokens_per_rank=%d", T, b->cfg.max_tokens_per_rank);
+    const bool have_logits = d_logits != nullptr;
+    const bool have_idx = d_topk_idx != nullptr || d_topk_w != nullptr;
+    if (have_logits == have_idx) return fail(EP_ERR_INVALID, "pass either d_logits or d_topk_idx + d_topk_w");
+    if (have_idx && (!d_topk_idx || !d_topk_w)) return fail(EP_ERR_INVALID, "d_topk_idx and d_topk_w go together");
+    if (have_logits && (route < EP_ROUTE_SOFTMAX || route > EP_ROUTE_GROUP_SIGMOID))
+        return fail(EP_ERR_INVALID, "unknown route %d", route);
+    if (have_logits && route == EP_ROUTE_GROUP_SIGMOID && b->cfg.num_groups > 1 &&
+        b->cfg.topk > b->cfg.topk_groups * (b->cfg.num_experts / b->cfg.num_groups))
+        return fail(EP_ERR_INVALID, "topk exceeds the experts of the kept groups");
+    if (!(mask_frac >= 0.0f && mask_frac <= 1.0f)) return fail(EP_ERR_INVALID, "mask_frac must be in [0, 1]");
+    ep::LayoutArgs a{};
+    a.T = T;
+    a.logits = d_logits;
+    a.in_idx = d_topk_idx;
+    a.in_w = d_topk_w;
+    a.route = route;
+    a.mask_seed = mask_seed;
+    double thr = floor((double)mask_frac * 4294967296.0);
+    a.mask_threshold = (uint64_t)thr;
+    cudaError_t e = ep::launch_layout(*b, a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "layout launch");
+    b->last_T = T;
+    return ok();
+}
+
+ep_status_t ep_dispatch(ep_buffer_t* b, int T, const void* d_x, void* stream) {
+    if (ep_status_t st = check_buf(b)) return st;
+    if (T != b->last_T) return fail(EP_ERR_INVALID, "T=%d does not match the last ep_get_layout (T=%d)", T, b->last_T);
+    if (T > 0 && !d_x) return fail(EP_ERR_INVALID, "d_x is NULL");
+    if ((uintptr_t)d_x % 16 != 0) return fail(EP_ERR_INVALID, "d_x must be 16-byte aligned");
+    cudaError_t e = ep::launch_dispatch(*b, T, d_x, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
+    return ok();
+}
+
+ep_status_t ep_combine(ep_buffer_t* b, int T, const void* d_y, const float* d_y_scale, void* d_out, void* stream) {
+    if (ep_status_t st = check_buf(b)) return st;
+    if (T != b->last_T) return fail(EP_ERR_INVALID, "T=%d does not match the last ep_get_layout (T=%d)", T, b->last_T);
+    if (T > 0 && (!d_y || !d_out)) return fail(EP_ERR_INVALID, "d_y and d_out must be non-NULL");
+    if ((uintptr_t)d_y % 16 != 0 || (uintptr_t)d_out % 16 != 0)
+        return fail(EP_ERR_INVALID, "d_y and d_out must be 16-byte aligned");
+    if (d_y_scale && (uintptr_t)d_y_scale % 4 != 0) return fail(EP_ERR_INVALID, "d_y_scale must be 4-byte aligned");
+    cudaError_t e = ep::launch_combine(*b, T, d_y, d_y_scale, d_out, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    return ok();
+}
+
+ep_status_t ep_check_errors(ep_buffer_t* b, uint32_t* word, int clear, void* stream) {
+    if (ep_status_t st = check_buf(b)) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, b->err, sizeof v, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess && clear) {
+        e = cudaMemsetAsync(b->err, 0, sizeof v, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "ep_check_errors");
+    if (word) *word = v;
+    if (v) return fail(EP_ERR_DEVICE, "device error word 0x%x", v);
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,62 @@
+// Host-side internals of libep: the buffer struct and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ep.h"
+
+struct ep_buffer {
+    ep_config_t cfg;
+    int64_t n_max;   // R * T_max tokens
+    int64_t m_max;   // R * T_max * K receive rows
+    int64_t nc_max;  // chunk capacity of the layout scratch
+    int device;
+    int sm_count;
+    int last_T;      // T of the last ep_get_layout (-1 = none)
+
+    // layout arrays (device)
+    int32_t* topk_idx;
+    float* topk_w;
+    uint8_t* is_token_in_rank;
+    int32_t* num_tokens_per_rank;
+    int32_t* cnt;
+    int32_t* num_tokens_per_expert;
+    int32_t* expert_off;
+    int32_t* rank_off;
+    int32_t* src_off;
+    int32_t* dst_row;
+    // layout scratch (device): per-chunk counts, later their prefix sums,
+    // [nc][E + R]; per-column prefix at each rank's first chunk, [E + R][R + 1]
+    int32_t* chunk;
+    int32_t* pref;
+    uint32_t* err;  // device error word
+    // receive buffers (device)
+    void* recv_x;
+    float* recv_scale;
+    int32_t* recv_src;
+    float* recv_w;
+};
+
+namespace ep {
+
+// Tokens per layout chunk for N tokens: 32 * 2^j, smallest with at most 1024
+// chunks (for N up to 32K tokens that is 32).
+int layout_chunk_tokens(int64_t n_tokens);
+
+struct LayoutArgs {
+    int T;
+    const float* logits;
+    const int32_t* in_idx;
+    const float* in_w;
+    int route;
+    uint64_t mask_seed;
+    uint64_t mask_threshold;  // in [0, 2^32]
+};
+
+cudaError_t launch_layout(const ep_buffer& b, const LayoutArgs& a, cudaStream_t stream);
+cudaError_t launch_dispatch(const ep_buffer& b, int T, const void* x, cudaStream_t stream);
+cudaError_t launch_combine(const ep_buffer& b, int T, const void* y, const float* y_scale, void* out,
+                           cudaStream_t stream);
+
+}  // namespace ep

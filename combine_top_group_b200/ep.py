@@ -1,0 +1,233 @@
+"""Thin ctypes binding of libep.so (C ABI in include/ep.h).
+
+The functions keep the C names and only marshal arguments. torch tensors
+become device pointers, the current torch stream becomes `stream`, and a
+non-OK status raises EpError. Every step of the path runs in the library's
+CUDA kernels. Importing this module loads the library and raises
+ImportError if it is missing: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libep.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m combine_top_group_b200.build` "
+        "(nvcc, sm_100a). The library has no CPU fallback.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+EP_OK, EP_ERR_INVALID, EP_ERR_CAPACITY, EP_ERR_OOM, EP_ERR_CUDA, EP_ERR_UNSUPPORTED, EP_ERR_DEVICE = range(7)
+EP_DEVERR_EXPERT_ID, EP_DEVERR_ROW_BOUNDS, EP_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
+EP_FLAG_FP8 = 0x1
+EP_ROUTE_SOFTMAX, EP_ROUTE_SOFTMAX_RENORM, EP_ROUTE_GROUP_SIGMOID = 0, 1, 2
+
+
+class EpConfig(ctypes.Structure):
+    _fields_ = [("num_ranks", ctypes.c_int32), ("max_tokens_per_rank", ctypes.c_int32),
+                ("hidden", ctypes.c_int32), ("num_experts", ctypes.c_int32), ("topk", ctypes.c_int32),
+                ("num_groups", ctypes.c_int32), ("topk_groups", ctypes.c_int32), ("num_sms", ctypes.c_int32),
+                ("flags", ctypes.c_uint32)]
+
+
+class EpLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "topk_idx", "topk_w", "is_token_in_rank", "num_tokens_per_rank", "cnt_src_expert",
+        "num_tokens_per_expert", "expert_off", "rank_off", "src_off", "dst_row")]
+
+
+_P = ctypes.c_void_p
+_st = ctypes.c_int
+_lib.ep_abi_version.restype = ctypes.c_int
+_lib.ep_status_string.argtypes = [_st]
+_lib.ep_status_string.restype = ctypes.c_char_p
+_lib.ep_last_error_message.restype = ctypes.c_char_p
+_lib.ep_default_config.argtypes = [ctypes.c_int] * 5
+_lib.ep_default_config.restype = EpConfig
+_lib.ep_buffer_workspace_bytes.argtypes = [ctypes.POINTER(EpConfig), ctypes.POINTER(ctypes.c_size_t)]
+_lib.ep_buffer_workspace_bytes.restype = _st
+_lib.ep_buffer_create.argtypes = [ctypes.POINTER(EpConfig), _P, ctypes.c_size_t, ctypes.POINTER(_P)]
+_lib.ep_buffer_create.restype = _st
+_lib.ep_buffer_destroy.argtypes = [_P]
+_lib.ep_buffer_destroy.restype = _st
+_lib.ep_buffer_layout.argtypes = [_P, ctypes.POINTER(EpLayout)]
+_lib.ep_buffer_layout.restype = _st
+_lib.ep_buffer_recv.argtypes = [_P, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P),
+                                ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_int64)]
+_lib.ep_buffer_recv.restype = _st
+_lib.ep_get_layout.argtypes = [_P, ctypes.c_int, _P, _P, _P, ctypes.c_int, ctypes.c_uint64, ctypes.c_float, _P]
+_lib.ep_get_layout.restype = _st
+_lib.ep_dispatch.argtypes = [_P, ctypes.c_int, _P, _P]
+_lib.ep_dispatch.restype = _st
+_lib.ep_combine.argtypes = [_P, ctypes.c_int, _P, _P, _P, _P]
+_lib.ep_combine.restype = _st
+_lib.ep_check_errors.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, _P]
+_lib.ep_check_errors.restype = _st
+
+EXPORTED = ("ep_abi_version", "ep_status_string", "ep_last_error_message", "ep_default_config",
+            "ep_buffer_workspace_bytes", "ep_buffer_create", "ep_buffer_destroy", "ep_buffer_layout",
+            "ep_buffer_recv", "ep_get_layout", "ep_dispatch", "ep_combine", "ep_check_errors")
+
+
+class EpError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.ep_last_error_message().decode()
+        super().__init__(f"{where}: {_lib.ep_status_string(status).decode()} ({msg})")
+
+
+def _check(status: int, where: str) -> None:
+    if status != EP_OK:
+        raise EpError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+class EpBuffer:
+    """Handle plus the torch-owned workspace it lives in."""
+
+    def __init__(self, handle: int, cfg: EpConfig, workspace: torch.Tensor):
+        self.handle = handle
+        self.cfg = cfg
+        self.workspace = workspace
+
+    @property
+    def fp8(self) -> bool:
+        return bool(self.cfg.flags & EP_FLAG_FP8)
+
+    def _view(self, ptr: int, dtype: torch.dtype, shape) -> torch.Tensor:
+        off = ptr - self.workspace.data_ptr()
+        n = 1
+        for s in shape:
+            n *= s
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        assert 0 <= off and off + nbytes <= self.workspace.numel()
+        return self.workspace.narrow(0, off, nbytes).view(dtype).view(*shape)
+
+    def __del__(self):
+        h, self.handle = getattr(self, "handle", None), None
+        if h:
+            _lib.ep_buffer_destroy(h)
+
+
+def ep_abi_version() -> int:
+    return _lib.ep_abi_version()
+
+
+def ep_status_string(status: int) -> str:
+    return _lib.ep_status_string(status).decode()
+
+
+def ep_last_error_message() -> str:
+    return _lib.ep_last_error_message().decode()
+
+
+def ep_default_config(num_ranks: int, max_tokens_per_rank: int, hidden: int, num_experts: int,
+                      topk: int) -> EpConfig:
+    return _lib.ep_default_config(num_ranks, max_tokens_per_rank, hidden, num_experts, topk)
+
+
+def ep_buffer_workspace_bytes(cfg: EpConfig) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.ep_buffer_workspace_bytes(ctypes.byref(cfg), ctypes.byref(n)), "ep_buffer_workspace_bytes")
+    return n.value
+
+
+def ep_buffer_create(cfg: EpConfig, workspace: torch.Tensor | None = None, device=None) -> EpBuffer:
+    """Wraps `workspace` (a uint8 CUDA tensor of at least
+    ep_buffer_workspace_bytes(cfg) bytes), allocating it first if None."""
+    nbytes = ep_buffer_workspace_bytes(cfg)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
+    h = _P()
+    _check(_lib.ep_buffer_create(ctypes.byref(cfg), workspace.data_ptr(), workspace.numel(), ctypes.byref(h)),
+           "ep_buffer_create")
+    return EpBuffer(h.value, cfg, workspace)
+
+
+def ep_buffer_destroy(buf: EpBuffer) -> None:
+    h, buf.handle = buf.handle, None
+    if h:
+        _check(_lib.ep_buffer_destroy(h), "ep_buffer_destroy")
+
+
+def ep_buffer_layout(buf: EpBuffer, T: int) -> dict:
+    """torch views of the layout arrays for T tokens per rank."""
+    lay = EpLayout()
+    _check(_lib.ep_buffer_layout(buf.handle, ctypes.byref(lay)), "ep_buffer_layout")
+    c = buf.cfg
+    R, E, K, N = c.num_ranks, c.num_experts, c.topk, c.num_ranks * T
+    return dict(
+        topk_idx=buf._view(lay.topk_idx, torch.int32, (N, K)),
+        topk_w=buf._view(lay.topk_w, torch.float32, (N, K)),
+        is_token_in_rank=buf._view(lay.is_token_in_rank, torch.uint8, (N, R)),
+        num_tokens_per_rank=buf._view(lay.num_tokens_per_rank, torch.int32, (R, R)),
+        cnt=buf._view(lay.cnt_src_expert, torch.int32, (R, E)),
+        num_tokens_per_expert=buf._view(lay.num_tokens_per_expert, torch.int32, (E,)),
+        expert_off=buf._view(lay.expert_off, torch.int32, (E + 1,)),
+        rank_off=buf._view(lay.rank_off, torch.int32, (R + 1,)),
+        src_off=buf._view(lay.src_off, torch.int32, (E, R)),
+        dst_row=buf._view(lay.dst_row, torch.int32, (N, K)),
+    )
+
+
+def ep_buffer_recv(buf: EpBuffer) -> dict:
+    """torch views of the receive buffers (M_max rows)."""
+    px, ps, pr, pw = _P(), _P(), _P(), _P()
+    m = ctypes.c_int64(0)
+    _check(_lib.ep_buffer_recv(buf.handle, ctypes.byref(px), ctypes.byref(ps), ctypes.byref(pr),
+                               ctypes.byref(pw), ctypes.byref(m)), "ep_buffer_recv")
+    H, M = buf.cfg.hidden, m.value
+    out = dict(max_rows=M,
+               recv_src=buf._view(pr.value, torch.int32, (M,)),
+               recv_w=buf._view(pw.value, torch.float32, (M,)))
+    if buf.fp8:
+        out["recv_x"] = buf._view(px.value, torch.uint8, (M, H))
+        out["recv_scale"] = buf._view(ps.value, torch.float32, (M, H // 128))
+    else:
+        out["recv_x"] = buf._view(px.value, torch.bfloat16, (M, H))
+        out["recv_scale"] = None
+    return out
+
+
+def ep_get_layout(buf: EpBuffer, T: int, logits=None, topk_idx=None, topk_w=None, route: int = 0,
+                  mask_seed: int = 0, mask_frac: float = 0.0, stream=None) -> None:
+    _check(_lib.ep_get_layout(buf.handle, T, _ptr(logits), _ptr(topk_idx), _ptr(topk_w), route,
+                              mask_seed & 0xFFFF_FFFF_FFFF_FFFF, mask_frac, _stream(stream)), "ep_get_layout")
+
+
+def ep_dispatch(buf: EpBuffer, T: int, x, stream=None) -> None:
+    _check(_lib.ep_dispatch(buf.handle, T, _ptr(x), _stream(stream)), "ep_dispatch")
+
+
+def ep_combine(buf: EpBuffer, T: int, y, y_scale, out, stream=None) -> None:
+    _check(_lib.ep_combine(buf.handle, T, _ptr(y), _ptr(y_scale), _ptr(out), _stream(stream)), "ep_combine")
+
+
+def ep_check_errors(buf: EpBuffer, clear: bool = True, stream=None) -> int:
+    """Synchronises the stream and returns the device error word (0 = clean)."""
+    w = ctypes.c_uint32(0)
+    st = _lib.ep_check_errors(buf.handle, ctypes.byref(w), 1 if clear else 0, _stream(stream))
+    if st not in (EP_OK, EP_ERR_DEVICE):
+        _check(st, "ep_check_errors")
+    return w.value

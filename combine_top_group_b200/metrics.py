@@ -1,0 +1,233 @@
+"""Host-side measurement helpers: algorithmic bytes per call, nvidia-smi clock
+sampling, peaks and ncu traffic lookup. Pure Python, with no GPU work."""
+from __future__ import annotations
+
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+
+from . import workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
+
+FALLBACK_HBM_GBS = 6650.0  # earlier measurement on this machine, used only without MEASURED_PEAKS.json
+
+
+# ---- algorithmic bytes -------------------------------------------------------
+# What the method itself must move, per call. Implementation-only traffic is
+# left out: the layout's per-chunk scratch and re-reads, and L2 misses.
+
+def layout_bytes(w: wl.Workload, N: int | None = None) -> int:
+    """Reads logits N*E*4. Writes topk_idx + topk_w + dst_row (N*K*12) and
+    is_token_in_rank (N*R)."""
+    N = w.N if N is None else N
+    return N * w.E * 4 + N * w.K * 12 + N * w.R
+
+
+def dispatch_bytes(w: wl.Workload, M: int, N: int | None = None) -> int:
+    """Reads each token once (N*H*2) and its dst_row + topk_w (N*K*8).
+    Writes M rows of H*b bytes (b = 1 FP8, 2 bf16), the FP8 scales
+    (M*H/128*4) and recv_src + recv_w (M*8)."""
+    N = w.N if N is None else N
+    b = 1 if w.fp8 else 2
+    scales = M * (w.H // 128) * 4 if w.fp8 else 0
+    return N * w.H * 2 + N * w.K * 8 + M * w.H * b + scales + M * 8
+
+
+def combine_bytes(w: wl.Workload, M: int, fused_fp8: bool = False, N: int | None = None) -> int:
+    """Reads the M expert-output rows (bf16: M*H*2; fused FP8: M*H + scales)
+    and dst_row + topk_w (N*K*8). Writes N*H*2."""
+    N = w.N if N is None else N
+    y = M * w.H + M * (w.H // 128) * 4 if fused_fp8 else M * w.H * 2
+    return y + N * w.K * 8 + N * w.H * 2
+
+
+# ---- peaks -------------------------------------------------------------------
+
+def hbm_peak() -> tuple[float, str]:
+    """(GB/s, source): the measured copy bandwidth, else the fallback."""
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---- ncu traffic (profiles/traffic.json) -------------------------------------
+
+def source_hash() -> str:
+    """Hash of every kernel source; a stored ncu traffic figure is only valid
+    for the sources it was captured from."""
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(kernel: str, workload: str) -> float | None:
+    """dram read+write bytes per launch from the committed ncu summary, or
+    None if absent or captured from other sources."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            data = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = data.get(workload, {}).get(kernel)
+    if not ent or ent.get("source_hash") != source_hash():
+        return None
+    return float(ent["dram_bytes_per_launch"])
+
+
+# ---- clocks ------------------------------------------------------------------
+
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+REASON_COLS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
+class ClockSampler:
+    """Samples the SM clock, power and clock-event (throttle) reasons while
+    the timed region runs. It reads NVML every 5 ms from a thread. Without
+    NVML it runs nvidia-smi every 200 ms. Read-only: no GPU setting is
+    touched."""
+
+    # NVML clock-event reason bits (nvml.h)
+    _BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+             "hw_thermal_slowdown": 0x40}
+
+    def __init__(self, pci_bus_id: str | None = None, interval_s: float = 0.005):
+        self.pci_bus_id = pci_bus_id
+        self.interval = interval_s
+        self.proc = None
+        self.thread = None
+        self.samples = []
+        self._stop = None
+
+    def start(self):
+        try:
+            import threading
+
+            import pynvml
+            pynvml.nvmlInit()
+            h = (pynvml.nvmlDeviceGetHandleByPciBusId(self.pci_bus_id) if self.pci_bus_id
+                 else pynvml.nvmlDeviceGetHandleByIndex(0))
+            self._stop = threading.Event()
+
+            def run():
+                while not self._stop.is_set():
+                    try:
+                        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((sm, mx, pw, rs))
+                    except Exception:  # noqa: BLE001 - sampling is best effort
+                        pass
+                    self._stop.wait(self.interval)
+
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+            return self
+        except Exception:  # noqa: BLE001 - fall back to nvidia-smi
+            self.thread = None
+        cmd = ["nvidia-smi", f"--query-gpu={CLOCK_QUERY}", "--format=csv", "-lms", "200"]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def stop(self) -> dict | None:
+        if self.thread is not None:
+            self._stop.set()
+            self.thread.join(timeout=5)
+            return summarize_nvml(self.samples, self._BITS)
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        return parse_clocks(out)
+
+
+def summarize_nvml(samples, bits) -> dict | None:
+    if not samples:
+        return None
+    sm = [s[0] for s in samples]
+    reasons = sorted({name for s in samples for name, b in bits.items() if s[3] & b})
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(s[1] for s in samples),
+            "reasons": reasons, "samples": len(samples), "power_w_max": max(s[2] for s in samples),
+            "source": "nvml"}
+
+
+def _num(s: str) -> float | None:
+    s = s.strip().split(" ")[0]
+    try:
+        return float(s)
+    except ValueError:
+        return None
+
+
+def parse_clocks(text: str) -> dict | None:
+    rows = list(csv.reader(io.StringIO(text)))
+    if len(rows) < 2:
+        return None
+    head = [h.strip() for h in rows[0]]
+
+    def col(name):
+        for i, h in enumerate(head):
+            if h.startswith(name):
+                return i
+        return None
+
+    i_sm, i_max, i_pw = col("clocks.sm"), col("clocks.max.sm"), col("power.draw")
+    sm, mx, power, reasons = [], [], [], set()
+    for r in rows[1:]:
+        if len(r) != len(head):
+            continue
+        v = _num(r[i_sm]) if i_sm is not None else None
+        if v is not None:
+            sm.append(v)
+        m = _num(r[i_max]) if i_max is not None else None
+        if m is not None:
+            mx.append(m)
+        p = _num(r[i_pw]) if i_pw is not None else None
+        if p is not None:
+            power.append(p)
+        for name in REASON_COLS:
+            i = col(f"clocks_event_reasons.{name}")
+            if i is not None and r[i].strip().lower() == "active":
+                reasons.add(name)
+    if not sm:
+        return None
+    loaded = [s for s, p in zip(sm, power)] if power else sm
+    return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx) if mx else None,
+            "reasons": sorted(reasons), "samples": len(sm),
+            "power_w_max": max(power) if power else None}
+
+
+def clocks_rejected(clk: dict | None) -> str | None:
+    """Why a measurement must be rejected, or None."""
+    if not clk:
+        return None
+    bad = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"} & set(clk.get("reasons", []))
+    if bad:
+        return "throttled: " + ",".join(sorted(bad))
+    if clk.get("sm_max_mhz") and clk["sm_mhz"] < 0.6 * clk["sm_max_mhz"] and not clk.get("reasons"):
+        return "SM clock far below max with no reason (clock lock?)"
+    return None

@@ -1,0 +1,195 @@
+/*
+ * ep.h -- C ABI of libep.so: MoE expert-parallel routing + layout, dispatch
+ * and combine on one B200 (sm_100a). EP ranks are emulated as disjoint
+ * receive partitions of one GPU's memory.
+ *
+ * The operations follow the DeepEP pages:
+ *  - "DeepEP：年度总结中的计算通信重叠摘记" (DeepEP overlap notes):
+ *    - §计算-通信重叠: group-limited gating;
+ *    - §节点内通信: Top-K fused into the communication kernel,
+ *      is_token_in_rank, sending only to target ranks, FP8 at 1 byte per
+ *      element.
+ *  - "DeepEP：面向MoE的高吞吐低延迟GPU通信库" (DeepEP summary):
+ *    - §工程化: dispatch and combine kernels;
+ *    - "如何调优 Buffer.set_num_sms": get_*_config and set_num_sms.
+ *  - the rocSHMEM / DeepEP buffer notes (mlqm.cn), §3.2 "RDMA buffer的问题":
+ *    one communication buffer, allocated once and sized for the worst case.
+ *
+ * Conventions for every function below:
+ *  - Pointers named d_* and every pointer handed out by ep_buffer_* are DEVICE
+ *    pointers. All others are host pointers.
+ *  - The caller owns all device memory: the workspace, the inputs and the
+ *    outputs. The library never allocates or frees device memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is stream-ordered. Only ep_check_errors blocks the host.
+ *  - Argument errors are caught on the host before any launch and returned as
+ *    a status. ep_last_error_message() then gives a one-line reason.
+ *  - Data errors found on the device (an expert id out of range, a row index
+ *    outside the buffer, a bounded wait that gave up) set bits of the
+ *    buffer's device error word. The kernels never trap. ep_check_errors
+ *    reads the word.
+ *  - A buffer is not thread-safe. Use one buffer per stream.
+ */
+#ifndef COMBINE_TOP_GROUP_EP_H
+#define COMBINE_TOP_GROUP_EP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define EP_ABI_VERSION 1
+
+typedef enum {
+    EP_OK = 0,
+    EP_ERR_INVALID = 1,     /* bad argument or shape */
+    EP_ERR_CAPACITY = 2,    /* more tokens than the buffer was sized for */
+    EP_ERR_OOM = 3,         /* workspace smaller than ep_buffer_workspace_bytes */
+    EP_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+    EP_ERR_UNSUPPORTED = 5, /* valid shape this build does not handle */
+    EP_ERR_DEVICE = 6       /* ep_check_errors found device error bits */
+} ep_status_t;
+
+/* Bits of the device error word. */
+#define EP_DEVERR_EXPERT_ID 0x1u  /* an expert id outside [-1, E); the slot was treated as masked */
+#define EP_DEVERR_ROW_BOUNDS 0x2u /* a receive row outside [0, M_max); the copy was skipped */
+#define EP_DEVERR_TIMEOUT 0x4u    /* a bounded wait inside a kernel gave up */
+
+/* ep_config_t.flags */
+#define EP_FLAG_FP8 0x1u /* dispatch casts to FP8 e4m3 with one fp32 scale per 128 channels */
+
+/* Routing rule applied by ep_get_layout to router logits. */
+typedef enum {
+    EP_ROUTE_SOFTMAX = 0,        /* top-K by logit; w = softmax probability */
+    EP_ROUTE_SOFTMAX_RENORM = 1, /* as above, w renormalised over the K chosen */
+    EP_ROUTE_GROUP_SIGMOID = 2   /* group-limited sigmoid gating (DeepEP overlap notes, §计算-通信重叠) */
+} ep_route_t;
+
+/* Buffer configuration. The ep_default_config analogue of DeepEP's
+ * Buffer.get_*_config (DeepEP summary, "如何调优 Buffer.set_num_sms"). */
+typedef struct {
+    int32_t num_ranks;           /* R: emulated EP ranks, 1..32 */
+    int32_t max_tokens_per_rank; /* T_max: capacity per rank, >= 1 */
+    int32_t hidden;              /* H: channels per token, a multiple of 128 */
+    int32_t num_experts;         /* E: a multiple of R, at most 1024; expert e lives on rank e / (E/R) */
+    int32_t topk;                /* K: 1..min(32, E) */
+    int32_t num_groups;          /* G: expert groups for group-limited gating (1 = none); E % G == 0 */
+    int32_t topk_groups;         /* KG: groups kept per token, 1..G */
+    int32_t num_sms;             /* SM cap for the data-movement kernels (0 = all), cf. Buffer.set_num_sms */
+    uint32_t flags;              /* EP_FLAG_* */
+} ep_config_t;
+
+typedef struct ep_buffer ep_buffer_t;
+
+/* Device views of the layout produced by ep_get_layout. N = R*T of the last
+ * call. Row-major arrays, int32 unless stated. */
+typedef struct {
+    int32_t *topk_idx;              /* [N, K]; -1 = masked slot */
+    float *topk_w;                  /* [N, K] fp32; 0 for masked slots */
+    uint8_t *is_token_in_rank;      /* [N, R] 0/1 (DeepEP overlap notes, §节点内通信) */
+    int32_t *num_tokens_per_rank;   /* [R_src, R_dst]: distinct tokens of source s that go to rank r */
+    int32_t *cnt_src_expert;        /* [R_src, E]: slots of source s routed to expert e */
+    int32_t *num_tokens_per_expert; /* [E]: receive rows of expert e */
+    int32_t *expert_off;            /* [E+1]: exclusive prefix sum of num_tokens_per_expert */
+    int32_t *rank_off;              /* [R+1]: rank_off[r] = expert_off[r*E/R] (partition of rank r) */
+    int32_t *src_off;               /* [E, R]: offset of source s inside expert e's rows */
+    int32_t *dst_row;               /* [N, K]: receive row of slot (g,k); -1 if masked */
+} ep_layout_t;
+
+/* Returns EP_ABI_VERSION. */
+int ep_abi_version(void);
+
+/* Static name of a status code. */
+const char *ep_status_string(ep_status_t status);
+
+/* One-line reason for the last non-OK status returned on this host thread
+ * ("" if none). */
+const char *ep_last_error_message(void);
+
+/* Config with no group limit, num_sms = 0, flags = 0. */
+ep_config_t ep_default_config(int num_ranks, int max_tokens_per_rank, int hidden,
+                              int num_experts, int topk);
+
+/* Workspace bytes needed by a buffer with this config. This is the worst
+ * case: M_max = R * T_max * K receive rows in total, which no routing can
+ * exceed (rocSHMEM / DeepEP buffer notes, §3.2: size for the worst case,
+ * allocate once). EP_ERR_INVALID / EP_ERR_UNSUPPORTED for bad configs. */
+ep_status_t ep_buffer_workspace_bytes(const ep_config_t *cfg, size_t *bytes);
+
+/* Wrap a caller-allocated device workspace (256-byte aligned, at least
+ * ep_buffer_workspace_bytes long) in a buffer handle. Zeroes the device error
+ * word with a synchronous cudaMemset. The handle is a small host struct, freed
+ * by ep_buffer_destroy. The workspace must outlive the handle.
+ * Errors: EP_ERR_INVALID (NULL or misaligned), EP_ERR_OOM (too small),
+ * EP_ERR_CUDA. */
+ep_status_t ep_buffer_create(const ep_config_t *cfg, void *d_workspace, size_t bytes,
+                             ep_buffer_t **out);
+
+/* Frees the host struct only. NULL is a no-op. */
+ep_status_t ep_buffer_destroy(ep_buffer_t *buf);
+
+/* Device views of the layout arrays inside the workspace. */
+ep_status_t ep_buffer_layout(const ep_buffer_t *buf, ep_layout_t *out);
+
+/* Device views of the receive buffers, M_max rows each:
+ *  recv_x      bf16 [M_max, H], or e4m3 [M_max, H] with EP_FLAG_FP8;
+ *  recv_scale  fp32 [M_max, H/128] with EP_FLAG_FP8, else NULL;
+ *  recv_src    int32 [M_max]: source token g of each row;
+ *  recv_w      fp32 [M_max]: routing weight of each row.
+ * The rows of rank r are [rank_off[r], rank_off[r+1]). Any out-pointer may be
+ * NULL. Also returns M_max through *max_rows if it is not NULL. */
+ep_status_t ep_buffer_recv(const ep_buffer_t *buf, void **recv_x, float **recv_scale,
+                           int32_t **recv_src, float **recv_w, int64_t *max_rows);
+
+/* Routing + layout for T tokens per rank (N = R*T, token g = s*T + t of
+ * source rank s). Top-K fused with the layout (DeepEP overlap notes,
+ * §节点内通信).
+ * Inputs, exactly one of:
+ *  - d_logits: fp32 [N, E] router logits, routed by `route`;
+ *  - d_topk_idx: int32 [N, K] plus d_topk_w: fp32 [N, K], taken as given.
+ *    Ids outside [-1, E) set EP_DEVERR_EXPERT_ID and become masked slots.
+ * mask_frac > 0 then masks slot (g,k) to -1 (weight 0) when the high 32 bits
+ * of splitmix64(mask_seed ^ (g*K + k)) fall below floor(mask_frac * 2^32).
+ * Writes every ep_layout_t array. Receive rows are ordered by
+ * (expert, source rank, token, slot).
+ * Errors: EP_ERR_CAPACITY if T > T_max; EP_ERR_INVALID for bad pointers, T,
+ * route or mask_frac. */
+ep_status_t ep_get_layout(ep_buffer_t *buf, int T, const float *d_logits,
+                          const int32_t *d_topk_idx, const float *d_topk_w, int route,
+                          uint64_t mask_seed, float mask_frac, void *stream);
+
+/* Dispatch (DeepEP summary, §工程化; only to the target experts, DeepEP
+ * overlap notes, §节点内通信). For every unmasked slot (g,k):
+ *  - recv_x[dst_row[g,k]] = x[g];
+ *  - recv_src[row] = g;
+ *  - recv_w[row] = topk_w[g,k].
+ * With EP_FLAG_FP8 each 128-channel block is cast as:
+ *  - amax = max(max|x|, 1e-4);
+ *  - q = e4m3_rne_satfinite(x * (448/amax));
+ *  - recv_scale = amax/448.
+ * d_x: bf16 [N, H] row-major, 16-byte aligned. T must equal the T of the
+ * last ep_get_layout on this buffer. Errors: EP_ERR_INVALID. */
+ep_status_t ep_dispatch(ep_buffer_t *buf, int T, const void *d_x, void *stream);
+
+/* Combine (DeepEP summary, §工程化):
+ *   out[g] = bf16_rne( sum over k ascending, unmasked, of w[g,k] * y[dst_row[g,k]] )
+ * accumulated in fp32 with one fused multiply-add per slot. d_y_scale == NULL:
+ * d_y is bf16 [rows, H]. Otherwise d_y is e4m3 [rows, H] and is dequantised
+ * in the kernel as e4m3 * d_y_scale[row, h/128] (fp32) before the fma.
+ * rows >= expert_off[E]. d_out: bf16 [N, H]. All pointers 16-byte aligned.
+ * T must equal the T of the last ep_get_layout. A token whose slots are all
+ * masked gets +0. Errors: EP_ERR_INVALID. */
+ep_status_t ep_combine(ep_buffer_t *buf, int T, const void *d_y, const float *d_y_scale,
+                       void *d_out, void *stream);
+
+/* Synchronises `stream` and reads the device error word into *word. clear != 0
+ * then resets it to 0. Returns EP_ERR_DEVICE if any bit was set, EP_OK if
+ * none, EP_ERR_CUDA on a CUDA failure. */
+ep_status_t ep_check_errors(ep_buffer_t *buf, uint32_t *word, int clear, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
