@@ -116,6 +116,10 @@ ep_status_t check_buf(const ep_buffer_t* b) {
 
 }  // namespace
 
+namespace ep {
+void set_last_error(const char* msg) { snprintf(g_msg, sizeof g_msg, "%s", msg); }
+}  // namespace ep
+
 extern "C" {
 
 int ep_abi_version(void) { return EP_ABI_VERSION; }

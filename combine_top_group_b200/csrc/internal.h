@@ -40,6 +40,9 @@ struct ep_buffer {
 
 namespace ep {
 
+// Sets the message ep_last_error_message() returns on this host thread.
+void set_last_error(const char* msg);
+
 // Tokens per layout chunk for N tokens: 32 * 2^j, smallest with at most 1024
 // chunks (for N up to 32K tokens that is 32).
 int layout_chunk_tokens(int64_t n_tokens);
@@ -55,6 +58,15 @@ struct LayoutArgs {
 };
 
 cudaError_t launch_layout(const ep_buffer& b, const LayoutArgs& a, cudaStream_t stream);
+
+// Scratch ints the layout kernels need for T tokens per rank: per-chunk
+// counts [nc][E + R] plus the per-column rank prefixes [E + R][R + 1].
+int64_t layout_scratch_ints(const ep_config_t& c, int T);
+
+// The same three layout kernels on caller-given outputs and caller-given
+// scratch (layout_scratch_ints(c, T) ints), with no ep_buffer.
+cudaError_t launch_layout_raw(const ep_config_t& c, const LayoutArgs& a, const ep_layout_t& out,
+                              int32_t* scratch, uint32_t* err, cudaStream_t stream);
 cudaError_t launch_dispatch(const ep_buffer& b, int T, const void* x, cudaStream_t stream);
 cudaError_t launch_combine(const ep_buffer& b, int T, const void* y, const float* y_scale, void* out,
                            cudaStream_t stream);

@@ -484,4 +484,65 @@ cudaError_t launch_layout(const ep_buffer& b, const LayoutArgs& a, cudaStream_t 
     return cudaGetLastError();
 }
 
+int64_t layout_scratch_ints(const ep_config_t& c, int T) {
+    const int ch = layout_chunk_tokens((int64_t)c.num_ranks * T);
+    const int64_t nc = (int64_t)c.num_ranks * ((T + ch - 1) / ch);
+    const int64_t J = (int64_t)c.num_experts + c.num_ranks;
+    return nc * J + J * (c.num_ranks + 1);
+}
+
+cudaError_t launch_layout_raw(const ep_config_t& c, const LayoutArgs& a, const ep_layout_t& out,
+                              int32_t* scratch, uint32_t* err, cudaStream_t st) {
+    LayoutParams p{};
+    p.R = c.num_ranks;
+    p.T = a.T;
+    p.E = c.num_experts;
+    p.K = c.topk;
+    p.L = c.num_experts / c.num_ranks;
+    p.G = c.num_groups;
+    p.KG = c.topk_groups;
+    p.ch = layout_chunk_tokens((int64_t)p.R * p.T);
+    p.ncpr = (p.T + p.ch - 1) / p.ch;
+    p.nc = p.R * p.ncpr;
+    p.J = p.E + p.R;
+    p.route = a.route;
+    p.logits = a.logits;
+    p.vec_logits = (a.logits != nullptr && (p.E % 4 == 0) && ((uintptr_t)a.logits % 16 == 0)) ? 1 : 0;
+    p.in_idx = a.in_idx;
+    p.in_w = a.in_w;
+    p.mask_seed = a.mask_seed;
+    p.mask_thr = a.mask_threshold;
+    p.topk_idx = out.topk_idx;
+    p.topk_w = out.topk_w;
+    p.itr = out.is_token_in_rank;
+    p.chunk = scratch;
+    p.pref = scratch + (int64_t)p.nc * p.J;
+    p.ntpr = out.num_tokens_per_rank;
+    p.cnt = out.cnt_src_expert;
+    p.ntpe = out.num_tokens_per_expert;
+    p.expert_off = out.expert_off;
+    p.rank_off = out.rank_off;
+    p.src_off = out.src_off;
+    p.dst_row = out.dst_row;
+    p.m_max = (int64_t)p.R * p.T * p.K;  // no receive buffer: rows of this call only
+    p.err = err;
+
+    cudaError_t e = cudaSuccess;
+    if (p.nc > 0) {
+        const int epl = (p.E + 31) / 32;
+        if (epl <= 1) e = launch_route<1>(p, st);
+        else if (epl <= 2) e = launch_route<2>(p, st);
+        else if (epl <= 4) e = launch_route<4>(p, st);
+        else if (epl <= 8) e = launch_route<8>(p, st);
+        else if (epl <= 16) e = launch_route<16>(p, st);
+        else e = launch_route<32>(p, st);
+        if (e != cudaSuccess) return e;
+    }
+    chunk_scan_kernel<<<(p.J + 31) / 32, dim3(32, 32), 0, st>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const size_t smem = sizeof(int) * (2 * p.E + 1);
+    assign_rows_kernel<<<p.nc > 0 ? p.nc : 1, kAssignThreads, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
 }  // namespace ep

@@ -1,0 +1,115 @@
+// ep_get_layout_noalloc: routing + layout for callers that cannot allocate
+// device memory. Think of code inside a host framework whose memory planner
+// owns every device byte, or a runtime with a fixed memory budget that may
+// not call cudaMalloc (or any allocator) after start-up. Such a caller has
+// its input and output tensors but no way to get a workspace.
+//
+// The only scratch the layout kernels need is the per-chunk counts and their
+// prefix sums. Here that scratch lives in the file-scope device array below,
+// so this entry point allocates nothing: no cudaMalloc, cudaFree or allocating
+// library routine.
+//
+// Shared scratch: every call on a device uses the same array, and it keeps
+// whatever the last call left in it. The kernels overwrite every scratch entry
+// they read within the call, so nothing needs clearing. Calls whose work
+// overlaps on the GPU (two streams, or two host threads) race on the array
+// and give wrong layouts. Order them on one stream. Every GPU that loads
+// this library holds the array (2 MiB) until the process exits.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include <mutex>
+
+#include "ep.h"
+#include "internal.h"
+
+namespace {
+
+// 2 MiB: enough for 1024 chunks x (256 experts + 8 ranks), i.e. the prefill
+// and large workloads (E = 256, R = 8) at any T.
+constexpr int64_t kNoAllocScratchInts = (2 << 20) / 4;
+
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchInts];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int32_t* g_scratch_ptr[kMaxDevices] = {};  // device address of g_noalloc_scratch, per device
+
+ep_status_t fail(ep_status_t st, const char* msg) {
+    ep::set_last_error(msg);
+    return st;
+}
+
+// Once per device, with that device current: the device address of the
+// scratch array. In host code the symbol itself is only a host-side stand-in,
+// so a kernel must never be given &g_noalloc_scratch directly.
+cudaError_t scratch_for_current_device(int32_t** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" ep_status_t ep_get_layout_noalloc(const ep_config_t* cfg, int T, const float* d_logits,
+                                             const int32_t* d_topk_idx, const float* d_topk_w, int route,
+                                             uint64_t mask_seed, float mask_frac, const ep_layout_t* out,
+                                             uint32_t* d_error_word, void* stream) {
+    size_t ignored = 0;
+    ep_status_t st = ep_buffer_workspace_bytes(cfg, &ignored);  // validates the config
+    if (st != EP_OK) return st;
+    if (!out || !d_error_word) return fail(EP_ERR_INVALID, "out and d_error_word must be non-NULL");
+    if (!out->topk_idx || !out->topk_w || !out->is_token_in_rank || !out->num_tokens_per_rank ||
+        !out->cnt_src_expert || !out->num_tokens_per_expert || !out->expert_off || !out->rank_off ||
+        !out->src_off || !out->dst_row)
+        return fail(EP_ERR_INVALID, "every ep_layout_t output pointer must be set");
+    if (T < 0) return fail(EP_ERR_INVALID, "T must be >= 0");
+    if (T > cfg->max_tokens_per_rank) return fail(EP_ERR_CAPACITY, "T exceeds max_tokens_per_rank");
+    const bool have_logits = d_logits != nullptr;
+    const bool have_idx = d_topk_idx != nullptr || d_topk_w != nullptr;
+    if (have_logits == have_idx) return fail(EP_ERR_INVALID, "pass either d_logits or d_topk_idx + d_topk_w");
+    if (have_idx && (!d_topk_idx || !d_topk_w)) return fail(EP_ERR_INVALID, "d_topk_idx and d_topk_w go together");
+    if (have_logits && (route < EP_ROUTE_SOFTMAX || route > EP_ROUTE_GROUP_SIGMOID))
+        return fail(EP_ERR_INVALID, "unknown route");
+    if (!(mask_frac >= 0.0f && mask_frac <= 1.0f)) return fail(EP_ERR_INVALID, "mask_frac must be in [0, 1]");
+    if (ep::layout_scratch_ints(*cfg, T) > kNoAllocScratchInts)
+        return fail(EP_ERR_CAPACITY,
+                    "layout scratch for this config and T exceeds the 2 MiB static scratch of "
+                    "ep_get_layout_noalloc; use ep_get_layout with a workspace");
+
+    int32_t* scratch = nullptr;
+    cudaError_t e = scratch_for_current_device(&scratch);
+    if (e != cudaSuccess) {
+        char m[200];
+        snprintf(m, sizeof m, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+        return fail(EP_ERR_CUDA, m);
+    }
+    ep::LayoutArgs a{};
+    a.T = T;
+    a.logits = d_logits;
+    a.in_idx = d_topk_idx;
+    a.in_w = d_topk_w;
+    a.route = route;
+    a.mask_seed = mask_seed;
+    a.mask_threshold = (uint64_t)floor((double)mask_frac * 4294967296.0);
+    e = ep::launch_layout_raw(*cfg, a, *out, scratch, d_error_word, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        char m[200];
+        snprintf(m, sizeof m, "layout launch: %s", cudaGetErrorString(e));
+        return fail(EP_ERR_CUDA, m);
+    }
+    ep::set_last_error("");
+    return EP_OK;
+}

@@ -69,10 +69,14 @@ _lib.ep_combine.argtypes = [_P, ctypes.c_int, _P, _P, _P, _P]
 _lib.ep_combine.restype = _st
 _lib.ep_check_errors.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, _P]
 _lib.ep_check_errors.restype = _st
+_lib.ep_get_layout_noalloc.argtypes = [ctypes.POINTER(EpConfig), ctypes.c_int, _P, _P, _P, ctypes.c_int,
+                                       ctypes.c_uint64, ctypes.c_float, ctypes.POINTER(EpLayout), _P, _P]
+_lib.ep_get_layout_noalloc.restype = _st
 
 EXPORTED = ("ep_abi_version", "ep_status_string", "ep_last_error_message", "ep_default_config",
             "ep_buffer_workspace_bytes", "ep_buffer_create", "ep_buffer_destroy", "ep_buffer_layout",
-            "ep_buffer_recv", "ep_get_layout", "ep_dispatch", "ep_combine", "ep_check_errors")
+            "ep_buffer_recv", "ep_get_layout", "ep_dispatch", "ep_combine", "ep_check_errors",
+            "ep_get_layout_noalloc")
 
 
 class EpError(RuntimeError):
@@ -231,3 +235,21 @@ def ep_check_errors(buf: EpBuffer, clear: bool = True, stream=None) -> int:
     if st not in (EP_OK, EP_ERR_DEVICE):
         _check(st, "ep_check_errors")
     return w.value
+
+
+def ep_get_layout_noalloc(cfg: EpConfig, T: int, out: dict, error_word, logits=None, topk_idx=None,
+                          topk_w=None, route: int = 0, mask_seed: int = 0, mask_frac: float = 0.0,
+                          stream=None) -> None:
+    """Routing + layout into the caller's own tensors (`out` holds the
+    ep_layout_t arrays by name, as ep_buffer_layout returns them;
+    `error_word` is a 1-element int32/uint32 CUDA tensor). It uses the
+    library's static scratch and allocates nothing."""
+    lay = EpLayout(topk_idx=_ptr(out["topk_idx"]), topk_w=_ptr(out["topk_w"]),
+                   is_token_in_rank=_ptr(out["is_token_in_rank"]),
+                   num_tokens_per_rank=_ptr(out["num_tokens_per_rank"]), cnt_src_expert=_ptr(out["cnt"]),
+                   num_tokens_per_expert=_ptr(out["num_tokens_per_expert"]),
+                   expert_off=_ptr(out["expert_off"]), rank_off=_ptr(out["rank_off"]),
+                   src_off=_ptr(out["src_off"]), dst_row=_ptr(out["dst_row"]))
+    _check(_lib.ep_get_layout_noalloc(ctypes.byref(cfg), T, _ptr(logits), _ptr(topk_idx), _ptr(topk_w), route,
+                                      mask_seed & 0xFFFF_FFFF_FFFF_FFFF, mask_frac, ctypes.byref(lay),
+                                      _ptr(error_word), _stream(stream)), "ep_get_layout_noalloc")

@@ -189,6 +189,39 @@ ep_status_t ep_combine(ep_buffer_t *buf, int T, const void *d_y, const float *d_
  * none, EP_ERR_CUDA on a CUDA failure. */
 ep_status_t ep_check_errors(ep_buffer_t *buf, uint32_t *word, int clear, void *stream);
 
+/* Routing + layout that allocates nothing, for callers that cannot get device
+ * memory beyond their own inputs and outputs: code under a host framework
+ * whose memory planner owns every device byte, or a runtime with a fixed
+ * budget that may not call cudaMalloc after start-up. The paper has no
+ * counterpart: it is a deployment variant of ep_get_layout.
+ *
+ * Computes exactly what ep_get_layout computes, with the same inputs and
+ * meaning. The outputs go to the caller's device arrays in *out, a host
+ * struct of device pointers, every one required, sized for N = R*T as
+ * ep_layout_t lists. The layout's scratch (per-chunk counts and their prefix
+ * sums) lives in a file-scope device array of 2 MiB that every GPU loading
+ * the library holds until exit. The call makes no cudaMalloc, cudaFree or
+ * other allocating call.
+ *  - Limit: R*ceil(T/ch)*(E+R) + (E+R)*(R+1) int32 scratch entries must fit
+ *    in 2 MiB, where ch is the chunk size (32 tokens, doubled until there are
+ *    at most 1024 chunks). E = 256 and R = 8 fit for any T. Beyond it the
+ *    call returns EP_ERR_CAPACITY and launches nothing.
+ *  - d_error_word: a device uint32 that receives EP_DEVERR_* bits with
+ *    atomicOr. The caller zeroes and reads it.
+ *  - Runs on the current device. `stream` must belong to it.
+ *  - Set-up: the first call on each device looks up the device address of
+ *    the static scratch (cudaGetSymbolAddress). Make that first call before
+ *    any stream capture.
+ *  - Every call on a device shares the one scratch array and leaves its
+ *    contents behind. The kernels rewrite every entry they read, so nothing
+ *    needs clearing, but calls whose GPU work overlaps (different streams or
+ *    host threads) race and give wrong results.
+ * Errors: as ep_get_layout, plus EP_ERR_INVALID for a NULL output pointer. */
+ep_status_t ep_get_layout_noalloc(const ep_config_t *cfg, int T, const float *d_logits,
+                                  const int32_t *d_topk_idx, const float *d_topk_w, int route,
+                                  uint64_t mask_seed, float mask_frac, const ep_layout_t *out,
+                                  uint32_t *d_error_word, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
