@@ -183,10 +183,7 @@ def run_ours(args, w: wl.Workload, rank: int, world: int, local_rank: int):
     t_disp = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
     t_comb = sum(e[2].elapsed_time(e[3]) for e in ev) / 1e3
     t_total = t_layout + t_disp + t_comb
-    if world > 1:
-        t = torch.tensor([t_total, t_layout, t_disp, t_comb], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_total, t_layout, t_disp, t_comb = t.tolist()
+    t_total, t_layout, t_disp, t_comb = metrics.max_over_ranks([t_total, t_layout, t_disp, t_comb], dev)
     K = args.steps
     value = world * bytes_step * K / t_total / 1e9
 
@@ -265,11 +262,7 @@ def measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps, world):
         one()
     e.record(stream)
     torch.cuda.synchronize(dev)
-    t = s.elapsed_time(e) / 1e3
-    if world > 1:
-        tt = torch.tensor([t], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t = tt.item()
+    t = metrics.max_over_ranks([s.elapsed_time(e) / 1e3], dev)[0]
     return {"value": world * bytes_step * steps / t / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": t / steps * 1e3}
 

@@ -49,6 +49,20 @@ def combine_bytes(w: wl.Workload, M: int, fused_fp8: bool = False, N: int | None
     return y + N * w.K * 8 + N * w.H * 2
 
 
+# ---- multi-rank timing --------------------------------------------------------
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank timings over the default process group
+    (all ranks call it). Single process: the values unchanged."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 # ---- peaks -------------------------------------------------------------------
 
 def hbm_peak() -> tuple[float, str]:

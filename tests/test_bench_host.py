@@ -1,0 +1,92 @@
+"""Host-side logic of the bench on the CPU:
+- algorithmic byte formulas;
+- clock parsing and the rejection rules;
+- max-over-ranks timing across 2 gloo ranks;
+- the reference arm's JSON line, and rank > 0 exiting quietly."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+from combine_top_group_b200 import metrics
+from combine_top_group_b200 import workloads as wl
+from conftest import ROOT
+
+
+def test_byte_formulas_prefill():
+    w = wl.WORKLOADS["prefill"]
+    M = w.N * w.K
+    d = metrics.dispatch_bytes(w, M)
+    c = metrics.combine_bytes(w, M)
+    # dominant terms: read N rows once, write M rows (bf16) / read M rows, write N rows
+    assert d == w.N * w.H * 2 + M * w.H * 2 + w.N * w.K * 8 + M * 8
+    assert c == M * w.H * 2 + w.N * w.H * 2 + w.N * w.K * 8
+    assert 4.22e9 < d < 4.24e9 and 4.22e9 < c < 4.24e9
+    assert metrics.layout_bytes(w) == w.N * w.E * 4 + w.N * w.K * 12 + w.N * w.R
+
+
+def test_byte_formulas_fp8():
+    w = wl.WORKLOADS["large"]
+    M = w.N * w.K
+    d = metrics.dispatch_bytes(w, M)
+    assert d == w.N * w.H * 2 + w.N * w.K * 8 + M * w.H + M * (w.H // 128) * 4 + M * 8
+    assert metrics.combine_bytes(w, M, fused_fp8=True) == M * w.H + M * 56 * 4 + w.N * w.K * 8 + w.N * w.H * 2
+
+
+CSV = """index, clocks.current.sm [MHz], clocks.max.sm [MHz], power.draw [W], clocks_event_reasons.active, clocks_event_reasons.hw_slowdown, clocks_event_reasons.hw_thermal_slowdown, clocks_event_reasons.sw_thermal_slowdown, clocks_event_reasons.sw_power_cap
+0, 1965 MHz, 1965 MHz, 700.1 W, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active
+0, 1800 MHz, 1965 MHz, 990.0 W, 0x0000000000000004, Not Active, Not Active, Not Active, Active
+0, 1900 MHz, 1965 MHz, 900.0 W, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active
+"""
+
+
+def test_parse_clocks_and_rules():
+    c = metrics.parse_clocks(CSV.replace("clocks.current.sm", "clocks.sm"))
+    assert c["sm_mhz"] == 1900 and c["sm_max_mhz"] == 1965 and c["reasons"] == ["sw_power_cap"]
+    assert metrics.clocks_rejected(c) is None
+    assert "throttled" in metrics.clocks_rejected({"sm_mhz": 1900, "sm_max_mhz": 1965, "reasons": ["hw_slowdown"]})
+    assert "clock lock" in metrics.clocks_rejected({"sm_mhz": 800, "sm_max_mhz": 1965, "reasons": []})
+    s = metrics.summarize_nvml([(1900, 1965, 800.0, 0x4), (1700, 1965, 990.0, 0x40)], metrics.ClockSampler._BITS)
+    assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"] and s["sm_mhz"] == 1800
+
+
+def _rank_main(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    got = metrics.max_over_ranks([1.0 + rank, 5.0 - rank])
+    q.put((rank, got))
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + os.getpid() % 1000
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res[0] == res[1] == [2.0, 5.0]
+
+
+def test_reference_arm_json_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "tiny",
+                        "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "GB/s"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "tiny",
+                        "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 0 and r.stdout.strip() == ""
