@@ -114,6 +114,34 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---- 256-bit global loads and stores (sm_100) ------------------------------
+
+struct __align__(32) u32x8 {
+    uint32_t v[8];
+};
+
+// Streaming 256-bit load: the data is read once.
+__device__ __forceinline__ u32x8 ld256_stream(const void* p) {
+    u32x8 a;
+    asm volatile("ld.global.cs.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(a.v[0]), "=r"(a.v[1]), "=r"(a.v[2]), "=r"(a.v[3]), "=r"(a.v[4]), "=r"(a.v[5]),
+                   "=r"(a.v[6]), "=r"(a.v[7])
+                 : "l"(p));
+    return a;
+}
+
+__device__ __forceinline__ void st256(void* p, const u32x8& a) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.v[0]), "r"(a.v[1]),
+                 "r"(a.v[2]), "r"(a.v[3]), "r"(a.v[4]), "r"(a.v[5]), "r"(a.v[6]), "r"(a.v[7])
+                 : "memory");
+}
+
+__device__ __forceinline__ void st256_stream(void* p, const u32x8& a) {
+    asm volatile("st.global.cs.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.v[0]), "r"(a.v[1]),
+                 "r"(a.v[2]), "r"(a.v[3]), "r"(a.v[4]), "r"(a.v[5]), "r"(a.v[6]), "r"(a.v[7])
+                 : "memory");
+}
+
 // ---- number formats -------------------------------------------------------
 
 __device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }

@@ -69,14 +69,14 @@ struct Plan {
 // Region order inside the workspace; every region is 256-byte aligned.
 enum {
     R_TOPK_IDX, R_TOPK_W, R_ITR, R_NTPR, R_CNT, R_NTPE, R_EOFF, R_ROFF, R_SOFF, R_DST,
-    R_CHUNK, R_PREF, R_ERR, R_RECV_X, R_RECV_SCALE, R_RECV_SRC, R_RECV_W, R_COUNT
+    R_SCRATCH, R_ERR, R_RECV_X, R_RECV_SCALE, R_RECV_SRC, R_RECV_W, R_COUNT
 };
 
 Plan plan_of(const ep_config_t* c, int64_t* n_max, int64_t* m_max, int64_t* nc_max) {
     const int64_t R = c->num_ranks, T = c->max_tokens_per_rank, H = c->hidden, E = c->num_experts,
                   K = c->topk;
     const int64_t N = R * T, M = N * K;
-    const int64_t nc = R * ((T + 31) / 32);  // most chunks: 32 tokens each
+    const int64_t scratch = ep::layout_scratch_ints(*c, ep::kMaxLayoutCtas);
     const bool fp8 = (c->flags & EP_FLAG_FP8) != 0;
     size_t sz[R_COUNT];
     sz[R_TOPK_IDX] = 4 * N * K;
@@ -89,8 +89,7 @@ Plan plan_of(const ep_config_t* c, int64_t* n_max, int64_t* m_max, int64_t* nc_m
     sz[R_ROFF] = 4 * (R + 1);
     sz[R_SOFF] = 4 * E * R;
     sz[R_DST] = 4 * N * K;
-    sz[R_CHUNK] = 4 * nc * (E + R);
-    sz[R_PREF] = 4 * (E + R) * (R + 1);
+    sz[R_SCRATCH] = 4 * scratch;
     sz[R_ERR] = 16;
     sz[R_RECV_X] = (size_t)M * H * (fp8 ? 1 : 2);
     sz[R_RECV_SCALE] = fp8 ? (size_t)M * (H / 128) * 4 : 0;
@@ -105,7 +104,7 @@ Plan plan_of(const ep_config_t* c, int64_t* n_max, int64_t* m_max, int64_t* nc_m
     p.total = cur;
     *n_max = N;
     *m_max = M;
-    *nc_max = nc;
+    *nc_max = ep::kMaxLayoutCtas;
     return p;
 }
 
@@ -202,8 +201,7 @@ ep_status_t ep_buffer_create(const ep_config_t* cfg, void* d_workspace, size_t b
     b->rank_off = reinterpret_cast<int32_t*>(w + p.off[R_ROFF]);
     b->src_off = reinterpret_cast<int32_t*>(w + p.off[R_SOFF]);
     b->dst_row = reinterpret_cast<int32_t*>(w + p.off[R_DST]);
-    b->chunk = reinterpret_cast<int32_t*>(w + p.off[R_CHUNK]);
-    b->pref = reinterpret_cast<int32_t*>(w + p.off[R_PREF]);
+    b->scratch = reinterpret_cast<int32_t*>(w + p.off[R_SCRATCH]);
     b->err = reinterpret_cast<uint32_t*>(w + p.off[R_ERR]);
     b->recv_x = w + p.off[R_RECV_X];
     b->recv_scale = (cfg->flags & EP_FLAG_FP8) ? reinterpret_cast<float*>(w + p.off[R_RECV_SCALE]) : nullptr;
@@ -215,6 +213,7 @@ ep_status_t ep_buffer_create(const ep_config_t* cfg, void* d_workspace, size_t b
     // legacy-stream memset, then wait for it: callers' streams may be
     // non-blocking and would not be ordered after it otherwise
     e = cudaMemset(b->err, 0, 16);
+    if (e == cudaSuccess) e = cudaMemset(b->scratch, 0, sizeof(int32_t) * ep::kLayoutControlInts);
     if (e == cudaSuccess) e = cudaStreamSynchronize(nullptr);
     if (prev != dev) cudaSetDevice(prev);
     if (e != cudaSuccess) {
@@ -282,6 +281,7 @@ ep_status_t ep_get_layout(ep_buffer_t* b, int T, const float* d_logits, const in
     a.mask_seed = mask_seed;
     double thr = floor((double)mask_frac * 4294967296.0);
     a.mask_threshold = (uint64_t)thr;
+    a.m_max = b->m_max;
     cudaError_t e = ep::launch_layout(*b, a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "layout launch");
     b->last_T = T;
@@ -292,7 +292,7 @@ ep_status_t ep_dispatch(ep_buffer_t* b, int T, const void* d_x, void* stream) {
     if (ep_status_t st = check_buf(b)) return st;
     if (T != b->last_T) return fail(EP_ERR_INVALID, "T=%d does not match the last ep_get_layout (T=%d)", T, b->last_T);
     if (T > 0 && !d_x) return fail(EP_ERR_INVALID, "d_x is NULL");
-    if ((uintptr_t)d_x % 16 != 0) return fail(EP_ERR_INVALID, "d_x must be 16-byte aligned");
+    if ((uintptr_t)d_x % 32 != 0) return fail(EP_ERR_INVALID, "d_x must be 32-byte aligned");
     cudaError_t e = ep::launch_dispatch(*b, T, d_x, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
     return ok();
@@ -302,8 +302,8 @@ ep_status_t ep_combine(ep_buffer_t* b, int T, const void* d_y, const float* d_y_
     if (ep_status_t st = check_buf(b)) return st;
     if (T != b->last_T) return fail(EP_ERR_INVALID, "T=%d does not match the last ep_get_layout (T=%d)", T, b->last_T);
     if (T > 0 && (!d_y || !d_out)) return fail(EP_ERR_INVALID, "d_y and d_out must be non-NULL");
-    if ((uintptr_t)d_y % 16 != 0 || (uintptr_t)d_out % 16 != 0)
-        return fail(EP_ERR_INVALID, "d_y and d_out must be 16-byte aligned");
+    if ((uintptr_t)d_y % 32 != 0 || (uintptr_t)d_out % 32 != 0)
+        return fail(EP_ERR_INVALID, "d_y and d_out must be 32-byte aligned");
     if (d_y_scale && (uintptr_t)d_y_scale % 4 != 0) return fail(EP_ERR_INVALID, "d_y_scale must be 4-byte aligned");
     cudaError_t e = ep::launch_combine(*b, T, d_y, d_y_scale, d_out, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "combine launch");
@@ -317,7 +317,9 @@ ep_status_t ep_check_errors(ep_buffer_t* b, uint32_t* word, int clear, void* str
     cudaError_t e = cudaMemcpyAsync(&v, b->err, sizeof v, cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e == cudaSuccess && clear) {
+        // also reset the layout's barrier words, which a timed-out launch may leave set
         e = cudaMemsetAsync(b->err, 0, sizeof v, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(b->scratch, 0, sizeof(int32_t) * ep::kLayoutControlInts, s);
         if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     }
     if (e != cudaSuccess) return cuda_fail(e, "ep_check_errors");

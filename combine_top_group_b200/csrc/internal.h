@@ -26,10 +26,8 @@ struct ep_buffer {
     int32_t* rank_off;
     int32_t* src_off;
     int32_t* dst_row;
-    // layout scratch (device): per-chunk counts, later their prefix sums,
-    // [nc][E + R]; per-column prefix at each rank's first chunk, [E + R][R + 1]
-    int32_t* chunk;
-    int32_t* pref;
+    // layout scratch (device): barrier words, per-chunk counts and prefixes
+    int32_t* scratch;
     uint32_t* err;  // device error word
     // receive buffers (device)
     void* recv_x;
@@ -43,9 +41,10 @@ namespace ep {
 // Sets the message ep_last_error_message() returns on this host thread.
 void set_last_error(const char* msg);
 
-// Tokens per layout chunk for N tokens: 32 * 2^j, smallest with at most 1024
-// chunks (for N up to 32K tokens that is 32).
-int layout_chunk_tokens(int64_t n_tokens);
+// Layout grid cap (CTAs = chunks) and the control words at the head of the
+// layout scratch (two barrier counters, zero between launches).
+constexpr int kMaxLayoutCtas = 1024;
+constexpr int kLayoutControlInts = 64;
 
 struct LayoutArgs {
     int T;
@@ -55,18 +54,20 @@ struct LayoutArgs {
     int route;
     uint64_t mask_seed;
     uint64_t mask_threshold;  // in [0, 2^32]
+    int64_t m_max;            // rows the receive side holds (bound check)
 };
 
-cudaError_t launch_layout(const ep_buffer& b, const LayoutArgs& a, cudaStream_t stream);
+// int32 entries of layout scratch for a grid of at most max_ctas CTAs:
+// control words, per-chunk counts [E+R][max_ctas], totals [E+R], rank
+// prefixes [E+R][R+1].
+int64_t layout_scratch_ints(const ep_config_t& c, int max_ctas);
 
-// Scratch ints the layout kernels need for T tokens per rank: per-chunk
-// counts [nc][E + R] plus the per-column rank prefixes [E + R][R + 1].
-int64_t layout_scratch_ints(const ep_config_t& c, int T);
-
-// The same three layout kernels on caller-given outputs and caller-given
-// scratch (layout_scratch_ints(c, T) ints), with no ep_buffer.
+// The layout kernel on caller-given outputs and scratch
+// (layout_scratch_ints(c, max_ctas) ints whose control words are zero).
 cudaError_t launch_layout_raw(const ep_config_t& c, const LayoutArgs& a, const ep_layout_t& out,
-                              int32_t* scratch, uint32_t* err, cudaStream_t stream);
+                              int32_t* scratch, int max_ctas, uint32_t* err, cudaStream_t stream);
+
+cudaError_t launch_layout(const ep_buffer& b, const LayoutArgs& a, cudaStream_t stream);
 cudaError_t launch_dispatch(const ep_buffer& b, int T, const void* x, cudaStream_t stream);
 cudaError_t launch_combine(const ep_buffer& b, int T, const void* y, const float* y_scale, void* out,
                            cudaStream_t stream);

@@ -2,22 +2,37 @@
 // dispatch needs: "DeepEP：年度总结中的计算通信重叠摘记", §节点内通信, fuses
 // Top-K with the sparse communication and builds is_token_in_rank.
 //
-// Three stream-ordered launches, with no host sync in between:
-//   A  route_count: one warp per token. It selects the top K (optionally
-//      group-limited, §计算-通信重叠), applies the slot mask and writes
-//      topk_idx / topk_w / is_token_in_rank. It also builds per-chunk expert
-//      and rank histograms in shared memory.
-//   B  chunk_scan: an exclusive scan over chunks for every expert and rank
-//      column, plus the prefix at each rank's first chunk.
-//   C  assign_rows: the exclusive scan over experts (expert_off). Then each
-//      chunk's slots, in (token, slot) order, get consecutive rows inside
-//      their expert's block via warp match/popc. Block 0 writes the small
-//      global arrays.
-// A chunk is a run of consecutive tokens of one source rank. Chunks are in
-// global token order, so scanning chunks in order places rows in (expert,
-// source rank, token, slot) order.
+// One persistent cooperative kernel. The grid is one resident wave, and every
+// CTA owns one chunk: a run of consecutive tokens of one source rank, so
+// chunks are in global token order. Phases, separated by bounded grid barriers:
+//   1  route: one warp per token. Top-K (optionally group-limited,
+//      §计算-通信重叠), the slot mask, and the topk_idx / topk_w /
+//      is_token_in_rank writes. Each warp takes a contiguous run of its
+//      chunk's tokens and counts its slots per expert and its tokens per
+//      destination rank in shared memory. The chunk's totals go to global
+//      scratch.
+//   2  scan: one CTA per expert/rank column. A block scan over the chunks
+//      gives each chunk's exclusive prefix and the column total. Reading it
+//      at each rank's first chunk gives src_off and cnt (expert columns) or
+//      num_tokens_per_rank (rank columns).
+//   3  place: every CTA scans the expert totals into expert_off. Its warps
+//      then turn their kept histograms into per-warp row bases and rank their
+//      own slots in (token, slot) order with match_any/popc, writing dst_row.
+// Receive rows come out ordered by (expert, source rank, token, slot).
+//
+// Routing arithmetic:
+//  - Expert ranking compares the logits exactly (order-preserving 32-bit
+//    keys; equal values go to the lower expert id).
+//  - Group scores (sum of the two largest sigmoids) run in fp32, with a
+//    bound on their error. If the gap between the last kept and the first
+//    dropped group is under 4e-6, well above that bound, the warp recomputes
+//    the scores in fp64, the precision the decision is defined in. The kept
+//    groups therefore always equal the fp64 ones.
+//  - Weights are computed in fp64 and rounded once to fp32.
 #include <cuda_runtime.h>
 #include <math.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -25,12 +40,14 @@
 namespace ep {
 namespace {
 
-constexpr int kRouteWarps = 8;  // warps (tokens in flight) per route_count block
-constexpr int kAssignThreads = 256;
+constexpr int kWarps = 8;  // warps per CTA
+constexpr int kThreads = kWarps * 32;
 
 struct LayoutParams {
-    int R, T, E, K, L, G, KG;
-    int ch, ncpr, nc, J;  // chunk tokens, chunks per rank, chunks, columns (E + R)
+    int R, T, E, K, L, G, KG, J;  // J = E + R histogram columns
+    uint32_t l_magic;             // e / L == __umulhi(e, l_magic) for 0 <= e < 2^16
+    int nb;                       // CTAs (one resident wave)
+    int ncpr, nc;                 // chunks per rank, chunks (nc <= nb)
     int route;
     int vec_logits;  // logits rows are 16-byte aligned and E % 4 == 0
     const float* logits;
@@ -41,40 +58,180 @@ struct LayoutParams {
     int32_t* topk_idx;
     float* topk_w;
     uint8_t* itr;
-    int32_t* chunk;
-    int32_t* pref;
+    int32_t* chunk;  // [J][nc]: chunk counts, then their exclusive prefix over chunks
+    int32_t* tot;    // [J]: column totals
     int32_t *ntpr, *cnt, *ntpe, *expert_off, *rank_off, *src_off, *dst_row;
     int64_t m_max;
     uint32_t* err;
+    uint32_t* bar;  // [2]: barrier arrivals, finished CTAs; both 0 between launches
 };
 
 __device__ __forceinline__ double sigmoid_d(double x) { return 1.0 / (1.0 + exp(-x)); }
+__device__ __forceinline__ float sigmoid_f(float x) { return __frcp_rn(1.0f + expf(-x)); }
 
-// Warp-wide top-2 of one value per lane (NEG = no value), across lanes that
-// differ in the bits of `span` (a power of two): butterfly over offsets span/2..1.
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Bounded grid-wide barrier (the grid is co-resident: cooperative launch).
+__device__ void grid_barrier(uint32_t* arrive, uint32_t target, uint32_t* err) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(arrive, 1u);
+        const unsigned long long t0 = globaltimer_ns();
+        while (ld_acquire(arrive) < target) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                set_error(err, EP_DEVERR_TIMEOUT);
+                break;
+            }
+            __nanosleep(64);
+        }
+        __threadfence();
+    }
+    __syncthreads();
+}
+
+// Top-2 of one pair per lane across lanes that differ in the bits of `span`
+// (a power of two): butterfly over offsets span/2..1.
 __device__ __forceinline__ void top2_merge(uint32_t& a, uint32_t& b, int span) {
     for (int off = span >> 1; off > 0; off >>= 1) {
-        uint32_t oa = __shfl_xor_sync(FULL, a, off);
-        uint32_t ob = __shfl_xor_sync(FULL, b, off);
-        // merge two sorted pairs (a >= b, oa >= ob) into the top two
-        uint32_t hi = max(a, oa);
-        uint32_t lo = max(min(a, oa), max(b, ob));
+        const uint32_t oa = __shfl_xor_sync(FULL, a, off);
+        const uint32_t ob = __shfl_xor_sync(FULL, b, off);
+        const uint32_t hi = max(a, oa);
+        const uint32_t lo = max(min(a, oa), max(b, ob));
         a = hi;
         b = lo;
     }
 }
 
-// Routes token g with one warp. Lane k < K ends up holding slot k's expert id
-// (-1 = masked) and weight.
+// This lane's two best candidates by (key desc, position asc), skipping
+// taken positions and zero keys. Returns key 0 where there is none.
 template <int EPL>
-__device__ __forceinline__ void route_token(const LayoutParams& p, int64_t g, int lane, int& my_e, float& my_w) {
+__device__ __forceinline__ void top2_of(const uint32_t (&key)[EPL], uint32_t taken, uint32_t& a, int& pa,
+                                        uint32_t& b, int& pb) {
+    a = 0u;
+    b = 0u;
+    pa = 0;
+    pb = 0;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+        const uint32_t k = ((taken >> j) & 1u) ? 0u : key[j];
+        if (k > a) {  // strict: an equal key later in the list stays behind
+            b = a;
+            pb = pa;
+            a = k;
+            pa = j;
+        } else if (k > b) {
+            b = k;
+            pb = j;
+        }
+    }
+}
+
+// Group scores and the kept-group mask (bit g set = group g kept).
+template <int EPL>
+__device__ __forceinline__ uint32_t kept_groups(const LayoutParams& p, const uint32_t (&key)[EPL], uint32_t a,
+                                                uint32_t b, int lane) {
+    const int gs = p.E / p.G;
+    const int e0 = lane * EPL;
+    const int lpg = gs / EPL;
+    int rank = 0;
+    if (gs % EPL == 0 && lpg <= 32 && (lpg & (lpg - 1)) == 0) {
+        // each group spans lpg whole lanes: the lanes' top-2, then a butterfly
+        top2_merge(a, b, lpg);
+        const int src = (lane < p.G) ? lane * lpg : 0;
+        const float s32 = sigmoid_f(key_value(a)) + sigmoid_f(key_value(b));
+        const float sc = __shfl_sync(FULL, s32, src);  // group `lane`'s fp32 score
+        for (int h = 0; h < p.G; ++h) {
+            const float sh = __shfl_sync(FULL, sc, h);
+            if (lane < p.G && (sh > sc || (sh == sc && h < lane))) ++rank;
+        }
+        bool certain = true;
+        if (p.KG < p.G) {
+            // fp32 sigmoid error <= 3*2^-23 (expf <= 2 ulp, add and rcp 0.5 ulp each),
+            // so a score errs by < 1e-6. A gap over 4e-6 decides as fp64 would.
+            const uint32_t m_last = __ballot_sync(FULL, lane < p.G && rank == p.KG - 1);
+            const uint32_t m_next = __ballot_sync(FULL, lane < p.G && rank == p.KG);
+            const float s_last = __shfl_sync(FULL, sc, __ffs(m_last) - 1);
+            const float s_next = __shfl_sync(FULL, sc, __ffs(m_next) - 1);
+            certain = (s_last - s_next) > 4e-6f;
+        }
+        if (!certain) {  // warp-uniform: decide in fp64
+            const double s64 = sigmoid_d((double)key_value(a)) + sigmoid_d((double)key_value(b));
+            const double sd = __shfl_sync(FULL, s64, src);
+            rank = 0;
+            for (int h = 0; h < p.G; ++h) {
+                const double sh = __shfl_sync(FULL, sd, h);
+                if (lane < p.G && (sh > sd || (sh == sd && h < lane))) ++rank;
+            }
+        }
+    } else {
+        // generic layout of groups over lanes: one warp-wide top-2 per group, fp64
+        double score = -1.0;
+        for (int grp = 0; grp < p.G; ++grp) {
+            uint32_t a = 0, b = 0;
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) {
+                const int e = e0 + j;
+                const uint32_t k = (e < p.E && e / gs == grp) ? key[j] : 0u;
+                if (k > a) {
+                    b = a;
+                    a = k;
+                } else if (k > b) {
+                    b = k;
+                }
+            }
+            top2_merge(a, b, 32);
+            if (lane == grp) score = sigmoid_d((double)key_value(a)) + sigmoid_d((double)key_value(b));
+        }
+        for (int h = 0; h < p.G; ++h) {
+            const double sh = __shfl_sync(FULL, score, h);
+            if (lane < p.G && (sh > score || (sh == score && h < lane))) ++rank;
+        }
+    }
+    return __ballot_sync(FULL, lane < p.G && rank < p.KG);
+}
+
+// This lane's EPL logits of token g (experts lane*EPL ..); zeros past E.
+template <int EPL>
+__device__ __forceinline__ void load_logits(const LayoutParams& p, int64_t g, int lane, float (&v)[EPL]) {
+    const float* row = p.logits + g * p.E;
+    const int e0 = lane * EPL;
+    if (EPL >= 4 && p.vec_logits) {
+#pragma unroll
+        for (int j = 0; j < EPL; j += 4) {
+            if (e0 + j < p.E) {
+                const float4 q = __ldcs(reinterpret_cast<const float4*>(row + e0 + j));
+                v[j] = q.x;
+                v[j + 1] = q.y;
+                v[j + 2] = q.z;
+                v[j + 3] = q.w;
+            } else {
+                v[j] = v[j + 1] = v[j + 2] = v[j + 3] = 0.0f;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) v[j] = (e0 + j < p.E) ? __ldcs(row + e0 + j) : 0.0f;
+    }
+}
+
+// Routes token g with one warp, from its logits vin (load_logits) when the
+// call routes logits. Lane k < K ends up holding slot k's expert id (-1 =
+// masked) and weight.
+template <int EPL>
+__device__ __forceinline__ void route_token(const LayoutParams& p, int64_t g, int lane, const float (&vin)[EPL],
+                                            int& my_e, float& my_w) {
     my_e = -1;
     my_w = 0.0f;
     if (p.logits == nullptr) {
         // caller-supplied top-k
         if (lane < p.K) {
             int e = p.in_idx[g * p.K + lane];
-            float w = p.in_w[g * p.K + lane];
+            const float w = p.in_w[g * p.K + lane];
             if (e < -1 || e >= p.E) {
                 set_error(p.err, EP_DEVERR_EXPERT_ID);
                 e = -1;
@@ -83,120 +240,59 @@ __device__ __forceinline__ void route_token(const LayoutParams& p, int64_t g, in
             my_w = w;
         }
     } else {
-        const float* row = p.logits + g * p.E;
-        float v[EPL];
         uint32_t key[EPL];
         const int e0 = lane * EPL;
-        if (EPL >= 4 && p.vec_logits) {
 #pragma unroll
-            for (int j = 0; j < EPL; j += 4) {
-                if (e0 + j < p.E) {
-                    float4 q = *reinterpret_cast<const float4*>(row + e0 + j);
-                    v[j] = q.x;
-                    v[j + 1] = q.y;
-                    v[j + 2] = q.z;
-                    v[j + 3] = q.w;
-                } else {
-                    v[j] = v[j + 1] = v[j + 2] = v[j + 3] = 0.0f;
-                }
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < EPL; ++j) v[j] = (e0 + j < p.E) ? row[e0 + j] : 0.0f;
-        }
-#pragma unroll
-        for (int j = 0; j < EPL; ++j) key[j] = (e0 + j < p.E) ? order_key(v[j]) : 0u;
+        for (int j = 0; j < EPL; ++j) key[j] = (e0 + j < p.E) ? order_key(vin[j]) : 0u;
+
+        // this lane's two best candidates; a lane rescans its list only when
+        // both have been taken
+        uint32_t a, b, taken = 0u;
+        int pa, pb;
+        top2_of<EPL>(key, 0u, a, pa, b, pb);
 
         if (p.route == EP_ROUTE_GROUP_SIGMOID && p.G > 1) {
-            // group score = sigmoid of the group's two largest logits, summed in fp64
+            const uint32_t kept = kept_groups<EPL>(p, key, a, b, lane);
             const int gs = p.E / p.G;
-            double score = -1.0;  // valid on lane g for g < G
-            const int lpg = gs / EPL;
-            if (gs % EPL == 0 && lpg <= 32 && (lpg & (lpg - 1)) == 0) {
-                // each group spans lpg whole lanes
-                uint32_t a = 0, b = 0;
+            if (gs % EPL == 0) {
+                // all of this lane's experts sit in group e0 / gs
+                if (!((kept >> (e0 / gs)) & 1u)) a = b = 0u;
+            } else {
 #pragma unroll
                 for (int j = 0; j < EPL; ++j) {
-                    uint32_t k = key[j];
-                    if (k > a) {
-                        b = a;
-                        a = k;
-                    } else if (k > b) {
-                        b = k;
-                    }
+                    const int e = e0 + j;
+                    if (e < p.E && !((kept >> (e / gs)) & 1u)) key[j] = 0u;
                 }
-                top2_merge(a, b, lpg);
-                double s = sigmoid_d((double)key_value(a)) + sigmoid_d((double)key_value(b));
-                // group g's score sits on lane g*lpg; move it to lane g
-                int src = (lane < p.G) ? lane * lpg : 0;
-                double sg = __shfl_sync(FULL, s, src);
-                if (lane < p.G) score = sg;
-            } else {
-                // generic: one warp-wide top-2 per group
-                for (int grp = 0; grp < p.G; ++grp) {
-                    uint32_t a = 0, b = 0;
-#pragma unroll
-                    for (int j = 0; j < EPL; ++j) {
-                        int e = e0 + j;
-                        uint32_t k = (e < p.E && e / gs == grp) ? key[j] : 0u;
-                        if (k > a) {
-                            b = a;
-                            a = k;
-                        } else if (k > b) {
-                            b = k;
-                        }
-                    }
-                    top2_merge(a, b, 32);
-                    if (lane == grp)
-                        score = sigmoid_d((double)key_value(a)) + sigmoid_d((double)key_value(b));
-                }
-            }
-            // keep the KG best groups: rank = groups strictly better (ties: lower id)
-            int rank = 0;
-            for (int h = 0; h < p.G; ++h) {
-                double sh = __shfl_sync(FULL, score, h);
-                if (lane < p.G && (sh > score || (sh == score && h < lane))) ++rank;
-            }
-            const uint32_t kept = __ballot_sync(FULL, lane < p.G && rank < p.KG);
-#pragma unroll
-            for (int j = 0; j < EPL; ++j) {
-                int e = e0 + j;
-                if (e < p.E && !((kept >> (e / gs)) & 1u)) key[j] = 0u;
+                top2_of<EPL>(key, 0u, a, pa, b, pb);
             }
         }
 
-        // top-K: K rounds of warp argmax on (value desc, expert id asc)
+        // top-K: K rounds of warp argmax on (logit desc, expert id asc)
         uint32_t top_key = 0;
+        uint32_t my_key = 0;
         for (int k = 0; k < p.K; ++k) {
-            uint32_t lk = 0;
-            int lj = 0;
-#pragma unroll
-            for (int j = 0; j < EPL; ++j) {
-                if (key[j] > lk) {  // strict: equal keys keep the lower id
-                    lk = key[j];
-                    lj = j;
-                }
-            }
-            const uint32_t wk = __reduce_max_sync(FULL, lk);
-            const uint32_t cand = (lk == wk && lk != 0u) ? (0xffffffffu - (uint32_t)(e0 + lj)) : 0u;
+            const uint32_t wk = __reduce_max_sync(FULL, a);
+            const uint32_t cand = (a == wk && a != 0u) ? ~(uint32_t)(e0 + pa) : 0u;
             const uint32_t wc = __reduce_max_sync(FULL, cand);
-            const int e = (int)(0xffffffffu - wc);
             if (k == 0) top_key = wk;
-            if (e0 <= e && e < e0 + EPL) {
-#pragma unroll
-                for (int j = 0; j < EPL; ++j)
-                    if (e0 + j == e) key[j] = 0u;
-            }
             if (lane == k) {
-                my_e = (wk != 0u) ? e : -1;
-                my_w = key_value(wk);  // the logit, for the weight below
+                my_e = (wk != 0u) ? (int)~wc : -1;
+                my_key = wk;
+            }
+            if (cand != 0u && cand == wc) {  // this lane's head won: pop it
+                taken |= 1u << pa;
+                a = b;
+                pa = pb;
+                b = 0u;
+                if (a == 0u) top2_of<EPL>(key, taken, a, pa, b, pb);
             }
         }
+        const float my_logit = key_value(my_key);
 
         // weights, fp64
         double wt = 0.0;
         if (p.route == EP_ROUTE_GROUP_SIGMOID) {
-            double s = (lane < p.K && my_e >= 0) ? sigmoid_d((double)my_w) : 0.0;
+            const double s = (lane < p.K && my_e >= 0) ? sigmoid_d((double)my_logit) : 0.0;
             double sum = 0.0;
             for (int k = 0; k < p.K; ++k) sum += __shfl_sync(FULL, s, k);
             wt = s / sum;
@@ -204,11 +300,11 @@ __device__ __forceinline__ void route_token(const LayoutParams& p, int64_t g, in
             const double mx = (double)key_value(top_key);
             double z = 0.0;
 #pragma unroll
-            for (int j = 0; j < EPL; ++j)
-                if (e0 + j < p.E) z += exp((double)v[j] - mx);
+            for (int j = 0; j < EPL; ++j)  // softmax routes never zero keys: key j is logit j
+                if (key[j] != 0u) z += exp((double)key_value(key[j]) - mx);
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(FULL, z, off);
-            double pk = (lane < p.K && my_e >= 0) ? exp((double)my_w - mx) / z : 0.0;
+            const double pk = (lane < p.K && my_e >= 0) ? exp((double)my_logit - mx) / z : 0.0;
             if (p.route == EP_ROUTE_SOFTMAX_RENORM) {
                 double sum = 0.0;
                 for (int k = 0; k < p.K; ++k) sum += __shfl_sync(FULL, pk, k);
@@ -221,7 +317,7 @@ __device__ __forceinline__ void route_token(const LayoutParams& p, int64_t g, in
     }
     // slot mask
     if (lane < p.K && p.mask_thr != 0ull) {
-        uint64_t h = splitmix64(p.mask_seed ^ (uint64_t)(g * p.K + lane));
+        const uint64_t h = splitmix64(p.mask_seed ^ (uint64_t)(g * p.K + lane));
         if ((h >> 32) < p.mask_thr) {
             my_e = -1;
             my_w = 0.0f;
@@ -229,85 +325,8 @@ __device__ __forceinline__ void route_token(const LayoutParams& p, int64_t g, in
     }
 }
 
-template <int EPL>
-__global__ void __launch_bounds__(kRouteWarps * 32) route_count_kernel(LayoutParams p) {
-    extern __shared__ int hist[];  // [J]
-    const int c = blockIdx.x;
-    const int s = c / p.ncpr;
-    const int t0 = (c % p.ncpr) * p.ch;
-    const int t1 = min(p.T, t0 + p.ch);
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    for (int j = threadIdx.x; j < p.J; j += blockDim.x) hist[j] = 0;
-    __syncthreads();
-    for (int t = t0 + warp; t < t1; t += kRouteWarps) {
-        const int64_t g = (int64_t)s * p.T + t;
-        int e;
-        float w;
-        route_token<EPL>(p, g, lane, e, w);
-        if (lane < p.K) {
-            p.topk_idx[g * p.K + lane] = e;
-            p.topk_w[g * p.K + lane] = w;
-            if (e >= 0) atomicAdd(&hist[e], 1);
-        }
-        const uint32_t ranks = __reduce_or_sync(FULL, (lane < p.K && e >= 0) ? (1u << (e / p.L)) : 0u);
-        if (lane < p.R) {
-            const uint32_t in = (ranks >> lane) & 1u;
-            p.itr[g * p.R + lane] = (uint8_t)in;
-            if (in) atomicAdd(&hist[p.E + lane], 1);
-        }
-    }
-    __syncthreads();
-    int32_t* out = p.chunk + (int64_t)c * p.J;
-    for (int j = threadIdx.x; j < p.J; j += blockDim.x) out[j] = hist[j];
-}
-
-// Block (32 x 32): x = column within a 32-column tile, y = segment of chunks.
-__global__ void __launch_bounds__(1024) chunk_scan_kernel(LayoutParams p) {
-    __shared__ int part[32][33];
-    const int tx = threadIdx.x, ty = threadIdx.y;
-    const int col = blockIdx.x * 32 + tx;
-    const int per = (p.nc + 31) / 32;
-    const int c0 = min(p.nc, ty * per);
-    const int c1 = min(p.nc, c0 + per);
-    int sum = 0;
-    if (col < p.J) {
-        for (int c = c0; c < c1; ++c) sum += p.chunk[(int64_t)c * p.J + col];
-    }
-    part[ty][tx] = sum;
-    __syncthreads();
-    {
-        // warp ty scans column ty over the 32 segments
-        const int lane = tx;
-        const int v = part[lane][ty];
-        int incl = v;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            int o = __shfl_up_sync(FULL, incl, off);
-            if (lane >= off) incl += o;
-        }
-        __syncthreads();
-        part[lane][ty] = incl - v;  // exclusive offset of segment `lane`
-        const int c2 = blockIdx.x * 32 + ty;
-        if (lane == 31 && c2 < p.J) p.pref[(int64_t)c2 * (p.R + 1) + p.R] = incl;  // column total
-    }
-    __syncthreads();
-    if (col < p.J) {
-        int run = part[ty][tx];
-        for (int c = c0; c < c1; ++c) {
-            const int64_t i = (int64_t)c * p.J + col;
-            const int x = p.chunk[i];
-            p.chunk[i] = run;
-            if (c % p.ncpr == 0) p.pref[(int64_t)col * (p.R + 1) + c / p.ncpr] = run;
-            run += x;
-        }
-        if (p.nc == 0 && ty == 0)
-            for (int r = 0; r < p.R; ++r) p.pref[(int64_t)col * (p.R + 1) + r] = 0;
-    }
-}
-
-// Exclusive scan of n <= 4 * blockDim.x values from `in` into out[0..n],
-// with out[n] = total. All threads of the block must call it.
+// Exclusive scan of n <= 4 * blockDim.x values in[j * stride] into out[0..n],
+// with out[n] = total. Called by every thread of the block.
 __device__ void block_exclusive_scan(const int32_t* in, int stride, int n, int* out, int* warp_tot) {
     const int t = threadIdx.x;
     const int lane = t & 31, warp = t >> 5, nw = blockDim.x >> 5;
@@ -322,17 +341,17 @@ __device__ void block_exclusive_scan(const int32_t* in, int stride, int n, int* 
     int incl = local;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        int o = __shfl_up_sync(FULL, incl, off);
+        const int o = __shfl_up_sync(FULL, incl, off);
         if (lane >= off) incl += o;
     }
     if (lane == 31) warp_tot[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        int wv = (lane < nw) ? warp_tot[lane] : 0;
+        const int wv = (lane < nw) ? warp_tot[lane] : 0;
         int wi = wv;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-            int o = __shfl_up_sync(FULL, wi, off);
+            const int o = __shfl_up_sync(FULL, wi, off);
             if (lane >= off) wi += o;
         }
         if (lane < nw) warp_tot[lane] = wi - wv;
@@ -350,160 +369,228 @@ __device__ void block_exclusive_scan(const int32_t* in, int stride, int n, int* 
     __syncthreads();
 }
 
-__global__ void __launch_bounds__(kAssignThreads) assign_rows_kernel(LayoutParams p) {
+template <int EPL>
+__global__ void __launch_bounds__(kThreads, 2) layout_kernel(LayoutParams p) {
     extern __shared__ int sm[];
-    int* eoff = sm;                 // [E + 1]
-    int* base = sm + p.E + 1;       // [E]
+    int* hist = sm;                      // [kWarps][J]: per-warp counts, later per-warp row bases
+    int* eoff = sm + kWarps * p.J;       // [max(E, nc) + 1]: scan output
     __shared__ int warp_tot[33];
-    const int R1 = p.R + 1;
-    // expert totals are the column totals of the first E columns
-    block_exclusive_scan(p.pref + p.R, R1, p.E, eoff, warp_tot);
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int c = blockIdx.x;
+    const bool has_chunk = c < p.nc;
+    int s = 0, t0 = 0, t1 = 0, w0 = 0, w1 = 0;
+    if (has_chunk) {
+        s = c / p.ncpr;
+        const int j = c % p.ncpr;
+        t0 = (int)((int64_t)j * p.T / p.ncpr);
+        t1 = (int)((int64_t)(j + 1) * p.T / p.ncpr);
+        const int n = t1 - t0;
+        w0 = t0 + warp * n / kWarps;
+        w1 = t0 + (warp + 1) * n / kWarps;
+    }
 
-    if (blockIdx.x == 0) {
-        for (int e = threadIdx.x; e <= p.E; e += blockDim.x) p.expert_off[e] = eoff[e];
-        for (int r = threadIdx.x; r <= p.R; r += blockDim.x) p.rank_off[r] = eoff[r * p.L];
-        for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
-            const int32_t* pe = p.pref + (int64_t)e * R1;
-            p.ntpe[e] = pe[p.R];
-            for (int s = 0; s < p.R; ++s) {
-                p.src_off[(int64_t)e * p.R + s] = pe[s];
-                p.cnt[(int64_t)s * p.E + e] = pe[s + 1] - pe[s];
-            }
+    // ---- phase 1: route; per-warp expert and rank histograms
+    for (int i = threadIdx.x; i < kWarps * p.J; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    int* my_hist = hist + warp * p.J;
+    float vnext[EPL];
+    if (p.logits != nullptr && w0 < w1) load_logits<EPL>(p, (int64_t)s * p.T + w0, lane, vnext);
+    for (int t = w0; t < w1; ++t) {
+        const int64_t g = (int64_t)s * p.T + t;
+        float vcur[EPL];
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) vcur[j] = vnext[j];
+        if (p.logits != nullptr && t + 1 < w1) load_logits<EPL>(p, g + 1, lane, vnext);  // prefetch
+        int e;
+        float w;
+        route_token<EPL>(p, g, lane, vcur, e, w);
+        if (lane < p.K) {
+            p.topk_idx[g * p.K + lane] = e;
+            p.topk_w[g * p.K + lane] = w;
+            if (e >= 0) atomicAdd(&my_hist[e], 1);
         }
-        for (int i = threadIdx.x; i < p.R * p.R; i += blockDim.x) {
-            const int s = i / p.R, r = i % p.R;
-            const int32_t* pr = p.pref + (int64_t)(p.E + r) * R1;
-            p.ntpr[i] = pr[s + 1] - pr[s];
+        const uint32_t ranks =
+            __reduce_or_sync(FULL, (lane < p.K && e >= 0)
+                                       ? (1u << (p.L == 1 ? (uint32_t)e : __umulhi((uint32_t)e, p.l_magic)))
+                                       : 0u);
+        if (lane < p.R) {
+            const uint32_t in = (ranks >> lane) & 1u;
+            p.itr[g * p.R + lane] = (uint8_t)in;
+            my_hist[p.E + lane] += (int)in;
         }
     }
-    if (p.nc == 0) return;
-
-    const int c = blockIdx.x;
-    const int s = c / p.ncpr;
-    const int t0 = (c % p.ncpr) * p.ch;
-    const int t1 = min(p.T, t0 + p.ch);
-    const int32_t* cpre = p.chunk + (int64_t)c * p.J;
-    for (int e = threadIdx.x; e < p.E; e += blockDim.x) base[e] = eoff[e] + cpre[e];
     __syncthreads();
-    if (threadIdx.x >= 32) return;
-
-    const int lane = threadIdx.x;
-    const unsigned lt = (1u << lane) - 1u;
-    const int64_t slot0 = ((int64_t)s * p.T + t0) * p.K;
-    const int nslots = (t1 - t0) * p.K;
-    for (int i0 = 0; i0 < nslots; i0 += 32) {
-        const int j = i0 + lane;
-        const bool active = j < nslots;
-        const int e = active ? p.topk_idx[slot0 + j] : -1;
-        const bool valid = e >= 0;
-        const unsigned peers = __match_any_sync(FULL, valid ? e : -1);
-        if (active) {
-            int32_t row = -1;
-            if (valid) {
-                const int64_t r = (int64_t)base[e] + __popc(peers & lt);
-                if (r < p.m_max) {
-                    row = (int32_t)r;
-                } else {
-                    set_error(p.err, EP_DEVERR_ROW_BOUNDS);
-                }
-            }
-            p.dst_row[slot0 + j] = row;
+    if (has_chunk) {
+        for (int j = threadIdx.x; j < p.J; j += kThreads) {
+            int sum = 0;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) sum += hist[w * p.J + j];
+            p.chunk[(int64_t)j * p.nc + c] = sum;
         }
-        __syncwarp();
-        if (valid && (peers >> lane) == 1u) base[e] += __popc(peers);  // highest lane of the group
-        __syncwarp();
+    }
+    grid_barrier(p.bar, (uint32_t)p.nb, p.err);
+
+    // ---- phase 2: per-column exclusive scan over chunks (one CTA per column)
+    for (int col = blockIdx.x; col < p.J; col += p.nb) {
+        int32_t* colp = p.chunk + (int64_t)col * p.nc;
+        block_exclusive_scan(colp, 1, p.nc, eoff, warp_tot);  // eoff: scratch here, [nc + 1]
+        for (int cc = threadIdx.x; cc < p.nc; cc += kThreads) colp[cc] = eoff[cc];
+        // prefix at each rank's first chunk; eoff[nc] is the column total
+        if (threadIdx.x < p.R) {
+            const int r = threadIdx.x;
+            const int a = (p.nc > 0) ? eoff[r * p.ncpr] : 0;
+            const int b = (p.nc > 0) ? eoff[(r + 1) * p.ncpr] : 0;  // (R * ncpr = nc) -> total
+            if (col < p.E) {
+                p.src_off[(int64_t)col * p.R + r] = a;
+                p.cnt[(int64_t)r * p.E + col] = b - a;
+            } else {
+                p.ntpr[(int64_t)r * p.R + (col - p.E)] = b - a;
+            }
+        }
+        if (threadIdx.x == 0) {
+            const int total = (p.nc > 0) ? eoff[p.nc] : 0;
+            p.tot[col] = total;
+            if (col < p.E) p.ntpe[col] = total;
+        }
+        __syncthreads();
+    }
+    grid_barrier(p.bar, 2u * (uint32_t)p.nb, p.err);
+
+    // ---- phase 3: expert offsets, per-warp bases, row placement
+    block_exclusive_scan(p.tot, 1, p.E, eoff, warp_tot);
+    if (blockIdx.x == 0) {
+        for (int e = threadIdx.x; e <= p.E; e += kThreads) p.expert_off[e] = eoff[e];
+        for (int r = threadIdx.x; r <= p.R; r += kThreads) p.rank_off[r] = eoff[r * p.L];
+    }
+    if (has_chunk) {
+        for (int e = threadIdx.x; e < p.E; e += kThreads) {
+            int run = eoff[e] + p.chunk[(int64_t)e * p.nc + c];
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) {
+                const int x = hist[w * p.J + e];
+                hist[w * p.J + e] = run;
+                run += x;
+            }
+        }
+        __syncthreads();
+        const unsigned lt = (1u << lane) - 1u;
+        const int64_t slot0 = ((int64_t)s * p.T + w0) * p.K;
+        const int nslots = (w1 - w0) * p.K;
+        for (int i0 = 0; i0 < nslots; i0 += 32) {
+            const int j = i0 + lane;
+            const bool active = j < nslots;
+            const int e = active ? p.topk_idx[slot0 + j] : -1;
+            const bool valid = e >= 0;
+            const unsigned peers = __match_any_sync(FULL, valid ? e : -1);
+            if (active) {
+                int32_t row = -1;
+                if (valid) {
+                    const int64_t r = (int64_t)my_hist[e] + __popc(peers & lt);
+                    if (r < p.m_max) row = (int32_t)r;
+                    else set_error(p.err, EP_DEVERR_ROW_BOUNDS);
+                }
+                p.dst_row[slot0 + j] = row;
+            }
+            __syncwarp();
+            if (valid && (peers >> lane) == 1u) my_hist[e] += __popc(peers);  // highest lane of the group
+            __syncwarp();
+        }
+    }
+
+    // the last CTA out resets the barrier words for the next launch
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(p.bar + 1, 1u) == (uint32_t)p.nb - 1u) {
+            p.bar[0] = 0u;
+            p.bar[1] = 0u;
+            __threadfence();
+        }
     }
 }
 
+// Resident CTAs per SM for each kernel instantiation and shared-memory size
+// (the occupancy query is a host-side cost worth skipping per call).
+struct OccCache {
+    std::mutex mu;
+    const void* fn[32] = {};
+    size_t smem[32] = {};
+    int dev[32] = {};
+    int per_sm[32] = {};
+    int n = 0;
+};
+OccCache g_occ;
+
+cudaError_t occupancy(const void* fn, size_t smem, int dev, int* per_sm) {
+    std::lock_guard<std::mutex> lock(g_occ.mu);
+    for (int i = 0; i < g_occ.n; ++i)
+        if (g_occ.fn[i] == fn && g_occ.smem[i] == smem && g_occ.dev[i] == dev) {
+            *per_sm = g_occ.per_sm[i];
+            return cudaSuccess;
+        }
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, fn, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (g_occ.n < 32) {
+        g_occ.fn[g_occ.n] = fn;
+        g_occ.smem[g_occ.n] = smem;
+        g_occ.dev[g_occ.n] = dev;
+        g_occ.per_sm[g_occ.n] = *per_sm;
+        ++g_occ.n;
+    }
+    return cudaSuccess;
+}
+
 template <int EPL>
-cudaError_t launch_route(const LayoutParams& p, cudaStream_t st) {
-    const size_t smem = sizeof(int) * p.J;
-    route_count_kernel<EPL><<<p.nc, kRouteWarps * 32, smem, st>>>(p);
+cudaError_t launch_epl(LayoutParams& p, int dev, int sm_count, int max_ctas, cudaStream_t st) {
+    auto kern = layout_kernel<EPL>;
+    const int scan_n = (p.E > max_ctas) ? p.E : max_ctas;
+    const size_t smem = sizeof(int) * ((size_t)kWarps * p.J + scan_n + 1);
+    if (smem > 48 * 1024) return cudaErrorInvalidConfiguration;
+    int per_sm = 0;
+    cudaError_t e = occupancy((const void*)kern, smem, dev, &per_sm);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    int nb = per_sm * sm_count;
+    if (nb > max_ctas) nb = max_ctas;
+    // small batches: about one token per warp, so the grid barriers stay cheap
+    const int64_t want = ((int64_t)p.R * p.T + kWarps - 1) / kWarps;
+    if (want < nb) nb = (int)(want > p.R ? want : p.R);
+    if (nb < p.R) return cudaErrorInvalidConfiguration;  // every rank needs a chunk
+    p.nb = nb;
+    int ncpr = nb / p.R;
+    if (ncpr > p.T) ncpr = p.T;
+    p.ncpr = ncpr > 0 ? ncpr : 1;
+    p.nc = (p.T > 0) ? p.R * ncpr : 0;
+    void* args[] = {&p};
+    e = cudaLaunchCooperativeKernel((const void*)kern, dim3(nb), dim3(kThreads), args, smem, st);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 }  // namespace
 
-int layout_chunk_tokens(int64_t n_tokens) {
-    int ch = 32;
-    while ((n_tokens + ch - 1) / ch > 1024) ch *= 2;
-    return ch;
-}
-
-cudaError_t launch_layout(const ep_buffer& b, const LayoutArgs& a, cudaStream_t st) {
-    const ep_config_t& c = b.cfg;
-    LayoutParams p{};
-    p.R = c.num_ranks;
-    p.T = a.T;
-    p.E = c.num_experts;
-    p.K = c.topk;
-    p.L = c.num_experts / c.num_ranks;
-    p.G = c.num_groups;
-    p.KG = c.topk_groups;
-    p.ch = layout_chunk_tokens((int64_t)p.R * p.T);
-    p.ncpr = (p.T + p.ch - 1) / p.ch;
-    p.nc = p.R * p.ncpr;
-    p.J = p.E + p.R;
-    p.route = a.route;
-    p.logits = a.logits;
-    p.vec_logits = (a.logits != nullptr && (p.E % 4 == 0) && ((uintptr_t)a.logits % 16 == 0)) ? 1 : 0;
-    p.in_idx = a.in_idx;
-    p.in_w = a.in_w;
-    p.mask_seed = a.mask_seed;
-    p.mask_thr = a.mask_threshold;
-    p.topk_idx = b.topk_idx;
-    p.topk_w = b.topk_w;
-    p.itr = b.is_token_in_rank;
-    p.chunk = b.chunk;
-    p.pref = b.pref;
-    p.ntpr = b.num_tokens_per_rank;
-    p.cnt = b.cnt;
-    p.ntpe = b.num_tokens_per_expert;
-    p.expert_off = b.expert_off;
-    p.rank_off = b.rank_off;
-    p.src_off = b.src_off;
-    p.dst_row = b.dst_row;
-    p.m_max = b.m_max;
-    p.err = b.err;
-
-    cudaError_t e = cudaSuccess;
-    if (p.nc > 0) {
-        const int epl = (p.E + 31) / 32;
-        if (epl <= 1) e = launch_route<1>(p, st);
-        else if (epl <= 2) e = launch_route<2>(p, st);
-        else if (epl <= 4) e = launch_route<4>(p, st);
-        else if (epl <= 8) e = launch_route<8>(p, st);
-        else if (epl <= 16) e = launch_route<16>(p, st);
-        else e = launch_route<32>(p, st);
-        if (e != cudaSuccess) return e;
-    }
-    chunk_scan_kernel<<<(p.J + 31) / 32, dim3(32, 32), 0, st>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const size_t smem = sizeof(int) * (2 * p.E + 1);
-    assign_rows_kernel<<<p.nc > 0 ? p.nc : 1, kAssignThreads, smem, st>>>(p);
-    return cudaGetLastError();
-}
-
-int64_t layout_scratch_ints(const ep_config_t& c, int T) {
-    const int ch = layout_chunk_tokens((int64_t)c.num_ranks * T);
-    const int64_t nc = (int64_t)c.num_ranks * ((T + ch - 1) / ch);
+int64_t layout_scratch_ints(const ep_config_t& c, int max_ctas) {
     const int64_t J = (int64_t)c.num_experts + c.num_ranks;
-    return nc * J + J * (c.num_ranks + 1);
+    return kLayoutControlInts + J * max_ctas + J;
 }
 
 cudaError_t launch_layout_raw(const ep_config_t& c, const LayoutArgs& a, const ep_layout_t& out,
-                              int32_t* scratch, uint32_t* err, cudaStream_t st) {
+                              int32_t* scratch, int max_ctas, uint32_t* err, cudaStream_t st) {
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
     LayoutParams p{};
     p.R = c.num_ranks;
     p.T = a.T;
     p.E = c.num_experts;
     p.K = c.topk;
     p.L = c.num_experts / c.num_ranks;
+    // ceil(2^32 / L): exact quotients for e < 2^16 since 2 <= L <= 1024 (L == 1 is e itself)
+    p.l_magic = p.L > 1 ? (uint32_t)((((uint64_t)1 << 32) + (uint64_t)p.L - 1) / (uint64_t)p.L) : 0u;
     p.G = c.num_groups;
     p.KG = c.topk_groups;
-    p.ch = layout_chunk_tokens((int64_t)p.R * p.T);
-    p.ncpr = (p.T + p.ch - 1) / p.ch;
-    p.nc = p.R * p.ncpr;
     p.J = p.E + p.R;
     p.route = a.route;
     p.logits = a.logits;
@@ -515,8 +602,6 @@ cudaError_t launch_layout_raw(const ep_config_t& c, const LayoutArgs& a, const e
     p.topk_idx = out.topk_idx;
     p.topk_w = out.topk_w;
     p.itr = out.is_token_in_rank;
-    p.chunk = scratch;
-    p.pref = scratch + (int64_t)p.nc * p.J;
     p.ntpr = out.num_tokens_per_rank;
     p.cnt = out.cnt_src_expert;
     p.ntpe = out.num_tokens_per_expert;
@@ -524,25 +609,36 @@ cudaError_t launch_layout_raw(const ep_config_t& c, const LayoutArgs& a, const e
     p.rank_off = out.rank_off;
     p.src_off = out.src_off;
     p.dst_row = out.dst_row;
-    p.m_max = (int64_t)p.R * p.T * p.K;  // no receive buffer: rows of this call only
+    p.m_max = a.m_max;
     p.err = err;
+    // scratch: [control][chunk J*max_ctas][tot J]
+    p.bar = reinterpret_cast<uint32_t*>(scratch);
+    p.chunk = scratch + kLayoutControlInts;
+    p.tot = p.chunk + (int64_t)p.J * max_ctas;
+    const int epl = (p.E + 31) / 32;
+    if (epl <= 1) return launch_epl<1>(p, dev, sms, max_ctas, st);
+    if (epl <= 2) return launch_epl<2>(p, dev, sms, max_ctas, st);
+    if (epl <= 4) return launch_epl<4>(p, dev, sms, max_ctas, st);
+    if (epl <= 8) return launch_epl<8>(p, dev, sms, max_ctas, st);
+    if (epl <= 16) return launch_epl<16>(p, dev, sms, max_ctas, st);
+    return launch_epl<32>(p, dev, sms, max_ctas, st);
+}
 
-    cudaError_t e = cudaSuccess;
-    if (p.nc > 0) {
-        const int epl = (p.E + 31) / 32;
-        if (epl <= 1) e = launch_route<1>(p, st);
-        else if (epl <= 2) e = launch_route<2>(p, st);
-        else if (epl <= 4) e = launch_route<4>(p, st);
-        else if (epl <= 8) e = launch_route<8>(p, st);
-        else if (epl <= 16) e = launch_route<16>(p, st);
-        else e = launch_route<32>(p, st);
-        if (e != cudaSuccess) return e;
-    }
-    chunk_scan_kernel<<<(p.J + 31) / 32, dim3(32, 32), 0, st>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const size_t smem = sizeof(int) * (2 * p.E + 1);
-    assign_rows_kernel<<<p.nc > 0 ? p.nc : 1, kAssignThreads, smem, st>>>(p);
-    return cudaGetLastError();
+cudaError_t launch_layout(const ep_buffer& b, const LayoutArgs& a, cudaStream_t st) {
+    ep_layout_t out;
+    out.topk_idx = b.topk_idx;
+    out.topk_w = b.topk_w;
+    out.is_token_in_rank = b.is_token_in_rank;
+    out.num_tokens_per_rank = b.num_tokens_per_rank;
+    out.cnt_src_expert = b.cnt;
+    out.num_tokens_per_expert = b.num_tokens_per_expert;
+    out.expert_off = b.expert_off;
+    out.rank_off = b.rank_off;
+    out.src_off = b.src_off;
+    out.dst_row = b.dst_row;
+    LayoutArgs aa = a;
+    aa.m_max = b.m_max;
+    return launch_layout_raw(b.cfg, aa, out, b.scratch, kMaxLayoutCtas, b.err, st);
 }
 
 }  // namespace ep

@@ -4,16 +4,17 @@
 // not call cudaMalloc (or any allocator) after start-up. Such a caller has
 // its input and output tensors but no way to get a workspace.
 //
-// The only scratch the layout kernels need is the per-chunk counts and their
-// prefix sums. Here that scratch lives in the file-scope device array below,
-// so this entry point allocates nothing: no cudaMalloc, cudaFree or allocating
-// library routine.
+// The only scratch the layout kernel needs is two grid-barrier counters plus
+// the per-chunk counts and their prefix sums. Here that scratch lives in the
+// file-scope device array below, so this entry point allocates nothing: no
+// cudaMalloc, cudaFree or allocating library routine.
 //
 // Shared scratch: every call on a device uses the same array, and it keeps
-// whatever the last call left in it. The kernels overwrite every scratch entry
-// they read within the call, so nothing needs clearing. Calls whose work
-// overlaps on the GPU (two streams, or two host threads) race on the array
-// and give wrong layouts. Order them on one stream. Every GPU that loads
+// whatever the last call left in it. Each call zeroes the barrier counters
+// (a stream-ordered memset of 256 bytes). The kernel overwrites every other
+// entry it reads within the call. Calls whose work overlaps on the GPU (two
+// streams, or two host threads) race on the array and give wrong layouts.
+// Order them on one stream. Every GPU that loads
 // this library holds the array (2 MiB) until the process exits.
 #include <cuda_runtime.h>
 #include <math.h>
@@ -27,8 +28,9 @@
 
 namespace {
 
-// 2 MiB: enough for 1024 chunks x (256 experts + 8 ranks), i.e. the prefill
-// and large workloads (E = 256, R = 8) at any T.
+// 2 MiB. The layout grid is capped so its chunk scratch fits:
+// (2 MiB/4 - 64 - (E+R)(R+2)) / (E+R) CTAs, e.g. all 1024 at E = 256, R = 8,
+// and about 460 at E = 1024, R = 32.
 constexpr int64_t kNoAllocScratchInts = (2 << 20) / 4;
 
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchInts];
@@ -84,10 +86,9 @@ extern "C" ep_status_t ep_get_layout_noalloc(const ep_config_t* cfg, int T, cons
     if (have_logits && (route < EP_ROUTE_SOFTMAX || route > EP_ROUTE_GROUP_SIGMOID))
         return fail(EP_ERR_INVALID, "unknown route");
     if (!(mask_frac >= 0.0f && mask_frac <= 1.0f)) return fail(EP_ERR_INVALID, "mask_frac must be in [0, 1]");
-    if (ep::layout_scratch_ints(*cfg, T) > kNoAllocScratchInts)
-        return fail(EP_ERR_CAPACITY,
-                    "layout scratch for this config and T exceeds the 2 MiB static scratch of "
-                    "ep_get_layout_noalloc; use ep_get_layout with a workspace");
+    const int64_t J = (int64_t)cfg->num_experts + cfg->num_ranks;
+    int64_t max_ctas = (kNoAllocScratchInts - ep::layout_scratch_ints(*cfg, 0)) / J;
+    if (max_ctas > ep::kMaxLayoutCtas) max_ctas = ep::kMaxLayoutCtas;
 
     int32_t* scratch = nullptr;
     cudaError_t e = scratch_for_current_device(&scratch);
@@ -104,7 +105,12 @@ extern "C" ep_status_t ep_get_layout_noalloc(const ep_config_t* cfg, int T, cons
     a.route = route;
     a.mask_seed = mask_seed;
     a.mask_threshold = (uint64_t)floor((double)mask_frac * 4294967296.0);
-    e = ep::launch_layout_raw(*cfg, a, *out, scratch, d_error_word, static_cast<cudaStream_t>(stream));
+    a.m_max = (int64_t)cfg->num_ranks * T * cfg->topk;  // no receive buffer: this call's rows
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    // zero the barrier words first: a call that timed out may have left them set
+    e = cudaMemsetAsync(scratch, 0, sizeof(int32_t) * ep::kLayoutControlInts, cs);
+    if (e == cudaSuccess)
+        e = ep::launch_layout_raw(*cfg, a, *out, scratch, (int)max_ctas, d_error_word, cs);
     if (e != cudaSuccess) {
         char m[200];
         snprintf(m, sizeof m, "layout launch: %s", cudaGetErrorString(e));

@@ -169,7 +169,7 @@ ep_status_t ep_get_layout(ep_buffer_t *buf, int T, const float *d_logits,
  *  - amax = max(max|x|, 1e-4);
  *  - q = e4m3_rne_satfinite(x * (448/amax));
  *  - recv_scale = amax/448.
- * d_x: bf16 [N, H] row-major, 16-byte aligned. T must equal the T of the
+ * d_x: bf16 [N, H] row-major, 32-byte aligned. T must equal the T of the
  * last ep_get_layout on this buffer. Errors: EP_ERR_INVALID. */
 ep_status_t ep_dispatch(ep_buffer_t *buf, int T, const void *d_x, void *stream);
 
@@ -178,14 +178,15 @@ ep_status_t ep_dispatch(ep_buffer_t *buf, int T, const void *d_x, void *stream);
  * accumulated in fp32 with one fused multiply-add per slot. d_y_scale == NULL:
  * d_y is bf16 [rows, H]. Otherwise d_y is e4m3 [rows, H] and is dequantised
  * in the kernel as e4m3 * d_y_scale[row, h/128] (fp32) before the fma.
- * rows >= expert_off[E]. d_out: bf16 [N, H]. All pointers 16-byte aligned.
+ * rows >= expert_off[E]. d_out: bf16 [N, H]. d_y and d_out 32-byte aligned.
  * T must equal the T of the last ep_get_layout. A token whose slots are all
  * masked gets +0. Errors: EP_ERR_INVALID. */
 ep_status_t ep_combine(ep_buffer_t *buf, int T, const void *d_y, const float *d_y_scale,
                        void *d_out, void *stream);
 
 /* Synchronises `stream` and reads the device error word into *word. clear != 0
- * then resets it to 0. Returns EP_ERR_DEVICE if any bit was set, EP_OK if
+ * then resets it to 0, together with the layout's grid-barrier words. After
+ * EP_DEVERR_TIMEOUT, call it with clear != 0 before the next ep_get_layout. Returns EP_ERR_DEVICE if any bit was set, EP_OK if
  * none, EP_ERR_CUDA on a CUDA failure. */
 ep_status_t ep_check_errors(ep_buffer_t *buf, uint32_t *word, int clear, void *stream);
 
@@ -198,14 +199,14 @@ ep_status_t ep_check_errors(ep_buffer_t *buf, uint32_t *word, int clear, void *s
  * Computes exactly what ep_get_layout computes, with the same inputs and
  * meaning. The outputs go to the caller's device arrays in *out, a host
  * struct of device pointers, every one required, sized for N = R*T as
- * ep_layout_t lists. The layout's scratch (per-chunk counts and their prefix
- * sums) lives in a file-scope device array of 2 MiB that every GPU loading
- * the library holds until exit. The call makes no cudaMalloc, cudaFree or
- * other allocating call.
- *  - Limit: R*ceil(T/ch)*(E+R) + (E+R)*(R+1) int32 scratch entries must fit
- *    in 2 MiB, where ch is the chunk size (32 tokens, doubled until there are
- *    at most 1024 chunks). E = 256 and R = 8 fit for any T. Beyond it the
- *    call returns EP_ERR_CAPACITY and launches nothing.
+ * ep_layout_t lists. The layout's scratch lives in a file-scope device array
+ * of 2 MiB that every GPU loading the library holds until exit: two barrier
+ * counters, plus the per-chunk counts and their prefix sums. The call makes no
+ * cudaMalloc, cudaFree or other allocating call.
+ *  - Limit: the 2 MiB bound the layout grid (one CTA per chunk) to
+ *    (524288 - 64 - (E+R)(R+2)) / (E+R) CTAs, at most 1024. All 1024 fit at
+ *    E = 256, R = 8, and about 460 at E = 1024, R = 32. No valid config is
+ *    rejected; a smaller grid only means longer chunks.
  *  - d_error_word: a device uint32 that receives EP_DEVERR_* bits with
  *    atomicOr. The caller zeroes and reads it.
  *  - Runs on the current device. `stream` must belong to it.
@@ -213,9 +214,11 @@ ep_status_t ep_check_errors(ep_buffer_t *buf, uint32_t *word, int clear, void *s
  *    the static scratch (cudaGetSymbolAddress). Make that first call before
  *    any stream capture.
  *  - Every call on a device shares the one scratch array and leaves its
- *    contents behind. The kernels rewrite every entry they read, so nothing
- *    needs clearing, but calls whose GPU work overlaps (different streams or
- *    host threads) race and give wrong results.
+ *    contents behind. Each call first zeroes the barrier counters with a
+ *    stream-ordered cudaMemsetAsync of 256 bytes (not an allocation). The
+ *    kernel rewrites every other entry it reads. Calls whose GPU work
+ *    overlaps (different streams or host threads) race and give wrong
+ *    results.
  * Errors: as ep_get_layout, plus EP_ERR_INVALID for a NULL output pointer. */
 ep_status_t ep_get_layout_noalloc(const ep_config_t *cfg, int T, const float *d_logits,
                                   const int32_t *d_topk_idx, const float *d_topk_w, int route,

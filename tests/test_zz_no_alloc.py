@@ -60,12 +60,37 @@ def test_noalloc_layout_matches_workspace_path_twice(name):
         assert ((a - b).abs() <= 2.0 ** -22 * b.abs()).all()
 
 
-def test_noalloc_rejects_configs_beyond_its_static_scratch():
+@pytest.mark.gpu
+def test_noalloc_large_expert_count_uses_a_capped_grid():
+    """E = 1024, R = 32: the static scratch holds fewer layout chunks than the
+    workspace path uses, and the layout must still be identical."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from combine_top_group_b200 import ep, runner
+    w = wl.Workload("wide", R=32, T=96, H=128, E=1024, K=8, G=8, KG=4, route=wl.ROUTE_GROUP_SIGMOID)
+    dev = torch.device("cuda:0")
+    cfg = runner.make_config(w)
+    logits = torch.from_numpy(wl.make_logits(w, 4)).to(dev)
+    ref_buf = ep.ep_buffer_create(cfg, device=dev)
+    ep.ep_get_layout(ref_buf, w.T, logits=logits, route=runner.route_of(w))
+    assert ep.ep_check_errors(ref_buf) == 0
+    ref = ep.ep_buffer_layout(ref_buf, w.T)
+    for _ in range(2):
+        out = _outputs(w, dev)
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        ep.ep_get_layout_noalloc(cfg, w.T, out, err, logits=logits, route=runner.route_of(w))
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        for key in ("topk_idx", "dst_row", "expert_off", "cnt", "num_tokens_per_rank", "is_token_in_rank"):
+            assert torch.equal(out[key], ref[key]), key
+
+
+def test_noalloc_rejects_missing_outputs_before_any_gpu_work():
     from combine_top_group_b200 import ep
-    cfg = ep.ep_default_config(32, 65536, 128, 1024, 8)  # 1024 chunks x 1056 columns > 2 MiB
+    cfg = ep.ep_default_config(8, 128, 1024, 64, 4)
     out = {k: 16 for k in ("topk_idx", "topk_w", "is_token_in_rank", "num_tokens_per_rank", "cnt",
-                           "num_tokens_per_expert", "expert_off", "rank_off", "src_off", "dst_row")}
+                           "num_tokens_per_expert", "expert_off", "rank_off", "src_off")}
+    out["dst_row"] = 0  # NULL
     with pytest.raises(ep.EpError) as ei:
-        ep.ep_get_layout_noalloc(cfg, 65536, out, 16, logits=16, stream=0)
-    assert ei.value.status == ep.EP_ERR_CAPACITY
-    assert "2 MiB" in ep.ep_last_error_message()
+        ep.ep_get_layout_noalloc(cfg, 128, out, 16, logits=16, stream=0)
+    assert ei.value.status == ep.EP_ERR_INVALID
