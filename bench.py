@@ -150,6 +150,9 @@ def run_ours(args, w: wl.Workload, rank: int, world: int, local_rank: int):
         if world > 1:
             dist.barrier()
 
+    props = torch.cuda.get_device_properties(dev)
+    bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+    clk = metrics.ClockSampler(pci_bus_id=bus).start()
     for _ in range(args.warmup):
         if flush is not None:
             flush.fill_(1)
@@ -157,11 +160,9 @@ def run_ours(args, w: wl.Workload, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize(dev)
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    props = torch.cuda.get_device_properties(dev)
-    bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
-    clk = metrics.ClockSampler(pci_bus_id=bus).start()
     barrier()
     torch.cuda.synchronize(dev)
+    t_host0 = time.perf_counter()
     for i in range(args.steps):
         if flush is not None:
             flush.fill_(1)
@@ -174,8 +175,9 @@ def run_ours(args, w: wl.Workload, rank: int, world: int, local_rank: int):
         pipe.combine(fused=fused, stream=stream)
         e[3].record(stream)
     torch.cuda.synchronize(dev)
+    t_host1 = time.perf_counter()
     barrier()
-    clocks = clk.stop()
+    clocks = clk.stop(t_host0, t_host1)
     if pipe.check_errors() != 0:
         raise RuntimeError("device error word set during the timed steps")
 

@@ -328,4 +328,17 @@ ep_status_t ep_check_errors(ep_buffer_t* b, uint32_t* word, int clear, void* str
     return ok();
 }
 
+ep_status_t ep_selftest_wait_timeout(uint32_t* d_words, uint64_t limit_ns, uint32_t* word, void* stream) {
+    if (!d_words || !word) return fail(EP_ERR_INVALID, "d_words and word must be non-NULL");
+    if (limit_ns < 1000 || limit_ns > 2000000000ull) return fail(EP_ERR_INVALID, "limit_ns must be in [1 us, 2 s]");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = ep::launch_barrier_timeout_selftest(d_words, limit_ns, s);
+    uint32_t v = 0;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&v, d_words + 2, sizeof v, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "ep_selftest_wait_timeout");
+    *word = v;
+    return ok();
+}
+
 }  // extern "C"

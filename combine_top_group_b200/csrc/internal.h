@@ -68,6 +68,10 @@ cudaError_t launch_layout_raw(const ep_config_t& c, const LayoutArgs& a, const e
                               int32_t* scratch, int max_ctas, uint32_t* err, cudaStream_t stream);
 
 cudaError_t launch_layout(const ep_buffer& b, const LayoutArgs& a, cudaStream_t stream);
+
+// Runs the layout's grid barrier with an unreachable target on 2 CTAs
+// (words: 4 device uint32; [2] receives the error bits).
+cudaError_t launch_barrier_timeout_selftest(uint32_t* words, unsigned long long limit_ns, cudaStream_t stream);
 cudaError_t launch_dispatch(const ep_buffer& b, int T, const void* x, cudaStream_t stream);
 cudaError_t launch_combine(const ep_buffer& b, int T, const void* y, const float* y_scale, void* out,
                            cudaStream_t stream);

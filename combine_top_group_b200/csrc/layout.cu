@@ -76,14 +76,15 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
 }
 
 // Bounded grid-wide barrier (the grid is co-resident: cooperative launch).
-__device__ void grid_barrier(uint32_t* arrive, uint32_t target, uint32_t* err) {
+__device__ void grid_barrier(uint32_t* arrive, uint32_t target, uint32_t* err,
+                             unsigned long long limit_ns = kWaitLimitNs) {
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
         atomicAdd(arrive, 1u);
         const unsigned long long t0 = globaltimer_ns();
         while (ld_acquire(arrive) < target) {
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 set_error(err, EP_DEVERR_TIMEOUT);
                 break;
             }
@@ -510,6 +511,13 @@ __global__ void __launch_bounds__(kThreads, 2) layout_kernel(LayoutParams p) {
     }
 }
 
+// Self-test of the bounded wait: the barrier target (one more arrival than the
+// grid has) can never be met, so every CTA must give up after limit_ns and
+// set EP_DEVERR_TIMEOUT.
+__global__ void barrier_timeout_selftest_kernel(uint32_t* bar, uint32_t* err, unsigned long long limit_ns) {
+    grid_barrier(bar, gridDim.x + 1u, err, limit_ns);
+}
+
 // Resident CTAs per SM for each kernel instantiation and shared-memory size
 // (the occupancy query is a host-side cost worth skipping per call).
 struct OccCache {
@@ -639,6 +647,17 @@ cudaError_t launch_layout(const ep_buffer& b, const LayoutArgs& a, cudaStream_t 
     LayoutArgs aa = a;
     aa.m_max = b.m_max;
     return launch_layout_raw(b.cfg, aa, out, b.scratch, kMaxLayoutCtas, b.err, st);
+}
+
+cudaError_t launch_barrier_timeout_selftest(uint32_t* words, unsigned long long limit_ns, cudaStream_t st) {
+    cudaError_t e = cudaMemsetAsync(words, 0, 4 * sizeof(uint32_t), st);
+    if (e != cudaSuccess) return e;
+    uint32_t* bar = words;
+    uint32_t* err = words + 2;
+    void* args[] = {&bar, &err, &limit_ns};
+    e = cudaLaunchCooperativeKernel((const void*)barrier_timeout_selftest_kernel, dim3(2), dim3(32), args, 0, st);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
 }
 
 }  // namespace ep

@@ -72,11 +72,13 @@ _lib.ep_check_errors.restype = _st
 _lib.ep_get_layout_noalloc.argtypes = [ctypes.POINTER(EpConfig), ctypes.c_int, _P, _P, _P, ctypes.c_int,
                                        ctypes.c_uint64, ctypes.c_float, ctypes.POINTER(EpLayout), _P, _P]
 _lib.ep_get_layout_noalloc.restype = _st
+_lib.ep_selftest_wait_timeout.argtypes = [_P, ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint32), _P]
+_lib.ep_selftest_wait_timeout.restype = _st
 
 EXPORTED = ("ep_abi_version", "ep_status_string", "ep_last_error_message", "ep_default_config",
             "ep_buffer_workspace_bytes", "ep_buffer_create", "ep_buffer_destroy", "ep_buffer_layout",
             "ep_buffer_recv", "ep_get_layout", "ep_dispatch", "ep_combine", "ep_check_errors",
-            "ep_get_layout_noalloc")
+            "ep_get_layout_noalloc", "ep_selftest_wait_timeout")
 
 
 class EpError(RuntimeError):
@@ -234,6 +236,16 @@ def ep_check_errors(buf: EpBuffer, clear: bool = True, stream=None) -> int:
     st = _lib.ep_check_errors(buf.handle, ctypes.byref(w), 1 if clear else 0, _stream(stream))
     if st not in (EP_OK, EP_ERR_DEVICE):
         _check(st, "ep_check_errors")
+    return w.value
+
+
+def ep_selftest_wait_timeout(words, limit_ns: int, stream=None) -> int:
+    """Runs a bounded wait that can never be satisfied; returns the error
+    bits it left (EP_DEVERR_TIMEOUT expected). `words`: 4-element int32/uint32
+    CUDA tensor."""
+    w = ctypes.c_uint32(0)
+    _check(_lib.ep_selftest_wait_timeout(_ptr(words), limit_ns, ctypes.byref(w), _stream(stream)),
+           "ep_selftest_wait_timeout")
     return w.value
 
 

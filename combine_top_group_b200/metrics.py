@@ -112,8 +112,9 @@ REASON_COLS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_
 
 
 class ClockSampler:
-    """Samples the SM clock, power and clock-event (throttle) reasons while
-    the timed region runs. It reads NVML every 5 ms from a thread. Without
+    """Samples the SM clock and clock-event (throttle) reasons from a thread
+    (NVML, every 1 ms; power every 10th sample), with host timestamps, so the
+    caller can keep the samples that fall inside its timed region. Without
     NVML it runs nvidia-smi every 200 ms. Read-only: no GPU setting is
     touched."""
 
@@ -121,34 +122,37 @@ class ClockSampler:
     _BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
              "hw_thermal_slowdown": 0x40}
 
-    def __init__(self, pci_bus_id: str | None = None, interval_s: float = 0.005):
+    def __init__(self, pci_bus_id: str | None = None, interval_s: float = 0.001):
         self.pci_bus_id = pci_bus_id
         self.interval = interval_s
         self.proc = None
         self.thread = None
-        self.samples = []
+        self.samples = []  # (t, sm_mhz, max_mhz, power_w or None, reasons)
         self._stop = None
 
     def start(self):
         try:
             import threading
+            import time
 
             import pynvml
             pynvml.nvmlInit()
             h = (pynvml.nvmlDeviceGetHandleByPciBusId(self.pci_bus_id) if self.pci_bus_id
                  else pynvml.nvmlDeviceGetHandleByIndex(0))
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
             self._stop = threading.Event()
 
             def run():
+                i = 0
                 while not self._stop.is_set():
                     try:
                         sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
-                        mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
-                        pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
                         rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
-                        self.samples.append((sm, mx, pw, rs))
+                        pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0 if i % 10 == 0 else None
+                        self.samples.append((time.perf_counter(), sm, mx, pw, rs))
                     except Exception:  # noqa: BLE001 - sampling is best effort
                         pass
+                    i += 1
                     self._stop.wait(self.interval)
 
             self.thread = threading.Thread(target=run, daemon=True)
@@ -163,11 +167,17 @@ class ClockSampler:
             self.proc = None
         return self
 
-    def stop(self) -> dict | None:
+    def stop(self, t0: float | None = None, t1: float | None = None) -> dict | None:
+        """Stops sampling. Summarises the samples taken in [t0, t1] (host
+        perf_counter times), or all of them if none fall inside."""
         if self.thread is not None:
             self._stop.set()
             self.thread.join(timeout=5)
-            return summarize_nvml(self.samples, self._BITS)
+            inside = [x for x in self.samples if (t0 is None or x[0] >= t0) and (t1 is None or x[0] <= t1)]
+            out = summarize_nvml([x[1:] for x in (inside or self.samples)], self._BITS)
+            if out is not None:
+                out["window"] = "timed region" if inside else "whole run (no sample inside the timed region)"
+            return out
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -180,12 +190,14 @@ class ClockSampler:
 
 
 def summarize_nvml(samples, bits) -> dict | None:
+    """samples: (sm_mhz, max_mhz, power_w or None, reasons)."""
     if not samples:
         return None
     sm = [s[0] for s in samples]
+    pw = [s[2] for s in samples if s[2] is not None]
     reasons = sorted({name for s in samples for name, b in bits.items() if s[3] & b})
     return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(s[1] for s in samples),
-            "reasons": reasons, "samples": len(samples), "power_w_max": max(s[2] for s in samples),
+            "reasons": reasons, "samples": len(samples), "power_w_max": max(pw) if pw else None,
             "source": "nvml"}
 
 

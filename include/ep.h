@@ -190,6 +190,15 @@ ep_status_t ep_combine(ep_buffer_t *buf, int T, const void *d_y, const float *d_
  * none, EP_ERR_CUDA on a CUDA failure. */
 ep_status_t ep_check_errors(ep_buffer_t *buf, uint32_t *word, int clear, void *stream);
 
+/* Diagnostic: proves that the library's bounded waits end. Runs the layout's
+ * grid barrier on 2 CTAs with a target that can never be reached, and a limit
+ * of limit_ns (1 us .. 2 s). Every CTA must give up and set EP_DEVERR_TIMEOUT.
+ * d_words: 4 device uint32 of scratch, owned by the caller. The call
+ * synchronises `stream` and returns the error bits in *word. It never traps,
+ * and the CUDA context stays usable. (The pages have no counterpart: it checks
+ * this implementation's failure detection.) */
+ep_status_t ep_selftest_wait_timeout(uint32_t *d_words, uint64_t limit_ns, uint32_t *word, void *stream);
+
 /* Routing + layout that allocates nothing, for callers that cannot get device
  * memory beyond their own inputs and outputs: code under a host framework
  * whose memory planner owns every device byte, or a runtime with a fixed

@@ -49,7 +49,8 @@ def test_parse_clocks_and_rules():
     assert metrics.clocks_rejected(c) is None
     assert "throttled" in metrics.clocks_rejected({"sm_mhz": 1900, "sm_max_mhz": 1965, "reasons": ["hw_slowdown"]})
     assert "clock lock" in metrics.clocks_rejected({"sm_mhz": 800, "sm_max_mhz": 1965, "reasons": []})
-    s = metrics.summarize_nvml([(1900, 1965, 800.0, 0x4), (1700, 1965, 990.0, 0x40)], metrics.ClockSampler._BITS)
+    s = metrics.summarize_nvml([(1900, 1965, 800.0, 0x4), (1700, 1965, None, 0x40)], metrics.ClockSampler._BITS)
+    assert s["power_w_max"] == 800.0
     assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"] and s["sm_mhz"] == 1800
 
 
