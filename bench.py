@@ -52,6 +52,10 @@ def parse_args(argv=None):
     ap.add_argument("--num-sms", type=int, default=0, help="SM cap for dispatch (0 = all)")
     ap.add_argument("--fused-fp8-combine", action="store_true",
                     help="FP8 workloads: combine straight from the e4m3 rows (fused dequant)")
+    ap.add_argument("--sweep-sms", action="store_true",
+                    help="also time dispatch/combine under SM budgets 20, 1/4, 1/2, 3/4 and all SMs")
+    ap.add_argument("--overlap", action="store_true",
+                    help="also time dispatch+combine (20 SMs, own stream) against a concurrent bf16 GEMM")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args(argv)
@@ -226,10 +230,92 @@ def run_ours(args, w: wl.Workload, rank: int, world: int, local_rank: int):
         out["clocks_rejected"] = why
     if e2e is not None:
         out["e2e"] = e2e
+    if args.sweep_sms:
+        out["sms_sweep"] = sweep_sms(pipe, w, fused, stream, bytes_dispatch, bytes_combine, props.multi_processor_count)
+    if args.overlap:
+        out["overlap"] = measure_overlap(pipe, w, dev, fused)
+    ep.ep_buffer_set_num_sms(pipe.buf, args.num_sms)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def sweep_sms(pipe, w, fused, stream, bytes_dispatch, bytes_combine, sm_count, steps=10):
+    """Dispatch and combine alone under SM budgets (Buffer.set_num_sms):
+    DeepEP's default 20, then 1/4, 1/2, 3/4 and all of the SMs."""
+    import torch
+
+    from combine_top_group_b200 import ep
+    rows = []
+    for n in (20, sm_count // 4, sm_count // 2, 3 * sm_count // 4, sm_count):
+        ep.ep_buffer_set_num_sms(pipe.buf, n)
+        pipe.dispatch(stream)
+        pipe.combine(fused=fused, stream=stream)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record(stream)
+        for _ in range(steps):
+            pipe.dispatch(stream)
+        ev[1].record(stream)
+        for _ in range(steps):
+            pipe.combine(fused=fused, stream=stream)
+        ev[2].record(stream)
+        torch.cuda.synchronize()
+        d = ev[0].elapsed_time(ev[1]) / steps / 1e3
+        c = ev[1].elapsed_time(ev[2]) / steps / 1e3
+        rows.append({"num_sms": n, "dispatch_us": d * 1e6, "dispatch_gbs": bytes_dispatch / d / 1e9,
+                     "combine_us": c * 1e6, "combine_gbs": bytes_combine / c / 1e9})
+    return rows
+
+
+def measure_overlap(pipe, w, dev, fused, comm_sms=20, reps=5):
+    """Compute/communication overlap (DeepEP overlap notes, §节点内通信):
+    dispatch + combine capped at `comm_sms` SMs on a communication stream, next
+    to a bf16 GEMM on a compute stream. The GEMM is a cuBLAS stand-in for the
+    expert work and is not part of the path. Reports both times alone and
+    together, and how much of the shorter one the overlap hid."""
+    import torch
+
+    from combine_top_group_b200 import ep
+    comp = torch.cuda.Stream(dev)
+    comm = torch.cuda.Stream(dev)
+    a = torch.randn(8192, 7168, dtype=torch.bfloat16, device=dev)
+    b = torch.randn(7168, 8192, dtype=torch.bfloat16, device=dev)
+    ep.ep_buffer_set_num_sms(pipe.buf, comm_sms)
+
+    def gemm():
+        with torch.cuda.stream(comp):
+            for _ in range(reps):
+                torch.matmul(a, b)
+
+    def comms():
+        for _ in range(reps):
+            pipe.dispatch(comm)
+            pipe.combine(fused=fused, stream=comm)
+
+    def timed(fn_list):
+        start = torch.cuda.Event(enable_timing=True)
+        start.record(torch.cuda.current_stream(dev))
+        ends = []
+        for st, fn in fn_list:
+            st.wait_event(start)
+            fn()
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(st)
+            ends.append(e)
+        torch.cuda.synchronize(dev)
+        return max(start.elapsed_time(e) for e in ends) / reps
+
+    timed([(comp, gemm), (comm, comms)])  # warm-up
+    t_gemm = timed([(comp, gemm)])
+    t_comm = timed([(comm, comms)])
+    t_both = timed([(comp, gemm), (comm, comms)])
+    ep.ep_buffer_set_num_sms(pipe.buf, 0)
+    t_comm_all = timed([(comm, comms)])
+    hidden = (t_gemm + t_comm - t_both) / min(t_gemm, t_comm)
+    return {"comm_sms": comm_sms, "gemm_ms": t_gemm, "comm_ms": t_comm, "comm_ms_all_sms": t_comm_all,
+            "together_ms": t_both, "serial_ms": t_gemm + t_comm, "hidden_frac_of_shorter": hidden,
+            "gemm": "bf16 8192x7168 @ 7168x8192 (cuBLAS stand-in for expert compute)"}
 
 
 def measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps, world):

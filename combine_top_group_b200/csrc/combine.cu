@@ -6,7 +6,8 @@
 // slots. FP8 expert outputs are dequantised in the same pass: e4m3 * scale
 // in fp32.
 //
-// One CTA per token. Each thread owns 16 channels of y: a 32-byte vector of
+// One CTA per token (a grid-stride loop when num_sms caps the grid). Each
+// thread owns 16 channels of y: a 32-byte vector of
 // bf16 (256-bit load) or a 16-byte vector of e4m3. It issues the K gathers of
 // that column before any arithmetic, so K loads are in flight per thread.
 // Loads use the streaming cache hint (y is read once). The 32 output bytes
@@ -55,7 +56,7 @@ __device__ __forceinline__ void stage_slots(const CombineParams& p, int64_t g, i
 __global__ void __launch_bounds__(kCombineThreads) combine_bf16_kernel(CombineParams p) {
     __shared__ int32_t s_row[kMaxK];
     __shared__ float s_w[kMaxK];
-    const int64_t g = blockIdx.x;
+    for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {  // grid-stride when num_sms caps the grid
     stage_slots(p, g, s_row, s_w);
     const int nvec = p.H / 16;  // 32-byte vectors: 16 bf16 channels
     const size_t rb = (size_t)p.H * 2;
@@ -88,12 +89,14 @@ __global__ void __launch_bounds__(kCombineThreads) combine_bf16_kernel(CombinePa
         for (int j = 0; j < 8; ++j) o.v[j] = pack_bf16x2(acc[2 * j], acc[2 * j + 1]);
         st256(p.out + (size_t)g * rb + (size_t)v * 32, o);
     }
+    __syncthreads();  // s_row / s_w are rewritten by the next token
+    }
 }
 
 __global__ void __launch_bounds__(kCombineThreads) combine_fp8_kernel(CombineParams p) {
     __shared__ int32_t s_row[kMaxK];
     __shared__ float s_w[kMaxK];
-    const int64_t g = blockIdx.x;
+    for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {  // grid-stride when num_sms caps the grid
     stage_slots(p, g, s_row, s_w);
     const int nvec = p.H / 16;  // 16 e4m3 channels (16 B) per vector
     const int nb = p.H / 128;
@@ -136,6 +139,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_fp8_kernel(CombinePar
         for (int j = 0; j < 8; ++j) o.v[j] = pack_bf16x2(acc[2 * j], acc[2 * j + 1]);
         st256(p.out + (size_t)g * p.H * 2 + (size_t)v * 32, o);
     }
+    __syncthreads();
+    }
 }
 
 }  // namespace
@@ -155,9 +160,19 @@ cudaError_t launch_combine(const ep_buffer& b, int T, const void* y, const float
     p.out = static_cast<uint8_t*>(out);
     p.err = b.err;
     if (p.N == 0) return cudaSuccess;
-    const unsigned grid = (unsigned)p.N;
-    if (y_scale == nullptr) combine_bf16_kernel<<<grid, kCombineThreads, 0, st>>>(p);
-    else combine_fp8_kernel<<<grid, kCombineThreads, 0, st>>>(p);
+    auto kern = (y_scale == nullptr) ? combine_bf16_kernel : combine_fp8_kernel;
+    int64_t grid = p.N;
+    const int sm_cap = (c.num_sms > 0 && c.num_sms < b.sm_count) ? c.num_sms : b.sm_count;
+    if (sm_cap < b.sm_count) {
+        // num_sms cap (Buffer.set_num_sms): a resident grid on sm_cap SMs' worth of CTAs
+        int per_sm = 0;
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kCombineThreads, 0);
+        if (e != cudaSuccess) return e;
+        grid = (int64_t)sm_cap * (per_sm > 0 ? per_sm : 1);
+        if (grid > p.N) grid = p.N;
+    }
+    if (grid > 0x7fffffff) grid = 0x7fffffff;
+    kern<<<(unsigned)grid, kCombineThreads, 0, st>>>(p);
     return cudaGetLastError();
 }
 

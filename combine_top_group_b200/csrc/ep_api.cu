@@ -229,6 +229,13 @@ ep_status_t ep_buffer_destroy(ep_buffer_t* buf) {
     return ok();
 }
 
+ep_status_t ep_buffer_set_num_sms(ep_buffer_t* b, int num_sms) {
+    if (ep_status_t st = check_buf(b)) return st;
+    if (num_sms < 0) return fail(EP_ERR_INVALID, "num_sms must be >= 0");
+    b->cfg.num_sms = num_sms;
+    return ok();
+}
+
 ep_status_t ep_buffer_layout(const ep_buffer_t* b, ep_layout_t* out) {
     if (ep_status_t st = check_buf(b)) return st;
     if (!out) return fail(EP_ERR_INVALID, "out is NULL");

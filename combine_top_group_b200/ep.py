@@ -56,6 +56,8 @@ _lib.ep_buffer_create.argtypes = [ctypes.POINTER(EpConfig), _P, ctypes.c_size_t,
 _lib.ep_buffer_create.restype = _st
 _lib.ep_buffer_destroy.argtypes = [_P]
 _lib.ep_buffer_destroy.restype = _st
+_lib.ep_buffer_set_num_sms.argtypes = [_P, ctypes.c_int]
+_lib.ep_buffer_set_num_sms.restype = _st
 _lib.ep_buffer_layout.argtypes = [_P, ctypes.POINTER(EpLayout)]
 _lib.ep_buffer_layout.restype = _st
 _lib.ep_buffer_recv.argtypes = [_P, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P),
@@ -76,7 +78,8 @@ _lib.ep_selftest_wait_timeout.argtypes = [_P, ctypes.c_uint64, ctypes.POINTER(ct
 _lib.ep_selftest_wait_timeout.restype = _st
 
 EXPORTED = ("ep_abi_version", "ep_status_string", "ep_last_error_message", "ep_default_config",
-            "ep_buffer_workspace_bytes", "ep_buffer_create", "ep_buffer_destroy", "ep_buffer_layout",
+            "ep_buffer_workspace_bytes", "ep_buffer_create", "ep_buffer_destroy", "ep_buffer_set_num_sms",
+            "ep_buffer_layout",
             "ep_buffer_recv", "ep_get_layout", "ep_dispatch", "ep_combine", "ep_check_errors",
             "ep_get_layout_noalloc", "ep_selftest_wait_timeout")
 
@@ -175,6 +178,12 @@ def ep_buffer_destroy(buf: EpBuffer) -> None:
     h, buf.handle = buf.handle, None
     if h:
         _check(_lib.ep_buffer_destroy(h), "ep_buffer_destroy")
+
+
+def ep_buffer_set_num_sms(buf: EpBuffer, num_sms: int) -> None:
+    """SM budget of dispatch and combine (0 = all); Buffer.set_num_sms analogue."""
+    _check(_lib.ep_buffer_set_num_sms(buf.handle, num_sms), "ep_buffer_set_num_sms")
+    buf.cfg.num_sms = num_sms
 
 
 def ep_buffer_layout(buf: EpBuffer, T: int) -> dict:

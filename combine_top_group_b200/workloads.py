@@ -55,6 +55,7 @@ class Workload:
     zipf_s: float = 0.0       # logit bias exponent (0 = none)
     mask_frac: float = 0.0    # fraction of top-k slots masked to -1
     mask_seed: int = 0x5EED
+    low_latency: bool = False  # fixed (expert, source rank) receive regions of T rows
 
     @property
     def N(self) -> int:
@@ -72,6 +73,8 @@ class Workload:
             extra += f" zipf{self.zipf_s}"
         if self.mask_frac:
             extra += f" mask{self.mask_frac}"
+        if self.low_latency:
+            extra += " low-latency-layout"
         return (f"{self.name} {self.R}x{self.T} H{self.H} E{self.E} top{self.K}{grp} "
                 f"{ROUTE_NAMES[self.route]} {fmt}{extra}")
 
@@ -83,6 +86,8 @@ WORKLOADS = {
     "tiny": Workload("tiny", R=4, T=128, H=1024, E=16, K=4, route=ROUTE_SOFTMAX),
     "decode": Workload("decode", R=8, T=128, H=7168, E=256, K=8,
                        route=ROUTE_SOFTMAX_RENORM, fp8=True),
+    "decode_ll": Workload("decode_ll", R=8, T=128, H=7168, E=256, K=8,
+                          route=ROUTE_SOFTMAX_RENORM, fp8=True, low_latency=True),
     "prefill": Workload("prefill", R=8, T=4096, H=7168, E=256, K=8, G=8, KG=4,
                         route=ROUTE_GROUP_SIGMOID),
     "skewed": Workload("skewed", R=8, T=4096, H=4096, E=64, K=6,

@@ -130,6 +130,15 @@ ep_status_t ep_buffer_create(const ep_config_t *cfg, void *d_workspace, size_t b
 /* Frees the host struct only. NULL is a no-op. */
 ep_status_t ep_buffer_destroy(ep_buffer_t *buf);
 
+/* Sets the SM budget of the buffer's dispatch and combine kernels: at most
+ * num_sms SMs' worth of resident CTAs, each looping over tokens; 0 = all SMs.
+ * This is the analogue of DeepEP's Buffer.set_num_sms (DeepEP summary,
+ * "如何调优 Buffer.set_num_sms"; DeepEP overlap notes, §节点内通信: 20
+ * communication SMs, the rest for compute). It takes effect from the next
+ * call. Results are identical under any budget.
+ * Errors: EP_ERR_INVALID for num_sms < 0. */
+ep_status_t ep_buffer_set_num_sms(ep_buffer_t *buf, int num_sms);
+
 /* Device views of the layout arrays inside the workspace. */
 ep_status_t ep_buffer_layout(const ep_buffer_t *buf, ep_layout_t *out);
 

@@ -59,6 +59,8 @@ def _load():
     lib.orc_apply_mask.restype = None
     lib.orc_layout.argtypes = [P, i32, i32, i32, i32, P, P, P, P, P, P, P, P]
     lib.orc_layout.restype = i32
+    lib.orc_layout_ll.argtypes = [P, i32, i32, i32, i32, i32, P]
+    lib.orc_layout_ll.restype = i32
     lib.orc_quant_fp8_row.argtypes = [P, i32, P, P]
     lib.orc_quant_fp8_row.restype = None
     lib.orc_dispatch.argtypes = [P, P, P, i64, i32, i32, i32, P, P, P, P]
@@ -163,6 +165,16 @@ def layout(idx: np.ndarray, R: int, T: int, E: int) -> dict:
     return out
 
 
+def layout_ll(idx: np.ndarray, R: int, T: int, T_max: int, E: int):
+    """Low-latency layout rows. Returns (dst_row int32 [N,K], error bits)."""
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    N, K = idx.shape
+    assert N == R * T
+    dst = np.empty((N, K), dtype=np.int32)
+    err = _load().orc_layout_ll(_p(idx), R, T, T_max, E, K, _p(dst))
+    return dst, int(err)
+
+
 # ---- dispatch / combine ----------------------------------------------------
 
 def quant_fp8_row(x_row: np.ndarray):
@@ -233,6 +245,10 @@ def run_path(x: np.ndarray, logits: np.ndarray | None, w, topk_idx=None, topk_w=
         idx, tw, margin = np.array(topk_idx, dtype=np.int32), np.array(topk_w, dtype=np.float32), None
     lay = layout(idx, w.R, w.T, w.E)
     M = int(lay["expert_off"][-1])
+    if getattr(w, "low_latency", False):
+        # fixed (expert, source rank) regions of T_max rows; the counts stay the same
+        lay["dst_row"], _ = layout_ll(idx, w.R, w.T, w.T, w.E)
+        M = w.E * w.R * w.T
     recv_x, recv_scale, recv_src, recv_w = dispatch(x, lay["dst_row"], tw, M, w.fp8)
     if w.fp8 and not fp8_combine_fused:
         y, ys = identity_expert_fp8(recv_x, recv_scale), None

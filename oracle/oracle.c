@@ -338,6 +338,41 @@ int orc_layout(const int32_t *idx, int R, int T, int E, int K,
     return err;
 }
 
+/* Low-latency layout, after the low-latency kernels of the DeepEP pages
+ * (DeepEP overlap notes, §计算-通信重叠: the decode-phase mode). Each
+ * (expert, source rank) pair owns a fixed region of T_max rows, so a row's
+ * place needs no prefix sum across ranks. */
+int orc_layout_ll(const int32_t *idx, int R, int T, int T_max, int E, int K, int32_t *dst_row)
+{
+    int err = 0;
+    int64_t *run = malloc(sizeof(int64_t) * (size_t)E);
+    for (int s = 0; s < R; ++s) {
+        for (int e = 0; e < E; ++e)
+            run[e] = 0;
+        for (int t = 0; t < T; ++t) {
+            int64_t g = (int64_t)s * T + t;
+            for (int k = 0; k < K; ++k) {
+                int e = idx[g * K + k];
+                if (e < -1 || e >= E)
+                    err |= 1;
+                if (e < 0 || e >= E) {
+                    dst_row[g * K + k] = -1;
+                    continue;
+                }
+                if (run[e] >= T_max) {
+                    err |= 2;
+                    dst_row[g * K + k] = -1;
+                    continue;
+                }
+                dst_row[g * K + k] = (int32_t)(((int64_t)e * R + s) * T_max + run[e]);
+                run[e] += 1;
+            }
+        }
+    }
+    free(run);
+    return err;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Dispatch                                                                  */
 /* ------------------------------------------------------------------------ */

@@ -60,6 +60,13 @@ int orc_layout(const int32_t *idx, int R, int T, int E, int K,
                int32_t *num_tokens_per_expert, int32_t *expert_off, int32_t *rank_off,
                int32_t *src_off, int32_t *dst_row);
 
+/* Low-latency layout: a fixed region of T_max rows per (expert e, source rank
+ * s). dst_row[g][k] = (e*R + s)*T_max + j, where j counts source s's earlier
+ * slots (in (token, slot) order) that chose e. A slot whose j reaches T_max
+ * (only possible with duplicate ids) gets -1, and bit 1 of the return value
+ * is set. Bit 0 flags ids outside [-1, E) (treated as masked). */
+int orc_layout_ll(const int32_t *idx, int R, int T, int T_max, int E, int K, int32_t *dst_row);
+
 /* ---- dispatch ---------------------------------------------------------- */
 /* Quantise one bf16 row of H channels (H % 128 == 0) to e4m3 with one fp32
  * scale per 128-channel block. */

@@ -148,6 +148,27 @@ def test_num_sms_cap_gives_identical_bytes(cuda):
     assert torch.equal(a.out, b.out)
 
 
+@pytest.mark.parametrize("num_sms", [1, 7, 37, 74])
+def test_set_num_sms_changes_nothing_but_the_grid(cuda, num_sms):
+    """Buffer.set_num_sms analogue: dispatch and combine (bf16 and fused FP8)
+    under an SM budget loop over tokens and give the same bytes."""
+    ep, runner = cuda
+    for name in ("tiny", "decode"):
+        w = wl.WORKLOADS[name]
+        pipe = runner.Pipeline(w, 4)
+        pipe.step(fused=True)
+        M = pipe.num_rows()
+        ref = (pipe.recv["recv_x"][:M].clone(), pipe.out.clone())
+        ep.ep_buffer_set_num_sms(pipe.buf, num_sms)
+        pipe.recv["recv_x"][:M].zero_()
+        pipe.out.zero_()
+        pipe.step(fused=True)
+        assert pipe.check_errors() == 0
+        assert torch.equal(pipe.recv["recv_x"][:M], ref[0]) and torch.equal(pipe.out, ref[1])
+    with pytest.raises(ep.EpError):
+        ep.ep_buffer_set_num_sms(pipe.buf, -1)
+
+
 def test_deterministic_bytes(cuda):
     ep, runner = cuda
     w = wl.WORKLOADS["decode"]

@@ -157,3 +157,48 @@ def test_layout_out_of_range_ids_flagged_and_masked():
     ref = oracle.layout(clean, R, T, E)
     for key in ("dst_row", "cnt", "expert_off", "is_token_in_rank", "num_tokens_per_rank"):
         assert np.array_equal(lay[key], ref[key]), key
+
+
+def test_layout_ll_hand_worked_example():
+    g = read_golden("layout_ll_example.txt")
+    R, T, T_max, E, K = (int(g[k][0]) for k in ("R", "T", "T_max", "E", "K"))
+    idx = _ints(g, "topk_idx", (R * T, K))
+    dst, err = oracle.layout_ll(idx, R, T, T_max, E)
+    assert err == 0
+    assert np.array_equal(dst, _ints(g, "dst_row", (R * T, K)))
+
+
+def _brute_force_ll(idx, R, T, T_max, E):
+    N, K = idx.shape
+    rows = np.full((N, K), -1, dtype=np.int32)
+    for s in range(R):
+        for e in range(E):
+            slots = [(g, k) for g in range(s * T, (s + 1) * T) for k in range(K) if idx[g, k] == e]
+            for j, (g, k) in enumerate(slots):
+                if j < T_max:
+                    rows[g, k] = (e * R + s) * T_max + j
+    return rows
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode"])
+def test_layout_ll_brute_force_and_regions(name):
+    w = wl.WORKLOADS[name]
+    idx, _, _ = oracle.route(wl.make_logits(w, 1), w.K, w.route, w.G, w.KG)
+    dst, err = oracle.layout_ll(idx, w.R, w.T, w.T, w.E)
+    assert err == 0
+    assert np.array_equal(dst, _brute_force_ll(idx, w.R, w.T, w.T, w.E))
+    # each (e, s) region holds rows base .. base + cnt[s][e] - 1, matching the standard layout's counts
+    cnt = oracle.layout(idx, w.R, w.T, w.E)["cnt"]
+    used = np.sort(dst[dst >= 0])
+    expect = np.sort(np.concatenate([(e * w.R + s) * w.T + np.arange(cnt[s, e])
+                                     for e in range(w.E) for s in range(w.R)]))
+    assert np.array_equal(used, expect)
+
+
+def test_layout_ll_overflow_with_duplicates_is_flagged():
+    # T_max = 2 but rank 0 sends expert 1 three times
+    idx = np.array([[1, 1], [1, 0], [0, 2], [3, 3]], dtype=np.int32)
+    dst, err = oracle.layout_ll(idx, 2, 2, 2, 4)
+    assert err & 2
+    # e1 from s0: slots (0,0)->j0, (0,1)->j1, (1,0) overflows; (1,1) is e0 from s0 -> (0*2+0)*2+0 = 0
+    assert list(dst[1]) == [-1, 0]
