@@ -141,7 +141,7 @@ def run_ours(args, w: wl.Workload, rank: int, world: int, local_rank: int):
         pipe.identity_expert()
     if pipe.check_errors() != 0:
         raise RuntimeError("device error word set during set-up")
-    M = pipe.num_rows()
+    M = pipe.moved_rows()
     bytes_layout = metrics.layout_bytes(w)
     bytes_dispatch = metrics.dispatch_bytes(w, M)
     bytes_combine = metrics.combine_bytes(w, M, fused_fp8=fused)

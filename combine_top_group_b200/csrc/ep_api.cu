@@ -55,9 +55,12 @@ ep_status_t validate(const ep_config_t* c) {
         if (c->topk > c->topk_groups * gs) return fail(EP_ERR_INVALID, "topk exceeds the experts of the kept groups");
     }
     if (c->num_sms < 0) return fail(EP_ERR_INVALID, "num_sms must be >= 0");
-    if (c->flags & ~EP_FLAG_FP8) return fail(EP_ERR_INVALID, "unknown flag bits");
+    if (c->flags & ~(EP_FLAG_FP8 | EP_FLAG_LOW_LATENCY)) return fail(EP_ERR_INVALID, "unknown flag bits");
     const int64_t m_max = (int64_t)c->num_ranks * c->max_tokens_per_rank * c->topk;
     if (m_max >= (int64_t)1 << 31) return fail(EP_ERR_UNSUPPORTED, "R*T_max*K must be < 2^31 (int32 row ids)");
+    if ((c->flags & EP_FLAG_LOW_LATENCY) &&
+        (int64_t)c->num_experts * c->num_ranks * c->max_tokens_per_rank >= (int64_t)1 << 31)
+        return fail(EP_ERR_UNSUPPORTED, "low-latency layout: E*R*T_max must be < 2^31 (int32 row ids)");
     return EP_OK;
 }
 
@@ -75,7 +78,8 @@ enum {
 Plan plan_of(const ep_config_t* c, int64_t* n_max, int64_t* m_max, int64_t* nc_max) {
     const int64_t R = c->num_ranks, T = c->max_tokens_per_rank, H = c->hidden, E = c->num_experts,
                   K = c->topk;
-    const int64_t N = R * T, M = N * K;
+    const int64_t N = R * T;
+    const int64_t M = (c->flags & EP_FLAG_LOW_LATENCY) ? E * R * T : N * K;
     const int64_t scratch = ep::layout_scratch_ints(*c, ep::kMaxLayoutCtas);
     const bool fp8 = (c->flags & EP_FLAG_FP8) != 0;
     size_t sz[R_COUNT];

@@ -55,6 +55,8 @@ struct LayoutArgs {
     uint64_t mask_seed;
     uint64_t mask_threshold;  // in [0, 2^32]
     int64_t m_max;            // rows the receive side holds (bound check)
+    int low_latency;          // fixed (expert, source rank) regions of T_max rows
+    int T_max;                // region size in low-latency mode
 };
 
 // int32 entries of layout scratch for a grid of at most max_ctas CTAs:

@@ -62,6 +62,8 @@ struct LayoutParams {
     int32_t* tot;    // [J]: column totals
     int32_t *ntpr, *cnt, *ntpe, *expert_off, *rank_off, *src_off, *dst_row;
     int64_t m_max;
+    int ll;     // low-latency layout: row = (e*R + s)*T_max + j
+    int T_max;  // region size (low-latency layout)
     uint32_t* err;
     uint32_t* bar;  // [2]: barrier arrivals, finished CTAs; both 0 between launches
 };
@@ -466,7 +468,11 @@ __global__ void __launch_bounds__(kThreads, 2) layout_kernel(LayoutParams p) {
     }
     if (has_chunk) {
         for (int e = threadIdx.x; e < p.E; e += kThreads) {
-            int run = eoff[e] + p.chunk[(int64_t)e * p.nc + c];
+            // standard: expert block + chunk prefix. Low-latency: fixed region of
+            // (e, s) + this rank's part of the chunk prefix
+            int run = p.ll ? (int)(((int64_t)e * p.R + s) * p.T_max) + p.chunk[(int64_t)e * p.nc + c] -
+                                 p.src_off[(int64_t)e * p.R + s]
+                           : eoff[e] + p.chunk[(int64_t)e * p.nc + c];
 #pragma unroll
             for (int w = 0; w < kWarps; ++w) {
                 const int x = hist[w * p.J + e];
@@ -488,7 +494,9 @@ __global__ void __launch_bounds__(kThreads, 2) layout_kernel(LayoutParams p) {
                 int32_t row = -1;
                 if (valid) {
                     const int64_t r = (int64_t)my_hist[e] + __popc(peers & lt);
-                    if (r < p.m_max) row = (int32_t)r;
+                    const bool in_region =
+                        !p.ll || r - ((int64_t)e * p.R + s) * p.T_max < (int64_t)p.T_max;  // only duplicates overflow
+                    if (r < p.m_max && in_region) row = (int32_t)r;
                     else set_error(p.err, EP_DEVERR_ROW_BOUNDS);
                 }
                 p.dst_row[slot0 + j] = row;
@@ -618,6 +626,8 @@ cudaError_t launch_layout_raw(const ep_config_t& c, const LayoutArgs& a, const e
     p.src_off = out.src_off;
     p.dst_row = out.dst_row;
     p.m_max = a.m_max;
+    p.ll = a.low_latency;
+    p.T_max = a.T_max;
     p.err = err;
     // scratch: [control][chunk J*max_ctas][tot J]
     p.bar = reinterpret_cast<uint32_t*>(scratch);
@@ -646,6 +656,8 @@ cudaError_t launch_layout(const ep_buffer& b, const LayoutArgs& a, cudaStream_t 
     out.dst_row = b.dst_row;
     LayoutArgs aa = a;
     aa.m_max = b.m_max;
+    aa.low_latency = (b.cfg.flags & EP_FLAG_LOW_LATENCY) ? 1 : 0;
+    aa.T_max = b.cfg.max_tokens_per_rank;
     return launch_layout_raw(b.cfg, aa, out, b.scratch, kMaxLayoutCtas, b.err, st);
 }
 

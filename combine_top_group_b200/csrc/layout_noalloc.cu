@@ -105,7 +105,10 @@ extern "C" ep_status_t ep_get_layout_noalloc(const ep_config_t* cfg, int T, cons
     a.route = route;
     a.mask_seed = mask_seed;
     a.mask_threshold = (uint64_t)floor((double)mask_frac * 4294967296.0);
-    a.m_max = (int64_t)cfg->num_ranks * T * cfg->topk;  // no receive buffer: this call's rows
+    a.low_latency = (cfg->flags & EP_FLAG_LOW_LATENCY) ? 1 : 0;
+    a.T_max = cfg->max_tokens_per_rank;
+    a.m_max = a.low_latency ? (int64_t)cfg->num_experts * cfg->num_ranks * cfg->max_tokens_per_rank
+                            : (int64_t)cfg->num_ranks * T * cfg->topk;  // no receive buffer: this call's rows
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     // zero the barrier words first: a call that timed out may have left them set
     e = cudaMemsetAsync(scratch, 0, sizeof(int32_t) * ep::kLayoutControlInts, cs);

@@ -26,6 +26,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 EP_OK, EP_ERR_INVALID, EP_ERR_CAPACITY, EP_ERR_OOM, EP_ERR_CUDA, EP_ERR_UNSUPPORTED, EP_ERR_DEVICE = range(7)
 EP_DEVERR_EXPERT_ID, EP_DEVERR_ROW_BOUNDS, EP_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 EP_FLAG_FP8 = 0x1
+EP_FLAG_LOW_LATENCY = 0x2
 EP_ROUTE_SOFTMAX, EP_ROUTE_SOFTMAX_RENORM, EP_ROUTE_GROUP_SIGMOID = 0, 1, 2
 
 

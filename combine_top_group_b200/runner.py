@@ -21,7 +21,7 @@ def make_config(w: wl.Workload, num_sms: int = 0, T_max: int | None = None) -> e
     cfg = ep.ep_default_config(w.R, T_max or w.T, w.H, w.E, w.K)
     cfg.num_groups, cfg.topk_groups = w.G, w.KG
     cfg.num_sms = num_sms
-    cfg.flags = ep.EP_FLAG_FP8 if w.fp8 else 0
+    cfg.flags = (ep.EP_FLAG_FP8 if w.fp8 else 0) | (ep.EP_FLAG_LOW_LATENCY if w.low_latency else 0)
     return cfg
 
 
@@ -71,6 +71,15 @@ class Pipeline:
 
     # --- harness ------------------------------------------------------------
     def num_rows(self) -> int:
+        """Receive rows the step uses: M (standard layout), or the whole
+        E*R*T_max region span (low-latency layout, rows are spread over it)."""
+        if self.w.low_latency:
+            return self.recv["max_rows"]
+        lay = ep.ep_buffer_layout(self.buf, self.w.T)
+        return int(lay["expert_off"][-1].item())
+
+    def moved_rows(self) -> int:
+        """Receive rows written by the step (expert_off[E])."""
         lay = ep.ep_buffer_layout(self.buf, self.w.T)
         return int(lay["expert_off"][-1].item())
 

@@ -59,6 +59,16 @@ typedef enum {
 
 /* ep_config_t.flags */
 #define EP_FLAG_FP8 0x1u /* dispatch casts to FP8 e4m3 with one fp32 scale per 128 channels */
+/* Low-latency (decode) receive layout, after the pages' low-latency kernels
+ * (DeepEP overlap notes, §计算-通信重叠). Expert e's rows from source rank s
+ * live in a fixed region of T_max rows: row = (e*R + s)*T_max + j, where j
+ * counts s's earlier slots (in token, slot order) that chose e. No prefix sum
+ * across ranks places a row. The buffer then holds M_max = E*R*T_max receive
+ * rows. The counts and prefix sums in ep_layout_t keep their meaning. In this
+ * mode cnt_src_expert[s][e] tells how much of region (e, s) is filled. A
+ * region overflows only if a caller's top-k repeats an expert; the extra
+ * slots are dropped with EP_DEVERR_ROW_BOUNDS. */
+#define EP_FLAG_LOW_LATENCY 0x2u
 
 /* Routing rule applied by ep_get_layout to router logits. */
 typedef enum {
@@ -142,12 +152,14 @@ ep_status_t ep_buffer_set_num_sms(ep_buffer_t *buf, int num_sms);
 /* Device views of the layout arrays inside the workspace. */
 ep_status_t ep_buffer_layout(const ep_buffer_t *buf, ep_layout_t *out);
 
-/* Device views of the receive buffers, M_max rows each:
+/* Device views of the receive buffers, M_max rows each (R*T_max*K, or
+ * E*R*T_max with EP_FLAG_LOW_LATENCY):
  *  recv_x      bf16 [M_max, H], or e4m3 [M_max, H] with EP_FLAG_FP8;
  *  recv_scale  fp32 [M_max, H/128] with EP_FLAG_FP8, else NULL;
  *  recv_src    int32 [M_max]: source token g of each row;
  *  recv_w      fp32 [M_max]: routing weight of each row.
- * The rows of rank r are [rank_off[r], rank_off[r+1]). Any out-pointer may be
+ * The rows of rank r are [rank_off[r], rank_off[r+1]) (low-latency mode:
+ * [r*(E/R)*R*T_max, (r+1)*(E/R)*R*T_max)). Any out-pointer may be
  * NULL. Also returns M_max through *max_rows if it is not NULL. */
 ep_status_t ep_buffer_recv(const ep_buffer_t *buf, void **recv_x, float **recv_scale,
                            int32_t **recv_src, float **recv_w, int64_t *max_rows);

@@ -260,3 +260,20 @@ def test_bounded_wait_gives_up_and_context_survives(cuda):
     assert pipe.check_errors() == 0
     ref = oracle.run_path(x, logits, w)
     assert np.array_equal(ep.ep_buffer_layout(pipe.buf, w.T)["dst_row"].cpu().numpy(), ref["dst_row"])
+
+
+def test_low_latency_region_overflow_flagged(cuda):
+    """Low-latency layout: a caller's top-k that repeats an expert beyond the
+    region's T_max rows gets the extra slot dropped with EP_DEVERR_ROW_BOUNDS,
+    exactly as the oracle places the rest."""
+    ep, runner = cuda
+    w = wl.Workload("ll_dup", R=2, T=2, H=128, E=4, K=2, low_latency=True)
+    idx = np.array([[1, 1], [1, 0], [0, 2], [3, 3]], dtype=np.int32)
+    tw = np.full((4, 2), 0.5, np.float32)
+    pipe = runner.Pipeline(w, 0)
+    pipe.layout(topk_idx=torch.from_numpy(idx).cuda(), topk_w=torch.from_numpy(tw).cuda())
+    err = pipe.check_errors()
+    assert err & ep.EP_DEVERR_ROW_BOUNDS
+    ref, ref_err = oracle.layout_ll(idx, 2, 2, 2, 4)
+    assert ref_err & 2
+    assert np.array_equal(ep.ep_buffer_layout(pipe.buf, 2)["dst_row"].cpu().numpy(), ref)

@@ -112,6 +112,7 @@ def _check_combine(got_bits, ref_bits):
 
 
 CASES = [("tiny", 0), ("tiny", 1), ("tiny", 2), ("decode", 0), ("decode", 1), ("decode", 2),
+         ("decode_ll", 0), ("decode_ll", 2),
          ("prefill", 0), ("prefill", 1), ("skewed", 0), ("skewed", 2), ("large", 0)]
 
 
@@ -134,40 +135,50 @@ def test_path_parity(cuda, name, seed):
         pipe.layout(topk_idx=torch.from_numpy(o_idx).cuda(), topk_w=torch.from_numpy(o_w).cuda())
         lay = {k: _to_host(v) for k, v in ep.ep_buffer_layout(pipe.buf, w.T).items()}
     o_lay = oracle.layout(o_idx, w.R, w.T, w.E)
+    if w.low_latency:
+        o_lay["dst_row"], ll_err = oracle.layout_ll(o_idx, w.R, w.T, w.T, w.E)
+        assert ll_err == 0
     for key in ("is_token_in_rank", "num_tokens_per_rank", "cnt", "num_tokens_per_expert", "expert_off",
                 "rank_off", "src_off", "dst_row"):
         assert np.array_equal(lay[key], o_lay[key]), key
-    M = int(o_lay["expert_off"][-1])
+    M = int(o_lay["expert_off"][-1])  # rows moved
 
     # ---- dispatch
     pipe.dispatch()
     assert pipe.check_errors() == 0
-    g_src = _to_host(pipe.recv["recv_src"][:M])
-    g_rw = _to_host(pipe.recv["recv_w"][:M])
     dst = o_lay["dst_row"]
-    o_src = np.full(M, -1, dtype=np.int32)
-    o_rw = np.zeros(M, dtype=np.float32)
     valid = dst >= 0
+    used = np.sort(dst[valid]).astype(np.int64)  # every receive row the step writes
+    assert len(used) == M
+    used_t = torch.from_numpy(used).cuda()
+    g_src = _to_host(pipe.recv["recv_src"].index_select(0, used_t))
+    g_rw = _to_host(pipe.recv["recv_w"].index_select(0, used_t))
     gg = np.repeat(np.arange(w.N), w.K).reshape(w.N, w.K)
-    o_src[dst[valid]] = gg[valid]
-    o_rw[dst[valid]] = o_w[valid]
+    order = np.argsort(dst[valid])
+    o_src = gg[valid][order].astype(np.int32)
+    o_rw = o_w[valid][order]
     assert np.array_equal(g_src, o_src)
     rel = np.abs(g_rw.astype(np.float64) - o_rw) / np.maximum(np.abs(o_rw), 1e-30)
     assert rel.max(initial=0.0) <= 2.0 ** -22
     # invariant: dispatch moves the layout's weights intact
-    assert np.array_equal(g_rw, lay["topk_w"][valid][np.argsort(dst[valid])])
+    assert np.array_equal(g_rw, lay["topk_w"][valid][order])
+    src_of_row = dict(zip(used.tolist(), o_src.tolist()))
 
     full = M * w.H <= 64 * 2 ** 20
-    rows = np.arange(M) if full else _sample_rows(M, o_lay["expert_off"], 3000, seed)
+    if full:
+        rows = used
+    else:
+        pick = _sample_rows(M, o_lay["expert_off"], 3000, seed)  # positions in the used-row list
+        rows = used[pick]
     rows_t = torch.from_numpy(rows).cuda()
     g_rows = _to_host(pipe.recv["recv_x"].index_select(0, rows_t))
     if not w.fp8:
-        assert np.array_equal(g_rows, x[o_src[rows]])
+        assert np.array_equal(g_rows, x[[src_of_row[int(r)] for r in rows]])
     else:
         g_sc = _to_host(pipe.recv["recv_scale"].index_select(0, rows_t))
         cache = {}
         for i, r in enumerate(rows):
-            g = int(o_src[r])
+            g = src_of_row[int(r)]
             if g not in cache:
                 cache[g] = oracle.quant_fp8_row(x[g])
             q, s = cache[g]
