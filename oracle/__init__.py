@@ -61,6 +61,16 @@ def _load():
     lib.orc_layout.restype = i32
     lib.orc_layout_ll.argtypes = [P, i32, i32, i32, i32, i32, P]
     lib.orc_layout_ll.restype = i32
+    lib.orc_layout_dedup.argtypes = [P, i32, i32, P, P, P]
+    lib.orc_layout_dedup.restype = i64
+    lib.orc_dispatch_dedup.argtypes = [P, P, P, P, i64, i32, i32, i32, i32, i32, P, P, P, P, P]
+    lib.orc_dispatch_dedup.restype = None
+    lib.orc_permute.argtypes = [P, P, P, P, P, i64, P, i32, i32, i32, P, P, P, P]
+    lib.orc_permute.restype = None
+    lib.orc_local_reduce.argtypes = [P, P, P, P, P, i64, P, i32, i32, P]
+    lib.orc_local_reduce.restype = None
+    lib.orc_combine_dedup.argtypes = [P, P, i64, i32, i32, P]
+    lib.orc_combine_dedup.restype = None
     lib.orc_quant_fp8_row.argtypes = [P, i32, P, P]
     lib.orc_quant_fp8_row.restype = None
     lib.orc_dispatch.argtypes = [P, P, P, i64, i32, i32, i32, P, P, P, P]
@@ -173,6 +183,73 @@ def layout_ll(idx: np.ndarray, R: int, T: int, T_max: int, E: int):
     dst = np.empty((N, K), dtype=np.int32)
     err = _load().orc_layout_ll(_p(idx), R, T, T_max, E, K, _p(dst))
     return dst, int(err)
+
+
+# ---- deduplicated receive --------------------------------------------------
+
+def layout_dedup(is_token_in_rank: np.ndarray, R: int, T: int) -> dict:
+    itr = np.ascontiguousarray(is_token_in_rank, dtype=np.uint8)
+    N = itr.shape[0]
+    assert N == R * T
+    out = dict(rank_row_off=np.empty(R + 1, dtype=np.int32), rank_src_off=np.empty((R, R), dtype=np.int32),
+               tok_row=np.empty((N, R), dtype=np.int32))
+    D = _load().orc_layout_dedup(_p(itr), R, T, _p(out["rank_row_off"]), _p(out["rank_src_off"]),
+                                 _p(out["tok_row"]))
+    out["D"] = int(D)
+    return out
+
+
+def dispatch_dedup(x, tok_row, topk_idx, topk_w, D: int, E: int, fp8: bool):
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    tok_row = np.ascontiguousarray(tok_row, dtype=np.int32)
+    topk_idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
+    topk_w = np.ascontiguousarray(topk_w, dtype=np.float32)
+    N, H = x.shape
+    R = tok_row.shape[1]
+    K = topk_idx.shape[1]
+    rx = np.zeros((D, H), dtype=np.uint8 if fp8 else np.uint16)
+    rs = np.zeros((D, H // 128), dtype=np.float32) if fp8 else None
+    src = np.full(D, -1, dtype=np.int32)
+    ti = np.full((D, K), -1, dtype=np.int32)
+    tw = np.zeros((D, K), dtype=np.float32)
+    _load().orc_dispatch_dedup(_p(x), _p(tok_row), _p(topk_idx), _p(topk_w), N, R, E, H, K, 1 if fp8 else 0,
+                               _p(rx), _p(rs), _p(src), _p(ti), _p(tw))
+    return dict(recv_x=rx, recv_scale=rs, recv_src=src, recv_topk_idx=ti, recv_topk_w=tw)
+
+
+def permute(dd: dict, dst_row: np.ndarray, M: int, fp8: bool):
+    dst_row = np.ascontiguousarray(dst_row, dtype=np.int32)
+    D, H = dd["recv_x"].shape
+    K = dst_row.shape[1]
+    rx = np.zeros((M, H), dtype=np.uint8 if fp8 else np.uint16)
+    rs = np.zeros((M, H // 128), dtype=np.float32) if fp8 else None
+    src = np.full(M, -1, dtype=np.int32)
+    w = np.zeros(M, dtype=np.float32)
+    _load().orc_permute(_p(dd["recv_x"]), _p(dd["recv_scale"]), _p(dd["recv_src"]), _p(dd["recv_topk_idx"]),
+                        _p(dd["recv_topk_w"]), D, _p(dst_row), H, K, 1 if fp8 else 0, _p(rx), _p(rs), _p(src), _p(w))
+    return rx, rs, src, w
+
+
+def local_reduce(y, y_scale, dd: dict, dst_row: np.ndarray):
+    y = np.ascontiguousarray(y)
+    dst_row = np.ascontiguousarray(dst_row, dtype=np.int32)
+    D = dd["recv_src"].shape[0]
+    H = y.shape[1]
+    K = dst_row.shape[1]
+    part = np.empty((D, H), dtype=np.uint16)
+    _load().orc_local_reduce(_p(y), _p(y_scale), _p(dd["recv_src"]), _p(dd["recv_topk_idx"]),
+                             _p(dd["recv_topk_w"]), D, _p(dst_row), H, K, _p(part))
+    return part
+
+
+def combine_dedup(partial: np.ndarray, tok_row: np.ndarray) -> np.ndarray:
+    partial = np.ascontiguousarray(partial, dtype=np.uint16)
+    tok_row = np.ascontiguousarray(tok_row, dtype=np.int32)
+    N, R = tok_row.shape
+    H = partial.shape[1]
+    out = np.empty((N, H), dtype=np.uint16)
+    _load().orc_combine_dedup(_p(partial), _p(tok_row), N, R, H, _p(out))
+    return out
 
 
 # ---- dispatch / combine ----------------------------------------------------

@@ -374,6 +374,154 @@ int orc_layout_ll(const int32_t *idx, int R, int T, int T_max, int E, int K, int
 }
 
 /* ------------------------------------------------------------------------ */
+/* Deduplicated (per destination rank) receive                                */
+/* ------------------------------------------------------------------------ */
+
+/* DeepEP overlap notes, §节点内通信: a token goes only to the ranks
+ * is_token_in_rank marks, once per rank, however many of that rank's experts
+ * it chose. */
+int64_t orc_layout_dedup(const uint8_t *is_token_in_rank, int R, int T, int32_t *rank_row_off,
+                         int32_t *rank_src_off, int32_t *tok_row)
+{
+    int64_t N = (int64_t)R * T;
+    int64_t *cnt = calloc((size_t)R * R, sizeof(int64_t)); /* [r][s] tokens of s sent to r */
+    for (int64_t g = 0; g < N; ++g)
+        for (int r = 0; r < R; ++r)
+            if (is_token_in_rank[g * R + r])
+                cnt[(int64_t)r * R + g / T] += 1;
+    int64_t acc = 0;
+    for (int r = 0; r < R; ++r) {
+        rank_row_off[r] = (int32_t)acc;
+        for (int s = 0; s < R; ++s) {
+            rank_src_off[r * R + s] = (int32_t)(acc - rank_row_off[r]);
+            acc += cnt[(int64_t)r * R + s];
+        }
+    }
+    rank_row_off[R] = (int32_t)acc;
+    int64_t *run = calloc((size_t)R, sizeof(int64_t));
+    for (int s = 0; s < R; ++s) {
+        for (int r = 0; r < R; ++r)
+            run[r] = 0;
+        for (int t = 0; t < T; ++t) {
+            int64_t g = (int64_t)s * T + t;
+            for (int r = 0; r < R; ++r) {
+                if (!is_token_in_rank[g * R + r]) {
+                    tok_row[g * R + r] = -1;
+                    continue;
+                }
+                tok_row[g * R + r] = (int32_t)(rank_row_off[r] + rank_src_off[r * R + s] + run[r]);
+                run[r] += 1;
+            }
+        }
+    }
+    free(cnt);
+    free(run);
+    return acc;
+}
+
+void orc_dispatch_dedup(const uint16_t *x, const int32_t *tok_row, const int32_t *topk_idx,
+                        const float *topk_w, int64_t N, int R, int E, int H, int K, int fp8,
+                        void *recv_x, float *recv_scale, int32_t *recv_src, int32_t *recv_topk_idx,
+                        float *recv_topk_w)
+{
+    int L = E / R, nb = H / 128;
+    uint8_t *q = fp8 ? malloc((size_t)H) : NULL;
+    float *sc = fp8 ? malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1)) : NULL;
+    for (int64_t g = 0; g < N; ++g) {
+        const uint16_t *xr = x + g * H;
+        if (fp8)
+            orc_quant_fp8_row(xr, H, q, sc);
+        for (int r = 0; r < R; ++r) {
+            int64_t row = tok_row[g * R + r];
+            if (row < 0)
+                continue;
+            recv_src[row] = (int32_t)g;
+            for (int k = 0; k < K; ++k) {
+                int e = topk_idx[g * K + k];
+                int here = (e >= 0 && e < E && e / L == r);
+                recv_topk_idx[row * K + k] = here ? e : -1;
+                recv_topk_w[row * K + k] = here ? topk_w[g * K + k] : 0.0f;
+            }
+            if (fp8) {
+                memcpy((uint8_t *)recv_x + row * H, q, (size_t)H);
+                memcpy(recv_scale + row * nb, sc, sizeof(float) * (size_t)nb);
+            } else {
+                memcpy((uint16_t *)recv_x + row * H, xr, sizeof(uint16_t) * (size_t)H);
+            }
+        }
+    }
+    free(q);
+    free(sc);
+}
+
+void orc_permute(const void *dedup_x, const float *dedup_scale, const int32_t *dedup_src,
+                 const int32_t *dedup_topk_idx, const float *dedup_topk_w, int64_t D, const int32_t *dst_row,
+                 int H, int K, int fp8, void *recv_x, float *recv_scale, int32_t *recv_src, float *recv_w)
+{
+    int nb = H / 128;
+    for (int64_t d = 0; d < D; ++d) {
+        int64_t g = dedup_src[d];
+        for (int k = 0; k < K; ++k) {
+            if (dedup_topk_idx[d * K + k] < 0)
+                continue;
+            int64_t row = dst_row[g * K + k];
+            if (row < 0)
+                continue;
+            recv_src[row] = (int32_t)g;
+            recv_w[row] = dedup_topk_w[d * K + k];
+            if (fp8) {
+                memcpy((uint8_t *)recv_x + row * H, (const uint8_t *)dedup_x + d * H, (size_t)H);
+                memcpy(recv_scale + row * nb, dedup_scale + d * nb, sizeof(float) * (size_t)nb);
+            } else {
+                memcpy((uint16_t *)recv_x + row * H, (const uint16_t *)dedup_x + d * H,
+                       sizeof(uint16_t) * (size_t)H);
+            }
+        }
+    }
+}
+
+void orc_local_reduce(const void *y, const float *y_scale, const int32_t *dedup_src,
+                      const int32_t *dedup_topk_idx, const float *dedup_topk_w, int64_t D,
+                      const int32_t *dst_row, int H, int K, uint16_t *partial)
+{
+    int nb = H / 128;
+    for (int64_t d = 0; d < D; ++d) {
+        int64_t g = dedup_src[d];
+        for (int h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int k = 0; k < K; ++k) {
+                if (dedup_topk_idx[d * K + k] < 0)
+                    continue;
+                int64_t row = dst_row[g * K + k];
+                if (row < 0)
+                    continue;
+                float v;
+                if (y_scale)
+                    v = orc_e4m3_decode(((const uint8_t *)y)[row * H + h]) * y_scale[row * nb + h / 128];
+                else
+                    v = orc_bf16_to_f32(((const uint16_t *)y)[row * H + h]);
+                acc = fmaf(dedup_topk_w[d * K + k], v, acc);
+            }
+            partial[d * H + h] = orc_f32_to_bf16(acc);
+        }
+    }
+}
+
+void orc_combine_dedup(const uint16_t *partial, const int32_t *tok_row, int64_t N, int R, int H, uint16_t *out)
+{
+    for (int64_t g = 0; g < N; ++g)
+        for (int h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int r = 0; r < R; ++r) {
+                int64_t d = tok_row[g * R + r];
+                if (d >= 0)
+                    acc += orc_bf16_to_f32(partial[d * H + h]);
+            }
+            out[g * H + h] = orc_f32_to_bf16(acc);
+        }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Dispatch                                                                  */
 /* ------------------------------------------------------------------------ */
 

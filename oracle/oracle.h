@@ -67,6 +67,49 @@ int orc_layout(const int32_t *idx, int R, int T, int E, int K,
  * is set. Bit 0 flags ids outside [-1, E) (treated as masked). */
 int orc_layout_ll(const int32_t *idx, int R, int T, int T_max, int E, int K, int32_t *dst_row);
 
+/* ---- deduplicated (per destination rank) receive ------------------------ */
+/* Rank-dedup layout (DeepEP overlap notes, §节点内通信: send each token only to
+ * the ranks is_token_in_rank marks). Token g goes once to every rank r it has
+ * an expert on. Receive rows are ordered by (destination rank r, source rank
+ * s, token t). Outputs:
+ *   rank_row_off i32 [R+1]      exclusive prefix of the rows per destination rank
+ *   rank_src_off i32 [R, R]     [r][s]: offset of source s inside rank r's rows
+ *   tok_row      i32 [N, R]     [g][r]: row of token g on rank r, -1 if not sent
+ * Returns the number of rows D. */
+int64_t orc_layout_dedup(const uint8_t *is_token_in_rank, int R, int T, int32_t *rank_row_off,
+                         int32_t *rank_src_off, int32_t *tok_row);
+
+/* Dedup dispatch: row tok_row[g][r] gets token g's hidden vector (bf16 copy,
+ * or the same FP8 cast as orc_dispatch), its id, and its top-k localised to
+ * rank r: recv_topk_idx[row][k] = idx[g][k] if expert idx[g][k] lives on r,
+ * else -1; recv_topk_w likewise (0 where -1). */
+void orc_dispatch_dedup(const uint16_t *x, const int32_t *tok_row, const int32_t *topk_idx,
+                        const float *topk_w, int64_t N, int R, int E, int H, int K, int fp8,
+                        void *recv_x, float *recv_scale, int32_t *recv_src, int32_t *recv_topk_idx,
+                        float *recv_topk_w);
+
+/* Local expert permutation on the receiving rank: dedup row d (token g =
+ * recv_src[d]) is copied to the expert-grouped row dst_row[g][k] of every slot
+ * k with recv_topk_idx[d][k] != -1 (plus its source id and weight). The
+ * result equals orc_dispatch's receive buffers. */
+void orc_permute(const void *dedup_x, const float *dedup_scale, const int32_t *dedup_src,
+                 const int32_t *dedup_topk_idx, const float *dedup_topk_w, int64_t D, const int32_t *dst_row,
+                 int H, int K, int fp8, void *recv_x, float *recv_scale, int32_t *recv_src, float *recv_w);
+
+/* Local reduce on the receiving rank: partial[d] = bf16( fma chain over k
+ * ascending with recv_topk_idx[d][k] != -1 of w * y[dst_row[g][k]] ) for
+ * token g = recv_src[d]. It is the rank's share of the combine, sent back as
+ * bf16. y as in orc_combine (bf16, or e4m3 + scales). */
+void orc_local_reduce(const void *y, const float *y_scale, const int32_t *dedup_src,
+                      const int32_t *dedup_topk_idx, const float *dedup_topk_w, int64_t D,
+                      const int32_t *dst_row, int H, int K, uint16_t *partial);
+
+/* Dedup combine: out[g] = bf16( sum over ranks r ascending with tok_row[g][r]
+ * != -1 of float(partial[tok_row[g][r]]) ), accumulated in fp32. Tokens not
+ * sent anywhere give +0. */
+void orc_combine_dedup(const uint16_t *partial, const int32_t *tok_row, int64_t N, int R, int H,
+                       uint16_t *out);
+
 /* ---- dispatch ---------------------------------------------------------- */
 /* Quantise one bf16 row of H channels (H % 128 == 0) to e4m3 with one fp32
  * scale per 128-channel block. */
