@@ -56,6 +56,9 @@ def parse_args(argv=None):
                     help="also time dispatch/combine under SM budgets 20, 1/4, 1/2, 3/4 and all SMs")
     ap.add_argument("--overlap", action="store_true",
                     help="also time dispatch+combine (20 SMs, own stream) against a concurrent bf16 GEMM")
+    ap.add_argument("--dedup", action="store_true",
+                    help="also time the deduplicated-receive pipeline (dispatch_dedup, permute, local_reduce, "
+                         "combine_dedup) on the same workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args(argv)
@@ -234,6 +237,8 @@ def run_ours(args, w: wl.Workload, rank: int, world: int, local_rank: int):
         out["sms_sweep"] = sweep_sms(pipe, w, fused, stream, bytes_dispatch, bytes_combine, props.multi_processor_count)
     if args.overlap:
         out["overlap"] = measure_overlap(pipe, w, dev, fused)
+    if args.dedup:
+        out["dedup"] = measure_dedup(w, rank, dev, fused, steps=min(args.steps, 10))
     ep.ep_buffer_set_num_sms(pipe.buf, args.num_sms)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w)
@@ -316,6 +321,54 @@ def measure_overlap(pipe, w, dev, fused, comm_sms=20, reps=5):
     return {"comm_sms": comm_sms, "gemm_ms": t_gemm, "comm_ms": t_comm, "comm_ms_all_sms": t_comm_all,
             "together_ms": t_both, "serial_ms": t_gemm + t_comm, "hidden_frac_of_shorter": hidden,
             "gemm": "bf16 8192x7168 @ 7168x8192 (cuBLAS stand-in for expert compute)"}
+
+
+def measure_dedup(w, seed, dev, fused, steps):
+    """Deduplicated receive (one row per token and destination rank), timed
+    kernel by kernel. rows_dedup / rows_expert is the share of expert rows
+    that would cross the links in a real multi-GPU all-to-all."""
+    import torch
+
+    from combine_top_group_b200 import runner
+    pipe = runner.Pipeline(w, seed=seed, device=dev, dedup=True)
+    stream = torch.cuda.current_stream(dev)
+    pipe.layout(stream)
+    pipe.dispatch_dedup(stream)
+    pipe.permute(stream)
+    if w.fp8 and not fused:
+        pipe.identity_expert()
+    pipe.local_reduce(fused=fused, stream=stream)
+    pipe.combine_dedup(stream)
+    if pipe.check_errors() != 0:
+        raise RuntimeError("device error word set in the dedup pipeline")
+    D, M = pipe.dedup_rows(), pipe.moved_rows()
+    names = ["layout", "dispatch_dedup", "permute", "local_reduce", "combine_dedup"]
+    calls = [lambda: pipe.layout(stream), lambda: pipe.dispatch_dedup(stream), lambda: pipe.permute(stream),
+             lambda: pipe.local_reduce(fused=fused, stream=stream), lambda: pipe.combine_dedup(stream)]
+    tot = [0.0] * len(calls)
+    for _ in range(steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+        ev[0].record(stream)
+        for i, c in enumerate(calls):
+            c()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize(dev)
+        for i in range(len(calls)):
+            tot[i] += ev[i].elapsed_time(ev[i + 1]) / 1e3
+    b = 1 if w.fp8 else 2
+    yb = (M * w.H + M * (w.H // 128) * 4) if (w.fp8 and fused) else M * w.H * 2
+    scales = (w.H // 128) * 4 if w.fp8 else 0
+    nbytes = [metrics.layout_bytes(w),
+              w.N * w.H * 2 + w.N * w.K * 8 + D * (w.H * b + scales + 4 + w.K * 8),  # x, topk, rows + ids + local top-k
+              D * (w.H * b + scales + w.K * 8 + 4) + M * (w.H * b + scales + 8),     # dedup rows in, expert rows out
+              yb + D * w.K * 8 + D * w.H * 2,                                        # expert outputs in, partials out
+              D * w.H * 2 + w.N * w.H * 2]                                           # partials in, out
+    res = {"rows_dedup": D, "rows_expert": M, "dedup_ratio": D / M if M else None, "steps": steps}
+    for n, t, nb in zip(names, tot, nbytes):
+        res[n + "_us"] = t / steps * 1e6
+        res[n + "_gbs"] = nb / (t / steps) / 1e9
+    del pipe
+    return res
 
 
 def measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps, world):

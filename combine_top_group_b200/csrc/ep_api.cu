@@ -55,7 +55,8 @@ ep_status_t validate(const ep_config_t* c) {
         if (c->topk > c->topk_groups * gs) return fail(EP_ERR_INVALID, "topk exceeds the experts of the kept groups");
     }
     if (c->num_sms < 0) return fail(EP_ERR_INVALID, "num_sms must be >= 0");
-    if (c->flags & ~(EP_FLAG_FP8 | EP_FLAG_LOW_LATENCY)) return fail(EP_ERR_INVALID, "unknown flag bits");
+    if (c->flags & ~(EP_FLAG_FP8 | EP_FLAG_LOW_LATENCY | EP_FLAG_DEDUP))
+        return fail(EP_ERR_INVALID, "unknown flag bits");
     const int64_t m_max = (int64_t)c->num_ranks * c->max_tokens_per_rank * c->topk;
     if (m_max >= (int64_t)1 << 31) return fail(EP_ERR_UNSUPPORTED, "R*T_max*K must be < 2^31 (int32 row ids)");
     if ((c->flags & EP_FLAG_LOW_LATENCY) &&
@@ -65,14 +66,16 @@ ep_status_t validate(const ep_config_t* c) {
 }
 
 struct Plan {
-    size_t off[20];
+    size_t off[32];
     size_t total;
 };
 
 // Region order inside the workspace; every region is 256-byte aligned.
 enum {
     R_TOPK_IDX, R_TOPK_W, R_ITR, R_NTPR, R_CNT, R_NTPE, R_EOFF, R_ROFF, R_SOFF, R_DST,
-    R_SCRATCH, R_ERR, R_RECV_X, R_RECV_SCALE, R_RECV_SRC, R_RECV_W, R_COUNT
+    R_SCRATCH, R_ERR, R_RECV_X, R_RECV_SCALE, R_RECV_SRC, R_RECV_W,
+    R_TOK_ROW, R_RANK_ROW_OFF, R_RANK_SRC_OFF, R_DD_X, R_DD_SCALE, R_DD_SRC, R_DD_TOPK_IDX, R_DD_TOPK_W, R_PARTIAL,
+    R_COUNT
 };
 
 Plan plan_of(const ep_config_t* c, int64_t* n_max, int64_t* m_max, int64_t* nc_max) {
@@ -99,6 +102,17 @@ Plan plan_of(const ep_config_t* c, int64_t* n_max, int64_t* m_max, int64_t* nc_m
     sz[R_RECV_SCALE] = fp8 ? (size_t)M * (H / 128) * 4 : 0;
     sz[R_RECV_SRC] = 4 * M;
     sz[R_RECV_W] = 4 * M;
+    const bool dd = (c->flags & EP_FLAG_DEDUP) != 0;
+    const int64_t D = dd ? R * T * (R < K ? R : K) : 0;
+    sz[R_TOK_ROW] = dd ? 4 * N * R : 0;
+    sz[R_RANK_ROW_OFF] = dd ? 4 * (R + 1) : 0;
+    sz[R_RANK_SRC_OFF] = dd ? 4 * R * R : 0;
+    sz[R_DD_X] = (size_t)D * H * (fp8 ? 1 : 2);
+    sz[R_DD_SCALE] = fp8 ? (size_t)D * (H / 128) * 4 : 0;
+    sz[R_DD_SRC] = 4 * D;
+    sz[R_DD_TOPK_IDX] = 4 * D * K;
+    sz[R_DD_TOPK_W] = 4 * D * K;
+    sz[R_PARTIAL] = (size_t)D * H * 2;
     Plan p{};
     size_t cur = 0;
     for (int i = 0; i < R_COUNT; ++i) {
@@ -211,6 +225,18 @@ ep_status_t ep_buffer_create(const ep_config_t* cfg, void* d_workspace, size_t b
     b->recv_scale = (cfg->flags & EP_FLAG_FP8) ? reinterpret_cast<float*>(w + p.off[R_RECV_SCALE]) : nullptr;
     b->recv_src = reinterpret_cast<int32_t*>(w + p.off[R_RECV_SRC]);
     b->recv_w = reinterpret_cast<float*>(w + p.off[R_RECV_W]);
+    const bool dd = (cfg->flags & EP_FLAG_DEDUP) != 0;
+    const int64_t R = cfg->num_ranks, K = cfg->topk;
+    b->d_max = dd ? R * cfg->max_tokens_per_rank * (R < K ? R : K) : 0;
+    b->tok_row = dd ? reinterpret_cast<int32_t*>(w + p.off[R_TOK_ROW]) : nullptr;
+    b->rank_row_off = dd ? reinterpret_cast<int32_t*>(w + p.off[R_RANK_ROW_OFF]) : nullptr;
+    b->rank_src_off = dd ? reinterpret_cast<int32_t*>(w + p.off[R_RANK_SRC_OFF]) : nullptr;
+    b->dd_x = dd ? w + p.off[R_DD_X] : nullptr;
+    b->dd_scale = (dd && (cfg->flags & EP_FLAG_FP8)) ? reinterpret_cast<float*>(w + p.off[R_DD_SCALE]) : nullptr;
+    b->dd_src = dd ? reinterpret_cast<int32_t*>(w + p.off[R_DD_SRC]) : nullptr;
+    b->dd_topk_idx = dd ? reinterpret_cast<int32_t*>(w + p.off[R_DD_TOPK_IDX]) : nullptr;
+    b->dd_topk_w = dd ? reinterpret_cast<float*>(w + p.off[R_DD_TOPK_W]) : nullptr;
+    b->partial = dd ? reinterpret_cast<uint16_t*>(w + p.off[R_PARTIAL]) : nullptr;
     int prev = 0;
     cudaGetDevice(&prev);
     if (prev != dev) cudaSetDevice(dev);
@@ -318,6 +344,66 @@ ep_status_t ep_combine(ep_buffer_t* b, int T, const void* d_y, const float* d_y_
     if (d_y_scale && (uintptr_t)d_y_scale % 4 != 0) return fail(EP_ERR_INVALID, "d_y_scale must be 4-byte aligned");
     cudaError_t e = ep::launch_combine(*b, T, d_y, d_y_scale, d_out, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    return ok();
+}
+
+ep_status_t ep_buffer_dedup(const ep_buffer_t* b, int32_t** tok_row, int32_t** rank_row_off, int32_t** rank_src_off,
+                            void** dd_x, float** dd_scale, int32_t** dd_src, int32_t** dd_topk_idx, float** dd_topk_w,
+                            uint16_t** partial, int64_t* max_rows) {
+    if (ep_status_t st = check_buf(b)) return st;
+    if (!(b->cfg.flags & EP_FLAG_DEDUP)) return fail(EP_ERR_INVALID, "buffer was created without EP_FLAG_DEDUP");
+    if (tok_row) *tok_row = b->tok_row;
+    if (rank_row_off) *rank_row_off = b->rank_row_off;
+    if (rank_src_off) *rank_src_off = b->rank_src_off;
+    if (dd_x) *dd_x = b->dd_x;
+    if (dd_scale) *dd_scale = b->dd_scale;
+    if (dd_src) *dd_src = b->dd_src;
+    if (dd_topk_idx) *dd_topk_idx = b->dd_topk_idx;
+    if (dd_topk_w) *dd_topk_w = b->dd_topk_w;
+    if (partial) *partial = b->partial;
+    if (max_rows) *max_rows = b->d_max;
+    return ok();
+}
+
+static ep_status_t check_dedup_call(const ep_buffer_t* b, int T) {
+    if (ep_status_t st = check_buf(b)) return st;
+    if (!(b->cfg.flags & EP_FLAG_DEDUP)) return fail(EP_ERR_INVALID, "buffer was created without EP_FLAG_DEDUP");
+    if (T != b->last_T) return fail(EP_ERR_INVALID, "T=%d does not match the last ep_get_layout (T=%d)", T, b->last_T);
+    return EP_OK;
+}
+
+ep_status_t ep_dispatch_dedup(ep_buffer_t* b, int T, const void* d_x, void* stream) {
+    if (ep_status_t st = check_dedup_call(b, T)) return st;
+    if (T > 0 && !d_x) return fail(EP_ERR_INVALID, "d_x is NULL");
+    if ((uintptr_t)d_x % 32 != 0) return fail(EP_ERR_INVALID, "d_x must be 32-byte aligned");
+    cudaError_t e = ep::launch_dispatch_dedup(*b, T, d_x, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dispatch_dedup launch");
+    return ok();
+}
+
+ep_status_t ep_permute(ep_buffer_t* b, int T, void* stream) {
+    if (ep_status_t st = check_dedup_call(b, T)) return st;
+    cudaError_t e = ep::launch_permute(*b, T, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "permute launch");
+    return ok();
+}
+
+ep_status_t ep_local_reduce(ep_buffer_t* b, int T, const void* d_y, const float* d_y_scale, void* stream) {
+    if (ep_status_t st = check_dedup_call(b, T)) return st;
+    if (T > 0 && !d_y) return fail(EP_ERR_INVALID, "d_y is NULL");
+    if ((uintptr_t)d_y % 32 != 0) return fail(EP_ERR_INVALID, "d_y must be 32-byte aligned");
+    if (d_y_scale && (uintptr_t)d_y_scale % 4 != 0) return fail(EP_ERR_INVALID, "d_y_scale must be 4-byte aligned");
+    cudaError_t e = ep::launch_local_reduce(*b, T, d_y, d_y_scale, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "local_reduce launch");
+    return ok();
+}
+
+ep_status_t ep_combine_dedup(ep_buffer_t* b, int T, void* d_out, void* stream) {
+    if (ep_status_t st = check_dedup_call(b, T)) return st;
+    if (T > 0 && !d_out) return fail(EP_ERR_INVALID, "d_out is NULL");
+    if ((uintptr_t)d_out % 32 != 0) return fail(EP_ERR_INVALID, "d_out must be 32-byte aligned");
+    cudaError_t e = ep::launch_combine_dedup(*b, T, d_out, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "combine_dedup launch");
     return ok();
 }
 

@@ -28,6 +28,17 @@ struct ep_buffer {
     int32_t* dst_row;
     // layout scratch (device): barrier words, per-chunk counts and prefixes
     int32_t* scratch;
+    // deduplicated receive (EP_FLAG_DEDUP; device)
+    int64_t d_max;  // R * T_max * min(R, K) rows
+    int32_t* tok_row;       // [N_max, R]
+    int32_t* rank_row_off;  // [R + 1]
+    int32_t* rank_src_off;  // [R, R]
+    void* dd_x;             // [d_max, H] bf16 or e4m3
+    float* dd_scale;        // [d_max, H/128] (FP8)
+    int32_t* dd_src;        // [d_max]
+    int32_t* dd_topk_idx;   // [d_max, K]
+    float* dd_topk_w;       // [d_max, K]
+    uint16_t* partial;      // [d_max, H] bf16
     uint32_t* err;  // device error word
     // receive buffers (device)
     void* recv_x;
@@ -57,6 +68,9 @@ struct LayoutArgs {
     int64_t m_max;            // rows the receive side holds (bound check)
     int low_latency;          // fixed (expert, source rank) regions of T_max rows
     int T_max;                // region size in low-latency mode
+    int32_t* tok_row = nullptr;       // dedup outputs (NULL: not wanted)
+    int32_t* rank_row_off = nullptr;
+    int32_t* rank_src_off = nullptr;
 };
 
 // int32 entries of layout scratch for a grid of at most max_ctas CTAs:
@@ -75,6 +89,10 @@ cudaError_t launch_layout(const ep_buffer& b, const LayoutArgs& a, cudaStream_t 
 // (words: 4 device uint32; [2] receives the error bits).
 cudaError_t launch_barrier_timeout_selftest(uint32_t* words, unsigned long long limit_ns, cudaStream_t stream);
 cudaError_t launch_dispatch(const ep_buffer& b, int T, const void* x, cudaStream_t stream);
+cudaError_t launch_dispatch_dedup(const ep_buffer& b, int T, const void* x, cudaStream_t stream);
+cudaError_t launch_permute(const ep_buffer& b, int T, cudaStream_t stream);
+cudaError_t launch_local_reduce(const ep_buffer& b, int T, const void* y, const float* y_scale, cudaStream_t stream);
+cudaError_t launch_combine_dedup(const ep_buffer& b, int T, void* out, cudaStream_t stream);
 cudaError_t launch_combine(const ep_buffer& b, int T, const void* y, const float* y_scale, void* out,
                            cudaStream_t stream);
 

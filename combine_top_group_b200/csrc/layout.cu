@@ -64,6 +64,8 @@ struct LayoutParams {
     int64_t m_max;
     int ll;     // low-latency layout: row = (e*R + s)*T_max + j
     int T_max;  // region size (low-latency layout)
+    int dedup;  // also place one row per (token, destination rank)
+    int32_t *tok_row, *rank_row_off, *rank_src_off;  // dedup outputs
     uint32_t* err;
     uint32_t* bar;  // [2]: barrier arrivals, finished CTAs; both 0 between launches
 };
@@ -449,6 +451,7 @@ __global__ void __launch_bounds__(kThreads, 2) layout_kernel(LayoutParams p) {
                 p.cnt[(int64_t)r * p.E + col] = b - a;
             } else {
                 p.ntpr[(int64_t)r * p.R + (col - p.E)] = b - a;
+                if (p.dedup) p.rank_src_off[(int64_t)(col - p.E) * p.R + r] = a;
             }
         }
         if (threadIdx.x == 0) {
@@ -466,7 +469,36 @@ __global__ void __launch_bounds__(kThreads, 2) layout_kernel(LayoutParams p) {
         for (int e = threadIdx.x; e <= p.E; e += kThreads) p.expert_off[e] = eoff[e];
         for (int r = threadIdx.x; r <= p.R; r += kThreads) p.rank_off[r] = eoff[r * p.L];
     }
+    __shared__ int s_rr[33];  // dedup: rows per destination rank, exclusive prefix
+    if (p.dedup) {
+        if (warp == 0) {
+            const int v = (lane < p.R) ? p.tot[p.E + lane] : 0;
+            int incl = v;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_up_sync(FULL, incl, off);
+                if (lane >= off) incl += o;
+            }
+            if (lane < p.R) s_rr[lane] = incl - v;
+            if (lane == p.R - 1) s_rr[p.R] = incl;
+        }
+        __syncthreads();
+        if (blockIdx.x == 0)
+            for (int r = threadIdx.x; r <= p.R; r += kThreads) p.rank_row_off[r] = s_rr[r];
+    }
     if (has_chunk) {
+        if (p.dedup) {
+            for (int r = threadIdx.x; r < p.R; r += kThreads) {
+                const int j = p.E + r;
+                int run = s_rr[r] + p.chunk[(int64_t)j * p.nc + c];
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) {
+                    const int x = hist[w * p.J + j];
+                    hist[w * p.J + j] = run;
+                    run += x;
+                }
+            }
+        }
         for (int e = threadIdx.x; e < p.E; e += kThreads) {
             // standard: expert block + chunk prefix. Low-latency: fixed region of
             // (e, s) + this rank's part of the chunk prefix
@@ -504,6 +536,22 @@ __global__ void __launch_bounds__(kThreads, 2) layout_kernel(LayoutParams p) {
             __syncwarp();
             if (valid && (peers >> lane) == 1u) my_hist[e] += __popc(peers);  // highest lane of the group
             __syncwarp();
+        }
+        if (p.dedup) {
+            // one row per (token, destination rank), tokens in order: lane = token
+            for (int t0w = w0; t0w < w1; t0w += 32) {
+                const int t = t0w + lane;
+                const bool active = t < w1;
+                const int64_t g = (int64_t)s * p.T + t;
+                for (int r = 0; r < p.R; ++r) {
+                    const bool in = active && p.itr[g * p.R + r] != 0;
+                    const unsigned bal = __ballot_sync(FULL, in);
+                    if (active) p.tok_row[g * p.R + r] = in ? my_hist[p.E + r] + __popc(bal & lt) : -1;
+                    __syncwarp();
+                    if (lane == 0) my_hist[p.E + r] += __popc(bal);
+                    __syncwarp();
+                }
+            }
         }
     }
 
@@ -628,6 +676,10 @@ cudaError_t launch_layout_raw(const ep_config_t& c, const LayoutArgs& a, const e
     p.m_max = a.m_max;
     p.ll = a.low_latency;
     p.T_max = a.T_max;
+    p.dedup = a.tok_row != nullptr;
+    p.tok_row = a.tok_row;
+    p.rank_row_off = a.rank_row_off;
+    p.rank_src_off = a.rank_src_off;
     p.err = err;
     // scratch: [control][chunk J*max_ctas][tot J]
     p.bar = reinterpret_cast<uint32_t*>(scratch);
@@ -658,6 +710,11 @@ cudaError_t launch_layout(const ep_buffer& b, const LayoutArgs& a, cudaStream_t 
     aa.m_max = b.m_max;
     aa.low_latency = (b.cfg.flags & EP_FLAG_LOW_LATENCY) ? 1 : 0;
     aa.T_max = b.cfg.max_tokens_per_rank;
+    if (b.cfg.flags & EP_FLAG_DEDUP) {
+        aa.tok_row = b.tok_row;
+        aa.rank_row_off = b.rank_row_off;
+        aa.rank_src_off = b.rank_src_off;
+    }
     return launch_layout_raw(b.cfg, aa, out, b.scratch, kMaxLayoutCtas, b.err, st);
 }
 

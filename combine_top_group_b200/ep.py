@@ -27,6 +27,7 @@ EP_OK, EP_ERR_INVALID, EP_ERR_CAPACITY, EP_ERR_OOM, EP_ERR_CUDA, EP_ERR_UNSUPPOR
 EP_DEVERR_EXPERT_ID, EP_DEVERR_ROW_BOUNDS, EP_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 EP_FLAG_FP8 = 0x1
 EP_FLAG_LOW_LATENCY = 0x2
+EP_FLAG_DEDUP = 0x4
 EP_ROUTE_SOFTMAX, EP_ROUTE_SOFTMAX_RENORM, EP_ROUTE_GROUP_SIGMOID = 0, 1, 2
 
 
@@ -75,6 +76,16 @@ _lib.ep_check_errors.restype = _st
 _lib.ep_get_layout_noalloc.argtypes = [ctypes.POINTER(EpConfig), ctypes.c_int, _P, _P, _P, ctypes.c_int,
                                        ctypes.c_uint64, ctypes.c_float, ctypes.POINTER(EpLayout), _P, _P]
 _lib.ep_get_layout_noalloc.restype = _st
+_lib.ep_buffer_dedup.argtypes = [_P] + [ctypes.POINTER(_P)] * 9 + [ctypes.POINTER(ctypes.c_int64)]
+_lib.ep_buffer_dedup.restype = _st
+_lib.ep_dispatch_dedup.argtypes = [_P, ctypes.c_int, _P, _P]
+_lib.ep_dispatch_dedup.restype = _st
+_lib.ep_permute.argtypes = [_P, ctypes.c_int, _P]
+_lib.ep_permute.restype = _st
+_lib.ep_local_reduce.argtypes = [_P, ctypes.c_int, _P, _P, _P]
+_lib.ep_local_reduce.restype = _st
+_lib.ep_combine_dedup.argtypes = [_P, ctypes.c_int, _P, _P]
+_lib.ep_combine_dedup.restype = _st
 _lib.ep_selftest_wait_timeout.argtypes = [_P, ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint32), _P]
 _lib.ep_selftest_wait_timeout.restype = _st
 
@@ -82,7 +93,8 @@ EXPORTED = ("ep_abi_version", "ep_status_string", "ep_last_error_message", "ep_d
             "ep_buffer_workspace_bytes", "ep_buffer_create", "ep_buffer_destroy", "ep_buffer_set_num_sms",
             "ep_buffer_layout",
             "ep_buffer_recv", "ep_get_layout", "ep_dispatch", "ep_combine", "ep_check_errors",
-            "ep_get_layout_noalloc", "ep_selftest_wait_timeout")
+            "ep_get_layout_noalloc", "ep_selftest_wait_timeout", "ep_buffer_dedup", "ep_dispatch_dedup",
+            "ep_permute", "ep_local_reduce", "ep_combine_dedup")
 
 
 class EpError(RuntimeError):
@@ -247,6 +259,46 @@ def ep_check_errors(buf: EpBuffer, clear: bool = True, stream=None) -> int:
     if st not in (EP_OK, EP_ERR_DEVICE):
         _check(st, "ep_check_errors")
     return w.value
+
+
+def ep_buffer_dedup(buf: EpBuffer, T: int) -> dict:
+    """torch views of the deduplicated-receive layout and buffers."""
+    ptrs = [_P() for _ in range(9)]
+    d = ctypes.c_int64(0)
+    _check(_lib.ep_buffer_dedup(buf.handle, *[ctypes.byref(q) for q in ptrs], ctypes.byref(d)), "ep_buffer_dedup")
+    c = buf.cfg
+    R, K, H, N, D = c.num_ranks, c.topk, c.hidden, c.num_ranks * T, d.value
+    out = dict(max_rows=D,
+               tok_row=buf._view(ptrs[0].value, torch.int32, (N, R)),
+               rank_row_off=buf._view(ptrs[1].value, torch.int32, (R + 1,)),
+               rank_src_off=buf._view(ptrs[2].value, torch.int32, (R, R)),
+               dd_src=buf._view(ptrs[5].value, torch.int32, (D,)),
+               dd_topk_idx=buf._view(ptrs[6].value, torch.int32, (D, K)),
+               dd_topk_w=buf._view(ptrs[7].value, torch.float32, (D, K)),
+               partial=buf._view(ptrs[8].value, torch.bfloat16, (D, H)))
+    if buf.fp8:
+        out["dd_x"] = buf._view(ptrs[3].value, torch.uint8, (D, H))
+        out["dd_scale"] = buf._view(ptrs[4].value, torch.float32, (D, H // 128))
+    else:
+        out["dd_x"] = buf._view(ptrs[3].value, torch.bfloat16, (D, H))
+        out["dd_scale"] = None
+    return out
+
+
+def ep_dispatch_dedup(buf: EpBuffer, T: int, x, stream=None) -> None:
+    _check(_lib.ep_dispatch_dedup(buf.handle, T, _ptr(x), _stream(stream)), "ep_dispatch_dedup")
+
+
+def ep_permute(buf: EpBuffer, T: int, stream=None) -> None:
+    _check(_lib.ep_permute(buf.handle, T, _stream(stream)), "ep_permute")
+
+
+def ep_local_reduce(buf: EpBuffer, T: int, y, y_scale, stream=None) -> None:
+    _check(_lib.ep_local_reduce(buf.handle, T, _ptr(y), _ptr(y_scale), _stream(stream)), "ep_local_reduce")
+
+
+def ep_combine_dedup(buf: EpBuffer, T: int, out, stream=None) -> None:
+    _check(_lib.ep_combine_dedup(buf.handle, T, _ptr(out), _stream(stream)), "ep_combine_dedup")
 
 
 def ep_selftest_wait_timeout(words, limit_ns: int, stream=None) -> int:

@@ -17,11 +17,12 @@ from . import ep
 from . import workloads as wl
 
 
-def make_config(w: wl.Workload, num_sms: int = 0, T_max: int | None = None) -> ep.EpConfig:
+def make_config(w: wl.Workload, num_sms: int = 0, T_max: int | None = None, dedup: bool = False) -> ep.EpConfig:
     cfg = ep.ep_default_config(w.R, T_max or w.T, w.H, w.E, w.K)
     cfg.num_groups, cfg.topk_groups = w.G, w.KG
     cfg.num_sms = num_sms
-    cfg.flags = (ep.EP_FLAG_FP8 if w.fp8 else 0) | (ep.EP_FLAG_LOW_LATENCY if w.low_latency else 0)
+    cfg.flags = ((ep.EP_FLAG_FP8 if w.fp8 else 0) | (ep.EP_FLAG_LOW_LATENCY if w.low_latency else 0)
+                 | (ep.EP_FLAG_DEDUP if dedup else 0))
     return cfg
 
 
@@ -34,10 +35,12 @@ class Pipeline:
     """Buffers and inputs of one workload, resident on `device`."""
 
     def __init__(self, w: wl.Workload, seed: int = 0, device: str = "cuda", num_sms: int = 0,
-                 T_max: int | None = None, x: np.ndarray | None = None, logits: np.ndarray | None = None):
+                 T_max: int | None = None, x: np.ndarray | None = None, logits: np.ndarray | None = None,
+                 dedup: bool = False):
         self.w = w
         self.device = torch.device(device)
-        self.buf = ep.ep_buffer_create(make_config(w, num_sms, T_max), device=self.device)
+        self.buf = ep.ep_buffer_create(make_config(w, num_sms, T_max, dedup), device=self.device)
+        self.dd = ep.ep_buffer_dedup(self.buf, w.T) if dedup else None
         xs = wl.make_x(w, seed) if x is None else x
         ls = wl.make_logits(w, seed) if logits is None else logits
         self.x = torch.from_numpy(xs.view(np.int16)).view(torch.bfloat16).to(self.device)
@@ -97,6 +100,36 @@ class Pipeline:
             r1 = min(M, r0 + chunk_rows)
             v = q[r0:r1].view(torch.float8_e4m3fn).float().view(r1 - r0, -1, 128)
             self.y[r0:r1] = (v * s[r0:r1, :, None]).view(r1 - r0, -1).to(torch.bfloat16)
+
+    # --- deduplicated receive (EP_FLAG_DEDUP) ----------------------------------
+    def dispatch_dedup(self, stream=None):
+        ep.ep_dispatch_dedup(self.buf, self.w.T, self.x, stream=stream)
+
+    def permute(self, stream=None):
+        ep.ep_permute(self.buf, self.w.T, stream=stream)
+
+    def local_reduce(self, fused: bool = False, stream=None):
+        w = self.w
+        if not w.fp8:
+            ep.ep_local_reduce(self.buf, w.T, self.recv["recv_x"], None, stream=stream)
+        elif fused:
+            ep.ep_local_reduce(self.buf, w.T, self.recv["recv_x"], self.recv["recv_scale"], stream=stream)
+        else:
+            assert self.y is not None, "run identity_expert() first"
+            ep.ep_local_reduce(self.buf, w.T, self.y, None, stream=stream)
+
+    def combine_dedup(self, stream=None):
+        ep.ep_combine_dedup(self.buf, self.w.T, self.out, stream=stream)
+
+    def dedup_rows(self) -> int:
+        return int(self.dd["rank_row_off"][-1].item())
+
+    def step_dedup(self, stream=None, fused: bool = False):
+        self.layout(stream)
+        self.dispatch_dedup(stream)
+        self.permute(stream)
+        self.local_reduce(fused=fused, stream=stream)
+        self.combine_dedup(stream)
 
     def step(self, stream=None, fused: bool = False):
         self.layout(stream)

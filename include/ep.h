@@ -69,6 +69,13 @@ typedef enum {
  * region overflows only if a caller's top-k repeats an expert; the extra
  * slots are dropped with EP_DEVERR_ROW_BOUNDS. */
 #define EP_FLAG_LOW_LATENCY 0x2u
+/* Deduplicated receive (DeepEP overlap notes, §节点内通信: a token is sent only
+ * to the ranks is_token_in_rank marks). The buffer also holds one row per
+ * (token, destination rank): at most R*T_max*min(R, K) rows, ordered by
+ * (destination rank, source rank, token). ep_get_layout then also fills the
+ * dedup layout (ep_buffer_dedup), and ep_dispatch_dedup, ep_permute,
+ * ep_local_reduce and ep_combine_dedup become available. */
+#define EP_FLAG_DEDUP 0x4u
 
 /* Routing rule applied by ep_get_layout to router logits. */
 typedef enum {
@@ -210,6 +217,50 @@ ep_status_t ep_combine(ep_buffer_t *buf, int T, const void *d_y, const float *d_
  * EP_DEVERR_TIMEOUT, call it with clear != 0 before the next ep_get_layout. Returns EP_ERR_DEVICE if any bit was set, EP_OK if
  * none, EP_ERR_CUDA on a CUDA failure. */
 ep_status_t ep_check_errors(ep_buffer_t *buf, uint32_t *word, int clear, void *stream);
+
+/* ---- deduplicated receive (EP_FLAG_DEDUP) ---------------------------------
+ * DeepEP overlap notes, §节点内通信: a token travels only to the ranks
+ * is_token_in_rank marks, once per rank. The receiving rank then:
+ *  - permutes the rows into expert order for its experts;
+ *  - reduces its experts' outputs into one bf16 partial row per (token, rank);
+ *  - hands the partials back, where they are summed across ranks.
+ * All calls below need a buffer created with EP_FLAG_DEDUP, and T equal to the
+ * last ep_get_layout's. They are stream-ordered, so each call follows the one
+ * before it on the same stream. */
+
+/* Device views of the dedup layout and buffers:
+ *  tok_row      int32 [N, R]: row of token g on rank r, -1 if not sent;
+ *  rank_row_off int32 [R+1]: exclusive prefix of the rows per destination rank (D = rank_row_off[R]);
+ *  rank_src_off int32 [R, R]: [r][s] = offset of source s inside rank r's rows;
+ *  dd_x         [D_max, H]: bf16, or e4m3 with dd_scale fp32 [D_max, H/128] (EP_FLAG_FP8);
+ *  dd_src       int32 [D_max]: source token of each row;
+ *  dd_topk_idx  int32 [D_max, K]: the token's top-k, -1 where the expert is not on this rank;
+ *  dd_topk_w    fp32 [D_max, K]: the matching weights (0 where -1);
+ *  partial      bf16 [D_max, H]: ep_local_reduce output.
+ * D_max = R*T_max*min(R, K). Any out-pointer may be NULL. */
+ep_status_t ep_buffer_dedup(const ep_buffer_t *buf, int32_t **tok_row, int32_t **rank_row_off,
+                            int32_t **rank_src_off, void **dd_x, float **dd_scale, int32_t **dd_src,
+                            int32_t **dd_topk_idx, float **dd_topk_w, uint16_t **partial, int64_t *max_rows);
+
+/* Dedup dispatch: for every rank r with tok_row[g][r] != -1, row tok_row[g][r]
+ * gets x[g] (bf16 copy, or the same FP8 cast as ep_dispatch), g, and the
+ * localised top-k. d_x as for ep_dispatch. Errors: EP_ERR_INVALID. */
+ep_status_t ep_dispatch_dedup(ep_buffer_t *buf, int T, const void *d_x, void *stream);
+
+/* Local expert permutation: each dedup row is copied to the expert-grouped
+ * receive row (recv_x, recv_scale, recv_src, recv_w, as ep_dispatch writes
+ * them) of each of its local slots. Follows ep_dispatch_dedup. */
+ep_status_t ep_permute(ep_buffer_t *buf, int T, void *stream);
+
+/* Local reduce: partial[d] = bf16( sum over the row's local slots k
+ * ascending, fp32 fma, of w * y[dst_row[g][k]] ). y as for ep_combine (bf16,
+ * or e4m3 + d_y_scale), 32-byte aligned. */
+ep_status_t ep_local_reduce(ep_buffer_t *buf, int T, const void *d_y, const float *d_y_scale, void *stream);
+
+/* Dedup combine: out[g] = bf16( sum over ranks r ascending, fp32, of
+ * partial[tok_row[g][r]] ); +0 for a token sent nowhere. d_out bf16 [N, H],
+ * 32-byte aligned. */
+ep_status_t ep_combine_dedup(ep_buffer_t *buf, int T, void *d_out, void *stream);
 
 /* Diagnostic: proves that the library's bounded waits end. Runs the layout's
  * grid barrier on 2 CTAs with a target that can never be reached, and a limit
