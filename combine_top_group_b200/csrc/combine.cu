@@ -34,112 +34,103 @@ struct CombineParams {
     uint32_t* err;
 };
 
-constexpr int kMaxK = 32;
 constexpr int kChunk = 8;  // slots gathered per pass: kChunk loads in flight per thread
 
-// Rows and weights of token g's slots into shared memory. A row outside the
-// buffer is reported and treated as masked.
-__device__ __forceinline__ void stage_slots(const CombineParams& p, int64_t g, int32_t* s_row, float* s_w) {
-    const int t = threadIdx.x;
-    if (t < p.K) {
-        int32_t r = __ldg(p.dst_row + g * p.K + t);
-        if (r >= p.m_max) {
-            set_error(p.err, EP_DEVERR_ROW_BOUNDS);
-            r = -1;
-        }
-        s_row[t] = r;
-        s_w[t] = __ldg(p.topk_w + g * p.K + t);
-    }
-    __syncthreads();
+// Receive row of slot k, read by every thread (broadcast, L1 after the first
+// warp) so that no warp waits on another; -1 for masked or out-of-range rows.
+__device__ __forceinline__ int32_t row_of(const CombineParams& p, int64_t g, int k) {
+    const int32_t r = __ldg(p.dst_row + g * p.K + k);
+    return (r < p.m_max) ? r : -1;
+}
+
+__device__ __forceinline__ void report_rows(const CombineParams& p, int64_t g) {
+    if (threadIdx.x < p.K && __ldg(p.dst_row + g * p.K + threadIdx.x) >= p.m_max)
+        set_error(p.err, EP_DEVERR_ROW_BOUNDS);
 }
 
 __global__ void __launch_bounds__(kCombineThreads) combine_bf16_kernel(CombineParams p) {
-    __shared__ int32_t s_row[kMaxK];
-    __shared__ float s_w[kMaxK];
-    for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {  // grid-stride when num_sms caps the grid
-    stage_slots(p, g, s_row, s_w);
     const int nvec = p.H / 16;  // 32-byte vectors: 16 bf16 channels
     const size_t rb = (size_t)p.H * 2;
-    for (int v = threadIdx.x; v < nvec; v += kCombineThreads) {
-        float acc[16];
+    for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {  // grid-stride when num_sms caps the grid
+        report_rows(p, g);
+        for (int v = threadIdx.x; v < nvec; v += kCombineThreads) {
+            float acc[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
-        for (int k0 = 0; k0 < p.K; k0 += kChunk) {
-            u32x8 q[kChunk];
-            int32_t row[kChunk];
+            for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
+            for (int k0 = 0; k0 < p.K; k0 += kChunk) {
+                u32x8 q[kChunk];
+                int32_t row[kChunk];
+                float w[kChunk];
 #pragma unroll
-            for (int i = 0; i < kChunk; ++i) {
-                row[i] = (k0 + i < p.K) ? s_row[k0 + i] : -1;
-                if (row[i] >= 0) q[i] = ld256_stream(p.y + (size_t)row[i] * rb + (size_t)v * 32);
-            }
+                for (int i = 0; i < kChunk; ++i) {
+                    row[i] = (k0 + i < p.K) ? row_of(p, g, k0 + i) : -1;
+                    w[i] = (row[i] >= 0) ? __ldg(p.topk_w + g * p.K + k0 + i) : 0.0f;
+                    if (row[i] >= 0) q[i] = ld256_stream(p.y + (size_t)row[i] * rb + (size_t)v * 32);
+                }
 #pragma unroll
-            for (int i = 0; i < kChunk; ++i) {
-                if (row[i] >= 0) {
-                    const float w = s_w[k0 + i];
+                for (int i = 0; i < kChunk; ++i) {
+                    if (row[i] >= 0) {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        acc[2 * j] = __fmaf_rn(w, bf16lo(q[i].v[j]), acc[2 * j]);
-                        acc[2 * j + 1] = __fmaf_rn(w, bf16hi(q[i].v[j]), acc[2 * j + 1]);
+                        for (int j = 0; j < 8; ++j) {
+                            acc[2 * j] = __fmaf_rn(w[i], bf16lo(q[i].v[j]), acc[2 * j]);
+                            acc[2 * j + 1] = __fmaf_rn(w[i], bf16hi(q[i].v[j]), acc[2 * j + 1]);
+                        }
                     }
                 }
             }
-        }
-        u32x8 o;
+            u32x8 o;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) o.v[j] = pack_bf16x2(acc[2 * j], acc[2 * j + 1]);
-        st256(p.out + (size_t)g * rb + (size_t)v * 32, o);
-    }
-    __syncthreads();  // s_row / s_w are rewritten by the next token
+            for (int j = 0; j < 8; ++j) o.v[j] = pack_bf16x2(acc[2 * j], acc[2 * j + 1]);
+            st256(p.out + (size_t)g * rb + (size_t)v * 32, o);
+        }
     }
 }
 
 __global__ void __launch_bounds__(kCombineThreads) combine_fp8_kernel(CombineParams p) {
-    __shared__ int32_t s_row[kMaxK];
-    __shared__ float s_w[kMaxK];
-    for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {  // grid-stride when num_sms caps the grid
-    stage_slots(p, g, s_row, s_w);
     const int nvec = p.H / 16;  // 16 e4m3 channels (16 B) per vector
     const int nb = p.H / 128;
     const size_t rb = (size_t)p.H;
-    for (int v = threadIdx.x; v < nvec; v += kCombineThreads) {
-        float acc[16];
+    for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {
+        report_rows(p, g);
+        for (int v = threadIdx.x; v < nvec; v += kCombineThreads) {
+            float acc[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
-        for (int k0 = 0; k0 < p.K; k0 += kChunk) {
-            uint4 q[kChunk];
-            float sc[kChunk];
-            int32_t row[kChunk];
+            for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
+            for (int k0 = 0; k0 < p.K; k0 += kChunk) {
+                uint4 q[kChunk];
+                float sc[kChunk];
+                int32_t row[kChunk];
+                float w[kChunk];
 #pragma unroll
-            for (int i = 0; i < kChunk; ++i) {
-                row[i] = (k0 + i < p.K) ? s_row[k0 + i] : -1;
-                if (row[i] >= 0) {
-                    q[i] = __ldcs(reinterpret_cast<const uint4*>(p.y + (size_t)row[i] * rb) + v);
-                    sc[i] = __ldg(p.y_scale + (size_t)row[i] * nb + v / 8);
+                for (int i = 0; i < kChunk; ++i) {
+                    row[i] = (k0 + i < p.K) ? row_of(p, g, k0 + i) : -1;
+                    w[i] = (row[i] >= 0) ? __ldg(p.topk_w + g * p.K + k0 + i) : 0.0f;
+                    if (row[i] >= 0) {
+                        q[i] = __ldcs(reinterpret_cast<const uint4*>(p.y + (size_t)row[i] * rb) + v);
+                        sc[i] = __ldg(p.y_scale + (size_t)row[i] * nb + v / 8);
+                    }
                 }
-            }
 #pragma unroll
-            for (int i = 0; i < kChunk; ++i) {
-                if (row[i] >= 0) {
-                    const float w = s_w[k0 + i];
-                    const uint32_t u[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+                for (int i = 0; i < kChunk; ++i) {
+                    if (row[i] >= 0) {
+                        const uint32_t u[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float2 a = unpack_e4m3x2(u[j] & 0xffffu);
-                        const float2 b = unpack_e4m3x2(u[j] >> 16);
-                        acc[4 * j + 0] = __fmaf_rn(w, __fmul_rn(a.x, sc[i]), acc[4 * j + 0]);
-                        acc[4 * j + 1] = __fmaf_rn(w, __fmul_rn(a.y, sc[i]), acc[4 * j + 1]);
-                        acc[4 * j + 2] = __fmaf_rn(w, __fmul_rn(b.x, sc[i]), acc[4 * j + 2]);
-                        acc[4 * j + 3] = __fmaf_rn(w, __fmul_rn(b.y, sc[i]), acc[4 * j + 3]);
+                        for (int j = 0; j < 4; ++j) {
+                            const float2 a = unpack_e4m3x2(u[j] & 0xffffu);
+                            const float2 b = unpack_e4m3x2(u[j] >> 16);
+                            acc[4 * j + 0] = __fmaf_rn(w[i], __fmul_rn(a.x, sc[i]), acc[4 * j + 0]);
+                            acc[4 * j + 1] = __fmaf_rn(w[i], __fmul_rn(a.y, sc[i]), acc[4 * j + 1]);
+                            acc[4 * j + 2] = __fmaf_rn(w[i], __fmul_rn(b.x, sc[i]), acc[4 * j + 2]);
+                            acc[4 * j + 3] = __fmaf_rn(w[i], __fmul_rn(b.y, sc[i]), acc[4 * j + 3]);
+                        }
                     }
                 }
             }
-        }
-        u32x8 o;
+            u32x8 o;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) o.v[j] = pack_bf16x2(acc[2 * j], acc[2 * j + 1]);
-        st256(p.out + (size_t)g * p.H * 2 + (size_t)v * 32, o);
-    }
-    __syncthreads();
+            for (int j = 0; j < 8; ++j) o.v[j] = pack_bf16x2(acc[2 * j], acc[2 * j + 1]);
+            st256(p.out + (size_t)g * p.H * 2 + (size_t)v * 32, o);
+        }
     }
 }
 
