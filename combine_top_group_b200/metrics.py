@@ -76,15 +76,41 @@ def hbm_peak() -> tuple[float, str]:
 
 # ---- ncu traffic (profiles/traffic.json) -------------------------------------
 
-def source_hash() -> str:
-    """Hash of every kernel source; a stored ncu traffic figure is only valid
-    for the sources it was captured from."""
+# The source files each kernel is built from: its own .cu (kernel + launcher)
+# and the shared headers. A stored traffic figure stays valid while these stay
+# unchanged, whatever happens to the other kernels.
+KERNEL_SOURCES = {
+    "layout": ("layout.cu",),
+    "dispatch": ("dispatch.cu",),
+    "combine": ("combine.cu",),
+    "dispatch_dedup": ("dedup.cu",),
+    "permute": ("dedup.cu",),
+    "local_reduce": ("dedup.cu",),
+    "combine_dedup": ("dedup.cu",),
+}
+SHARED_SOURCES = ("common.cuh", "internal.h")
+
+# ncu function names of each kernel (template instances share the name)
+NCU_NAMES = {
+    "layout": "layout_kernel",
+    "dispatch": ("dispatch_bf16_kernel", "dispatch_fp8_kernel"),
+    "combine": ("combine_bf16_kernel", "combine_fp8_kernel"),
+}
+
+
+def source_hash(kernel: str | None = None) -> str:
+    """Hash of the sources a kernel is built from (all kernel sources when
+    `kernel` is None); a stored ncu traffic figure is only valid for the
+    sources it was captured from."""
+    if kernel is None:
+        names = sorted(n for n in os.listdir(CSRC) if n.endswith((".cu", ".cuh", ".h")))
+    else:
+        names = sorted(set(KERNEL_SOURCES[kernel]) | set(SHARED_SOURCES))
     h = hashlib.sha256()
-    for name in sorted(os.listdir(CSRC)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(CSRC, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+    for name in names:
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -97,9 +123,74 @@ def stored_traffic(kernel: str, workload: str) -> float | None:
     except (OSError, ValueError):
         return None
     ent = data.get(workload, {}).get(kernel)
-    if not ent or ent.get("source_hash") != source_hash():
+    if not ent or ent.get("source_hash") != source_hash(kernel):
         return None
     return float(ent["dram_bytes_per_launch"])
+
+
+def _ncu_num(v: str) -> float:
+    return float(v.replace(",", ""))
+
+
+def parse_ncu_metrics(text: str) -> list[dict]:
+    """Rows of an `ncu --metrics ... --csv` log: one dict per (launch, metric)
+    with the kernel name, the launch id, the metric name, unit and value."""
+    lines = text.splitlines()
+    start = next((i for i, l in enumerate(lines) if l.startswith('"ID"')), None)
+    if start is None:
+        return []
+    rows = []
+    for r in csv.DictReader(io.StringIO("\n".join(lines[start:]))):
+        try:
+            rows.append({"id": int(r["ID"]), "kernel": r["Kernel Name"], "metric": r["Metric Name"],
+                         "unit": r["Metric Unit"], "value": _ncu_num(r["Metric Value"])})
+        except (KeyError, ValueError):
+            continue
+    return rows
+
+
+_UNIT_BYTES = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6, "GB": 1e9}
+
+
+def traffic_from_ncu(text: str) -> dict:
+    """Per kernel (layout / dispatch / combine): dram read and write bytes of
+    the last captured launch."""
+    per_launch: dict[int, dict] = {}
+    for r in parse_ncu_metrics(text):
+        ent = per_launch.setdefault(r["id"], {"kernel": r["kernel"]})
+        if r["metric"] in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            ent[r["metric"]] = r["value"] * _UNIT_BYTES.get(r["unit"], 1)
+    out = {}
+    for _, ent in sorted(per_launch.items()):
+        for kern, prefixes in NCU_NAMES.items():
+            names = (prefixes,) if isinstance(prefixes, str) else prefixes
+            if any(f"::{n}<" in ent["kernel"] or f"::{n}(" in ent["kernel"] for n in names) \
+                    and "dram__bytes_read.sum" in ent:
+                rd = int(ent["dram__bytes_read.sum"])
+                wr = int(ent.get("dram__bytes_write.sum", 0))
+                out[kern] = {"dram_bytes_per_launch": rd + wr, "dram_read": rd, "dram_write": wr,
+                             "source_hash": source_hash(kern)}
+    return out
+
+
+def record_traffic(csv_path: str, workload: str, command: str, note: str) -> dict:
+    """Writes the per-kernel dram bytes of an ncu capture into the traffic file
+    under `workload`, stamped with each kernel's source hash."""
+    with open(csv_path) as f:
+        ent = traffic_from_ncu(f.read())
+    try:
+        with open(TRAFFIC_FILE) as f:
+            data = json.load(f)
+    except (OSError, ValueError):
+        data = {}
+    slot = data.setdefault(workload, {})
+    slot.update(ent)
+    slot["command"] = command
+    slot["note"] = note
+    with open(TRAFFIC_FILE, "w") as f:
+        json.dump(data, f, indent=1, sort_keys=False)
+        f.write("\n")
+    return ent
 
 
 # ---- clocks ------------------------------------------------------------------
@@ -257,3 +348,14 @@ def clocks_rejected(clk: dict | None) -> str | None:
     if clk.get("sm_max_mhz") and clk["sm_mhz"] < 0.6 * clk["sm_max_mhz"] and not clk.get("reasons"):
         return "SM clock far below max with no reason (clock lock?)"
     return None
+
+
+if __name__ == "__main__":
+    import argparse
+    ap = argparse.ArgumentParser(description="record ncu dram traffic per kernel")
+    ap.add_argument("csv")
+    ap.add_argument("workload")
+    ap.add_argument("--command", required=True)
+    ap.add_argument("--note", default="")
+    a = ap.parse_args()
+    print(json.dumps(record_traffic(a.csv, a.workload, a.command, a.note), indent=1))

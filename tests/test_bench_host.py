@@ -91,3 +91,38 @@ def test_reference_arm_other_ranks_exit_quietly():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "tiny",
                         "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=300, env=env)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+NCU_CSV = '''==PROF== Connected to process 1
+"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Block Size","Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"
+"0","1","python3.12","h","void unnamed>::layout_kernel<8>(unnamed>::LayoutParams)","1","7","(256, 1, 1)","(296, 1, 1)","0","10.0","m","dram__bytes_read.sum","Mbyte","33.63"
+"0","1","python3.12","h","void unnamed>::layout_kernel<8>(unnamed>::LayoutParams)","1","7","(256, 1, 1)","(296, 1, 1)","0","10.0","m","dram__bytes_write.sum","byte","0"
+"1","1","python3.12","h","void unnamed>::dispatch_bf16_kernel<1>(unnamed>::DispatchParams)","1","7","(448, 1, 1)","(32768, 1, 1)","0","10.0","m","dram__bytes_read.sum","byte","472,184,064"
+"1","1","python3.12","h","void unnamed>::dispatch_bf16_kernel<1>(unnamed>::DispatchParams)","1","7","(448, 1, 1)","(32768, 1, 1)","0","10.0","m","dram__bytes_write.sum","byte","3698034176"
+"2","1","python3.12","h","void unnamed>::combine_dedup_kernel(unnamed>::P)","1","7","(128, 1, 1)","(10, 1, 1)","0","10.0","m","dram__bytes_read.sum","byte","5"
+"3","1","python3.12","h","void unnamed>::combine_bf16_kernel<1>(unnamed>::CombineParams)","1","7","(128, 1, 1)","(32768, 1, 1)","0","10.0","m","dram__bytes_read.sum","Gbyte","3.76"
+"3","1","python3.12","h","void unnamed>::combine_bf16_kernel<1>(unnamed>::CombineParams)","1","7","(128, 1, 1)","(32768, 1, 1)","0","10.0","m","dram__bytes_write.sum","Mbyte","458.6"
+'''
+
+
+def test_ncu_traffic_parse_and_hash(tmp_path, monkeypatch):
+    t = metrics.traffic_from_ncu(NCU_CSV)
+    assert set(t) == {"layout", "dispatch", "combine"}  # combine_dedup is not the combine kernel
+    assert t["layout"]["dram_bytes_per_launch"] == 33_630_000
+    assert t["dispatch"]["dram_read"] == 472_184_064 and t["dispatch"]["dram_write"] == 3_698_034_176
+    assert t["combine"]["dram_bytes_per_launch"] == 3_760_000_000 + 458_600_000
+    # per-kernel hashes: each kernel's figure is tied to its own sources only
+    assert t["dispatch"]["source_hash"] == metrics.source_hash("dispatch")
+    assert len({metrics.source_hash(k) for k in ("layout", "dispatch", "combine")}) == 3
+    f = tmp_path / "traffic.json"
+    c = tmp_path / "ncu.csv"
+    c.write_text(NCU_CSV)
+    monkeypatch.setattr(metrics, "TRAFFIC_FILE", str(f))
+    metrics.record_traffic(str(c), "prefill", "ncu ...", "test")
+    assert metrics.stored_traffic("dispatch", "prefill") == 472_184_064 + 3_698_034_176
+    assert metrics.stored_traffic("dispatch", "large") is None
+    data = json.loads(f.read_text())
+    data["prefill"]["combine"]["source_hash"] = "0" * 16  # captured from other sources
+    f.write_text(json.dumps(data))
+    assert metrics.stored_traffic("combine", "prefill") is None
+    assert metrics.stored_traffic("dispatch", "prefill") is not None
