@@ -37,7 +37,8 @@ sys.path.insert(0, HERE)
 from combine_top_group_b200 import metrics  # noqa: E402
 from combine_top_group_b200 import workloads as wl  # noqa: E402
 
-ORACLE_SAMPLE_T = 128  # tokens per rank in the CPU oracle's bounded sample
+ORACLE_SAMPLE_T = 1024  # tokens per rank in the CPU oracle's bounded sample
+CPU_BASELINE_MIN_S = 10.0  # seconds of oracle work behind cpu_baseline
 
 
 def parse_args(argv=None):
@@ -75,37 +76,48 @@ def workload_desc(w: wl.Workload) -> dict:
 # CPU oracle (test infrastructure) as the timed baseline
 # ---------------------------------------------------------------------------
 
-def oracle_step_sample(w: wl.Workload, seed: int = 0):
-    """One oracle pass over a bounded sample of the workload: the same shape,
-    with ORACLE_SAMPLE_T tokens per rank. Returns (seconds, algorithmic
-    bytes)."""
-    import oracle  # test infrastructure: only this leg of the bench runs it
+def oracle_sample(w: wl.Workload, seed: int = 0):
+    """A bounded sample of the workload for the CPU oracle: the same shape with
+    ORACLE_SAMPLE_T tokens per rank, and its seeded inputs."""
     ws = w.with_tokens(min(w.T, ORACLE_SAMPLE_T))
-    x = wl.make_x(ws, seed)
-    logits = wl.make_logits(ws, seed)
+    return ws, wl.make_x(ws, seed), wl.make_logits(ws, seed)
+
+
+def oracle_step(ws: wl.Workload, x, logits):
+    """One oracle pass (route, layout, dispatch, identity expert, combine) over
+    the sample. Returns (seconds, algorithmic bytes)."""
+    import oracle  # test infrastructure: only the CPU legs of the bench run it
     t0 = time.perf_counter()
     res = oracle.run_path(x, logits, ws)
     dt = time.perf_counter() - t0
     M = res["M"]
-    nbytes = metrics.layout_bytes(ws) + metrics.dispatch_bytes(ws, M) + metrics.combine_bytes(ws, M)
-    return dt, nbytes, ws
+    return dt, metrics.layout_bytes(ws) + metrics.dispatch_bytes(ws, M) + metrics.combine_bytes(ws, M)
 
 
 def cpu_baseline(w: wl.Workload) -> dict:
-    dt, nbytes, ws = oracle_step_sample(w)
-    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"one full path (route, layout, dispatch, identity expert, combine) over "
-                      f"{ws.R}x{ws.T} tokens of the same shape; {dt:.2f} s single-threaded C"}
+    """The oracle on the host, repeated over the sample until CPU_BASELINE_MIN_S
+    of work has been timed."""
+    ws, x, logits = oracle_sample(w)
+    tot_t, tot_b, reps = 0.0, 0, 0
+    while tot_t < CPU_BASELINE_MIN_S:
+        dt, nb = oracle_step(ws, x, logits)
+        tot_t += dt
+        tot_b += nb
+        reps += 1
+    return {"value": tot_b / tot_t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{reps} passes of the whole path (route, layout, dispatch, identity expert, combine) "
+                      f"over {ws.R}x{ws.T} tokens of the same shape; {tot_t:.1f} s single-threaded C"}
 
 
 def run_reference(args, w: wl.Workload, rank: int, world: int):
     if rank != 0:
         return
+    ws, x, logits = oracle_sample(w)
     for _ in range(args.warmup):
-        oracle_step_sample(w)
+        oracle_step(ws, x, logits)
     tot_t, tot_b = 0.0, 0
     for _ in range(args.steps):
-        dt, nb, ws = oracle_step_sample(w)
+        dt, nb = oracle_step(ws, x, logits)
         tot_t += dt
         tot_b += nb
     value = tot_b / tot_t / 1e9
@@ -116,7 +128,8 @@ def run_reference(args, w: wl.Workload, rank: int, world: int):
         "vs_baseline": None, "dtype": "bf16" if not w.fp8 else "fp8_e4m3", "data": "synthetic",
         "config": workload_desc(w),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"each step: the whole path over {ws.R}x{ws.T} tokens of the same shape"},
+                         "sample": f"each step: the whole path over {ws.R}x{ws.T} tokens of the same shape "
+                                   f"(single-threaded C)"},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -199,7 +212,7 @@ def run_ours(args, w: wl.Workload, rank: int, world: int, local_rank: int):
     # end to end through the C ABI from pinned host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps=min(K, 5), world=world)
+        e2e = measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps=max(K, 8), world=world)
 
     peak, peak_src = metrics.hbm_peak()
     d_avg, c_avg = t_disp / K, t_comb / K
@@ -373,7 +386,13 @@ def measure_dedup(w, seed, dev, fused, steps):
 
 def measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps, world):
     """Same metric, through the C ABI, with the step's inputs copied in from
-    pinned host memory and its result copied back, inside the timed region."""
+    pinned host memory and its result copied back, inside the timed region.
+
+    Steps are double-buffered: device x / logits / out have two slots, the
+    host-to-device copies run on one copy stream and the device-to-host copies
+    on another, so step i+1's inputs and step i-1's result cross PCIe (full
+    duplex) while step i computes. Every step still copies all of its inputs
+    in and its whole result out."""
     import torch
     import torch.distributed as dist
     x_h = pipe.x.cpu().pin_memory()
@@ -381,31 +400,57 @@ def measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps, world):
     out_h = torch.empty(pipe.out.shape, dtype=pipe.out.dtype).pin_memory()
     h2d = x_h.numel() * x_h.element_size() + l_h.numel() * l_h.element_size()
     d2h = out_h.numel() * out_h.element_size()
+    xs = [pipe.x, torch.empty_like(pipe.x)]
+    ls = [pipe.logits, torch.empty_like(pipe.logits)]
+    outs = [pipe.out, torch.empty_like(pipe.out)]
+    keep = (pipe.x, pipe.logits, pipe.out)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
 
-    def one():
-        pipe.x.copy_(x_h, non_blocking=True)
-        pipe.logits.copy_(l_h, non_blocking=True)
+    def one(i):
+        k = i % 2
+        s_in.wait_event(comp_done[k])  # step i-2 has finished reading slot k's inputs
+        with torch.cuda.stream(s_in):
+            xs[k].copy_(x_h, non_blocking=True)
+            ls[k].copy_(l_h, non_blocking=True)
+        in_done[k].record(s_in)
+        stream.wait_event(in_done[k])
+        stream.wait_event(out_done[k])  # step i-2's result has left slot k
+        pipe.x, pipe.logits, pipe.out = xs[k], ls[k], outs[k]
         pipe.layout(stream)
         pipe.dispatch(stream)
         if w.fp8 and not fused:
             pipe.combine(fused=False, stream=stream)  # y made once from the same inputs
         else:
             pipe.combine(fused=fused, stream=stream)
-        out_h.copy_(pipe.out, non_blocking=True)
+        comp_done[k].record(stream)
+        s_out.wait_event(comp_done[k])
+        with torch.cuda.stream(s_out):
+            out_h.copy_(outs[k], non_blocking=True)
+        out_done[k].record(s_out)
 
-    one()
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(stream)
-    for _ in range(steps):
-        one()
-    e.record(stream)
-    torch.cuda.synchronize(dev)
+    try:
+        for i in range(2):  # warm-up; records every event once
+            one(i)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        s_in.wait_event(s)
+        for i in range(steps):
+            one(i)
+        stream.wait_event(out_done[(steps - 1) % 2])
+        stream.wait_event(out_done[steps % 2])
+        e.record(stream)
+        torch.cuda.synchronize(dev)
+    finally:
+        pipe.x, pipe.logits, pipe.out = keep
     t = metrics.max_over_ranks([s.elapsed_time(e) / 1e3], dev)[0]
     return {"value": world * bytes_step * steps / t / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": t / steps * 1e3}
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": t / steps * 1e3,
+            "copies": "pinned host buffers; H2D and D2H on two copy streams, double-buffered across steps"}
 
 
 def main(argv=None):
