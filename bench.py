@@ -60,6 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--dedup", action="store_true",
                     help="also time the deduplicated-receive pipeline (dispatch_dedup, permute, local_reduce, "
                          "combine_dedup) on the same workload")
+    ap.add_argument("--shard", action="store_true",
+                    help="also time the one-rank-per-GPU calls, R ranks emulated on this GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args(argv)
@@ -252,6 +254,9 @@ def run_ours(args, w: wl.Workload, rank: int, world: int, local_rank: int):
         out["overlap"] = measure_overlap(pipe, w, dev, fused)
     if args.dedup:
         out["dedup"] = measure_dedup(w, rank, dev, fused, steps=min(args.steps, 10))
+    if args.shard:
+        out["shard"] = (measure_shard(pipe, w, dev, fused, bytes_dispatch, bytes_combine, steps=min(args.steps, 10))
+                        if world == 1 else {"skipped": "the emulated ranks run on one GPU (--gpus 1)"})
     ep.ep_buffer_set_num_sms(pipe.buf, args.num_sms)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w)
@@ -381,6 +386,48 @@ def measure_dedup(w, seed, dev, fused, steps):
         res[n + "_us"] = t / steps * 1e6
         res[n + "_gbs"] = nb / (t / steps) / 1e9
     del pipe
+    return res
+
+
+def measure_shard(pipe, w, dev, fused, bytes_dispatch, bytes_combine, steps):
+    """The one-rank-per-GPU calls (EP_FLAG_SHARD) with all R ranks emulated on
+    this GPU: per step R layouts, the count all-gather (device copies), R
+    placements, R dispatches and R combines, each phase timed with events.
+    The same rows move as in the single-buffer path, so the same algorithmic
+    bytes apply."""
+    import torch
+
+    from combine_top_group_b200 import shard
+    stream = torch.cuda.current_stream(dev)
+    out = torch.empty_like(pipe.out)
+    em = shard.EmulatedRanks(w, pipe.x, pipe.logits, out)
+    em.step(stream)
+    if w.fp8 and not fused:
+        em.identity_expert()
+    if em.check_errors() != 0:
+        raise RuntimeError("device error word set in the one-rank-per-GPU path")
+    same = bool(torch.equal(out.view(torch.int16), pipe.out.view(torch.int16))) if not w.fp8 or fused else None
+    names = ["layout", "exchange", "place", "dispatch", "combine"]
+    calls = [lambda: em.layout(stream), lambda: em.exchange(stream), lambda: em.place(stream),
+             lambda: em.dispatch(stream), lambda: em.combine(stream)]
+    tot = [0.0] * len(calls)
+    for _ in range(steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+        ev[0].record(stream)
+        for i, c in enumerate(calls):
+            c()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize(dev)
+        for i in range(len(calls)):
+            tot[i] += ev[i].elapsed_time(ev[i + 1]) / 1e3
+    res = {"ranks": w.R, "steps": steps, "launches_per_step": 4 * w.R + 1 + w.R,
+           "out_equals_single_buffer": same, "received_rows": em.received_rows()}
+    for n, t in zip(names, tot):
+        res[n + "_us"] = t / steps * 1e6
+    res["dispatch_gbs"] = bytes_dispatch / (tot[3] / steps) / 1e9
+    res["combine_gbs"] = bytes_combine / (tot[4] / steps) / 1e9
+    res["step_us"] = sum(tot) / steps * 1e6
+    del em
     return res
 
 

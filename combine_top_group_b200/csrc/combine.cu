@@ -12,6 +12,11 @@
 // that column before any arithmetic, so K loads are in flight per thread.
 // Loads use the streaming cache hint (y is read once). The 32 output bytes
 // go out in one 256-bit store.
+//
+// The same kernels serve one rank of a one-process-per-GPU deployment (PeerY):
+// each slot's row is then read from the expert output of its destination
+// rank, through a table of that rank's device pointers (peer memory over
+// NVLink on a multi-GPU node).
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -30,8 +35,23 @@ struct CombineParams {
     const float* y_scale;
     const int32_t* dst_row;
     const float* topk_w;
+    const uint8_t* dst_rank;  // [N, K] destination rank of each slot (PeerY only)
+    int num_peers;
     uint8_t* out;
     uint32_t* err;
+};
+
+// Expert output of the single-buffer layout: one array holds every row.
+struct LocalY {
+    static constexpr bool kPeer = false;
+};
+
+// Expert output of every rank (device pointers, peer-mapped where the rank is
+// another GPU); scales only for FP8 y.
+struct PeerY {
+    static constexpr bool kPeer = true;
+    const uint8_t* y[kMaxPeers];
+    const float* scale[kMaxPeers];
 };
 
 constexpr int kChunk = 8;  // slots gathered per pass: kChunk loads in flight per thread
@@ -43,16 +63,29 @@ __device__ __forceinline__ int32_t row_of(const CombineParams& p, int64_t g, int
     return (r < p.m_max) ? r : -1;
 }
 
-__device__ __forceinline__ void report_rows(const CombineParams& p, int64_t g) {
-    if (threadIdx.x < p.K && __ldg(p.dst_row + g * p.K + threadIdx.x) >= p.m_max)
-        set_error(p.err, EP_DEVERR_ROW_BOUNDS);
+// Start of the row of slot k in y (PeerY): the destination rank's array.
+__device__ __forceinline__ const uint8_t* peer_row(const CombineParams& p, const PeerY& py, int64_t g, int k,
+                                                   int32_t r, size_t rb) {
+    const int d = __ldg(p.dst_rank + g * p.K + k);
+    return (d < p.num_peers) ? py.y[d] + (size_t)r * rb : nullptr;
 }
 
-__global__ void __launch_bounds__(kCombineThreads) combine_bf16_kernel(CombineParams p) {
+template <class Y>
+__device__ __forceinline__ void report_rows(const CombineParams& p, int64_t g) {
+    if (threadIdx.x < p.K) {
+        const int32_t r = __ldg(p.dst_row + g * p.K + threadIdx.x);
+        bool bad = r >= p.m_max;
+        if constexpr (Y::kPeer) bad = bad || (r >= 0 && __ldg(p.dst_rank + g * p.K + threadIdx.x) >= p.num_peers);
+        if (bad) set_error(p.err, EP_DEVERR_ROW_BOUNDS);
+    }
+}
+
+template <class Y>
+__global__ void __launch_bounds__(kCombineThreads) combine_bf16_kernel(CombineParams p, Y py) {
     const int nvec = p.H / 16;  // 32-byte vectors: 16 bf16 channels
     const size_t rb = (size_t)p.H * 2;
     for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {  // grid-stride when num_sms caps the grid
-        report_rows(p, g);
+        report_rows<Y>(p, g);
         for (int v = threadIdx.x; v < nvec; v += kCombineThreads) {
             float acc[16];
 #pragma unroll
@@ -64,8 +97,15 @@ __global__ void __launch_bounds__(kCombineThreads) combine_bf16_kernel(CombinePa
 #pragma unroll
                 for (int i = 0; i < kChunk; ++i) {
                     row[i] = (k0 + i < p.K) ? row_of(p, g, k0 + i) : -1;
-                    w[i] = (row[i] >= 0) ? __ldg(p.topk_w + g * p.K + k0 + i) : 0.0f;
-                    if (row[i] >= 0) q[i] = ld256_stream(p.y + (size_t)row[i] * rb + (size_t)v * 32);
+                    if constexpr (Y::kPeer) {
+                        const uint8_t* base = (row[i] >= 0) ? peer_row(p, py, g, k0 + i, row[i], rb) : nullptr;
+                        if (base == nullptr) row[i] = -1;
+                        w[i] = (row[i] >= 0) ? __ldg(p.topk_w + g * p.K + k0 + i) : 0.0f;
+                        if (row[i] >= 0) q[i] = ld256_stream(base + (size_t)v * 32);
+                    } else {
+                        w[i] = (row[i] >= 0) ? __ldg(p.topk_w + g * p.K + k0 + i) : 0.0f;
+                        if (row[i] >= 0) q[i] = ld256_stream(p.y + (size_t)row[i] * rb + (size_t)v * 32);
+                    }
                 }
 #pragma unroll
                 for (int i = 0; i < kChunk; ++i) {
@@ -86,12 +126,13 @@ __global__ void __launch_bounds__(kCombineThreads) combine_bf16_kernel(CombinePa
     }
 }
 
-__global__ void __launch_bounds__(kCombineThreads) combine_fp8_kernel(CombineParams p) {
+template <class Y>
+__global__ void __launch_bounds__(kCombineThreads) combine_fp8_kernel(CombineParams p, Y py) {
     const int nvec = p.H / 16;  // 16 e4m3 channels (16 B) per vector
     const int nb = p.H / 128;
     const size_t rb = (size_t)p.H;
     for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {
-        report_rows(p, g);
+        report_rows<Y>(p, g);
         for (int v = threadIdx.x; v < nvec; v += kCombineThreads) {
             float acc[16];
 #pragma unroll
@@ -104,10 +145,25 @@ __global__ void __launch_bounds__(kCombineThreads) combine_fp8_kernel(CombinePar
 #pragma unroll
                 for (int i = 0; i < kChunk; ++i) {
                     row[i] = (k0 + i < p.K) ? row_of(p, g, k0 + i) : -1;
+                    const uint8_t* base = nullptr;
+                    const float* sbase = p.y_scale;
+                    if constexpr (Y::kPeer) {
+                        if (row[i] >= 0) {
+                            const int d = __ldg(p.dst_rank + g * p.K + k0 + i);
+                            if (d < p.num_peers) {
+                                base = py.y[d] + (size_t)row[i] * rb;
+                                sbase = py.scale[d];
+                            } else {
+                                row[i] = -1;
+                            }
+                        }
+                    } else {
+                        base = p.y + (size_t)row[i] * rb;
+                    }
                     w[i] = (row[i] >= 0) ? __ldg(p.topk_w + g * p.K + k0 + i) : 0.0f;
                     if (row[i] >= 0) {
-                        q[i] = __ldcs(reinterpret_cast<const uint4*>(p.y + (size_t)row[i] * rb) + v);
-                        sc[i] = __ldg(p.y_scale + (size_t)row[i] * nb + v / 8);
+                        q[i] = __ldcs(reinterpret_cast<const uint4*>(base) + v);
+                        sc[i] = __ldg(sbase + (size_t)row[i] * nb + v / 8);
                     }
                 }
 #pragma unroll
@@ -134,25 +190,11 @@ __global__ void __launch_bounds__(kCombineThreads) combine_fp8_kernel(CombinePar
     }
 }
 
-}  // namespace
-
-cudaError_t launch_combine(const ep_buffer& b, int T, const void* y, const float* y_scale, void* out,
-                           cudaStream_t st) {
-    const ep_config_t& c = b.cfg;
-    CombineParams p{};
-    p.N = (int64_t)c.num_ranks * T;
-    p.K = c.topk;
-    p.H = c.hidden;
-    p.m_max = b.m_max;
-    p.y = static_cast<const uint8_t*>(y);
-    p.y_scale = y_scale;
-    p.dst_row = b.dst_row;
-    p.topk_w = b.topk_w;
-    p.out = static_cast<uint8_t*>(out);
-    p.err = b.err;
-    if (p.N == 0) return cudaSuccess;
-    auto kern = (y_scale == nullptr) ? combine_bf16_kernel : combine_fp8_kernel;
+template <class Y>
+cudaError_t launch_y(const ep_buffer& b, const CombineParams& p, const Y& py, bool fp8, cudaStream_t st) {
+    auto kern = fp8 ? combine_fp8_kernel<Y> : combine_bf16_kernel<Y>;
     int64_t grid = p.N;
+    const ep_config_t& c = b.cfg;
     const int sm_cap = (c.num_sms > 0 && c.num_sms < b.sm_count) ? c.num_sms : b.sm_count;
     if (sm_cap < b.sm_count) {
         // num_sms cap (Buffer.set_num_sms): a resident grid on sm_cap SMs' worth of CTAs
@@ -163,8 +205,47 @@ cudaError_t launch_combine(const ep_buffer& b, int T, const void* y, const float
         if (grid > p.N) grid = p.N;
     }
     if (grid > 0x7fffffff) grid = 0x7fffffff;
-    kern<<<(unsigned)grid, kCombineThreads, 0, st>>>(p);
+    kern<<<(unsigned)grid, kCombineThreads, 0, st>>>(p, py);
     return cudaGetLastError();
+}
+
+CombineParams params_of(const ep_buffer& b, int64_t N, const void* y, const float* y_scale, void* out) {
+    const ep_config_t& c = b.cfg;
+    CombineParams p{};
+    p.N = N;
+    p.K = c.topk;
+    p.H = c.hidden;
+    p.m_max = b.m_max;
+    p.y = static_cast<const uint8_t*>(y);
+    p.y_scale = y_scale;
+    p.dst_row = b.dst_row;
+    p.topk_w = b.topk_w;
+    p.out = static_cast<uint8_t*>(out);
+    p.err = b.err;
+    return p;
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const ep_buffer& b, int T, const void* y, const float* y_scale, void* out,
+                           cudaStream_t st) {
+    const CombineParams p = params_of(b, (int64_t)b.cfg.num_ranks * T, y, y_scale, out);
+    if (p.N == 0) return cudaSuccess;
+    return launch_y(b, p, LocalY{}, y_scale != nullptr, st);
+}
+
+cudaError_t launch_shard_combine(const ep_buffer& b, int T, const void* const* peer_y,
+                                 const float* const* peer_scale, void* out, cudaStream_t st) {
+    CombineParams p = params_of(b, T, nullptr, nullptr, out);
+    if (p.N == 0) return cudaSuccess;
+    p.dst_rank = b.dst_rank;
+    p.num_peers = b.cfg.num_ranks;
+    PeerY py{};
+    for (int d = 0; d < b.cfg.num_ranks; ++d) {
+        py.y[d] = static_cast<const uint8_t*>(peer_y[d]);
+        py.scale[d] = peer_scale ? peer_scale[d] : nullptr;
+    }
+    return launch_y(b, p, py, peer_scale != nullptr, st);
 }
 
 }  // namespace ep

@@ -197,4 +197,48 @@ __device__ __forceinline__ uint64_t splitmix64(uint64_t counter) {
 
 __device__ __forceinline__ void set_error(uint32_t* err, uint32_t bit) { atomicOr(err, bit); }
 
+// Exclusive scan of n <= 4 * blockDim.x values in[j * stride] into out[0..n],
+// with out[n] = total. Called by every thread of the block.
+__device__ inline void block_exclusive_scan(const int32_t* in, int stride, int n, int* out, int* warp_tot) {
+    const int t = threadIdx.x;
+    const int lane = t & 31, warp = t >> 5, nw = blockDim.x >> 5;
+    int v[4];
+    int local = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int j = 4 * t + i;
+        v[i] = (j < n) ? in[(int64_t)j * stride] : 0;
+        local += v[i];
+    }
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(FULL, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int wv = (lane < nw) ? warp_tot[lane] : 0;
+        int wi = wv;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(FULL, wi, off);
+            if (lane >= off) wi += o;
+        }
+        if (lane < nw) warp_tot[lane] = wi - wv;
+        if (lane == nw - 1) warp_tot[32] = wi;
+    }
+    __syncthreads();
+    int run = warp_tot[warp] + incl - local;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int j = 4 * t + i;
+        if (j < n) out[j] = run;
+        run += v[i];
+    }
+    if (t == 0) out[n] = warp_tot[32];
+    __syncthreads();
+}
+
 }  // namespace ep

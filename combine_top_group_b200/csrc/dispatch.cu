@@ -21,6 +21,11 @@
 // warp fetching the row indices itself, the warps drift apart, their rows
 // interleave, and prefill dispatch slows from 682 to 708 us.
 // Every row index is checked against the buffer (EP_DEVERR_ROW_BOUNDS).
+//
+// The same kernels serve one rank of a one-process-per-GPU deployment
+// (PeerRecv): each slot's row then goes to the receive buffer of its
+// destination rank, through a table of that rank's device pointers (peer
+// memory over NVLink on a multi-GPU node).
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -36,39 +41,78 @@ struct DispatchParams {
     const uint8_t* x;  // bf16 [N, H]
     const int32_t* dst_row;
     const float* topk_w;
-    uint8_t* recv_x;
-    float* recv_scale;
-    int32_t* recv_src;
-    float* recv_w;
+    const uint8_t* dst_rank;  // [N, K] destination rank of each slot (PeerRecv only)
+    int num_peers;            // entries of the PeerRecv tables
+    int64_t g_base;           // global id of local token 0 (recv_src)
     uint32_t* err;
+};
+
+// Receive arrays of the single-buffer layout: every row lives in this buffer.
+struct LocalRecv {
+    static constexpr bool kPeer = false;
+    uint8_t* x;
+    float* scale;
+    int32_t* src;
+    float* w;
+    __device__ __forceinline__ uint8_t* x_of(int) const { return x; }
+    __device__ __forceinline__ float* scale_of(int) const { return scale; }
+    __device__ __forceinline__ int32_t* src_of(int) const { return src; }
+    __device__ __forceinline__ float* w_of(int) const { return w; }
+};
+
+// Receive arrays of every destination rank (device pointers, peer-mapped
+// where the rank is another GPU).
+struct PeerRecv {
+    static constexpr bool kPeer = true;
+    uint8_t* x[kMaxPeers];
+    float* scale[kMaxPeers];
+    int32_t* src[kMaxPeers];
+    float* w[kMaxPeers];
+    __device__ __forceinline__ uint8_t* x_of(int d) const { return x[d]; }
+    __device__ __forceinline__ float* scale_of(int d) const { return scale[d]; }
+    __device__ __forceinline__ int32_t* src_of(int d) const { return src[d]; }
+    __device__ __forceinline__ float* w_of(int d) const { return w[d]; }
 };
 
 constexpr int kMaxK = 32;
 
-// Loads the token's K receive rows (checked) and writes recv_src / recv_w.
-__device__ __forceinline__ void stage_rows(const DispatchParams& p, int64_t g, int32_t* s_row) {
+// Loads the token's K receive rows (checked) and destination ranks, and
+// writes recv_src / recv_w.
+template <class Recv>
+__device__ __forceinline__ void stage_rows(const DispatchParams& p, const Recv& rv, int64_t g, int32_t* s_row,
+                                           int32_t* s_rank) {
     const int t = threadIdx.x;
     if (t < p.K) {
         int32_t r = __ldg(p.dst_row + g * p.K + t);
+        int d = 0;
+        if constexpr (Recv::kPeer) {
+            d = __ldg(p.dst_rank + g * p.K + t);
+            if (r >= 0 && d >= p.num_peers) {
+                set_error(p.err, EP_DEVERR_ROW_BOUNDS);
+                r = -1;
+            }
+            s_rank[t] = d;
+        }
         if (r >= p.m_max) {
             set_error(p.err, EP_DEVERR_ROW_BOUNDS);
             r = -1;
         }
         s_row[t] = r;
         if (r >= 0) {
-            p.recv_src[r] = (int32_t)g;
-            p.recv_w[r] = __ldg(p.topk_w + g * p.K + t);
+            rv.src_of(d)[r] = (int32_t)(p.g_base + g);
+            rv.w_of(d)[r] = __ldg(p.topk_w + g * p.K + t);
         }
     }
 }
 
-template <int VPT>
-__global__ void __launch_bounds__(512) dispatch_bf16_kernel(DispatchParams p) {
+template <int VPT, class Recv>
+__global__ void __launch_bounds__(512) dispatch_bf16_kernel(DispatchParams p, Recv rv) {
     __shared__ int32_t s_row[kMaxK];
+    __shared__ int32_t s_rank[Recv::kPeer ? kMaxK : 1];
     const int nv = p.H / 16;  // 32-byte vectors per bf16 row
     const size_t rb = (size_t)p.H * 2;
     for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {
-        stage_rows(p, g, s_row);
+        stage_rows(p, rv, g, s_row, s_rank);
         u32x8 v[VPT];
 #pragma unroll
         for (int j = 0; j < VPT; ++j) {
@@ -79,7 +123,7 @@ __global__ void __launch_bounds__(512) dispatch_bf16_kernel(DispatchParams p) {
         for (int k = 0; k < p.K; ++k) {
             const int32_t r = s_row[k];
             if (r < 0) continue;
-            uint8_t* dst = p.recv_x + (size_t)r * rb;
+            uint8_t* dst = rv.x_of(Recv::kPeer ? s_rank[k] : 0) + (size_t)r * rb;
 #pragma unroll
             for (int j = 0; j < VPT; ++j) {
                 const int c = threadIdx.x + j * blockDim.x;
@@ -90,15 +134,16 @@ __global__ void __launch_bounds__(512) dispatch_bf16_kernel(DispatchParams p) {
     }
 }
 
-template <int VPT>
-__global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchParams p) {
+template <int VPT, class Recv>
+__global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchParams p, Recv rv) {
     __shared__ int32_t s_row[kMaxK];
+    __shared__ int32_t s_rank[Recv::kPeer ? kMaxK : 1];
     const int nv = p.H / 16;  // 16-channel vectors per row: 32 B in, 16 B out
     const int nb = p.H / 128;
     const size_t rb_in = (size_t)p.H * 2;
     const int lane = threadIdx.x & 31;
     for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {
-        stage_rows(p, g, s_row);
+        stage_rows(p, rv, g, s_row, s_rank);
         uint4 q[VPT];
         float sc[VPT];
 #pragma unroll
@@ -131,13 +176,15 @@ __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchParams p) {
         for (int k = 0; k < p.K; ++k) {
             const int32_t r = s_row[k];
             if (r < 0) continue;
-            uint8_t* dst = p.recv_x + (size_t)r * p.H;
+            const int d = Recv::kPeer ? s_rank[k] : 0;
+            uint8_t* dst = rv.x_of(d) + (size_t)r * p.H;
+            float* scale = rv.scale_of(d);
 #pragma unroll
             for (int j = 0; j < VPT; ++j) {
                 const int c = threadIdx.x + j * blockDim.x;
                 if (c < nv) {
                     __stcs(reinterpret_cast<uint4*>(dst) + c, q[j]);
-                    if ((lane & 7) == 0) p.recv_scale[(size_t)r * nb + c / 8] = sc[j];
+                    if ((lane & 7) == 0) scale[(size_t)r * nb + c / 8] = sc[j];
                 }
             }
         }
@@ -145,9 +192,9 @@ __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchParams p) {
     }
 }
 
-template <typename KernelT>
-cudaError_t launch_rows(KernelT kernel, int threads, int sm_cap, int full_sms, const DispatchParams& p,
-                        cudaStream_t st) {
+template <class Recv>
+cudaError_t launch_rows(void (*kernel)(DispatchParams, Recv), int threads, int sm_cap, int full_sms,
+                        const DispatchParams& p, const Recv& rv, cudaStream_t st) {
     int64_t grid = p.N;
     if (sm_cap < full_sms) {
         // num_sms cap (Buffer.set_num_sms): a resident grid on sm_cap SMs' worth of CTAs
@@ -158,7 +205,7 @@ cudaError_t launch_rows(KernelT kernel, int threads, int sm_cap, int full_sms, c
         if (grid > p.N) grid = p.N;
     }
     if (grid > 0x7fffffff) grid = 0x7fffffff;
-    kernel<<<(unsigned)grid, threads, 0, st>>>(p);
+    kernel<<<(unsigned)grid, threads, 0, st>>>(p, rv);
     return cudaGetLastError();
 }
 
@@ -172,37 +219,67 @@ void shape_of(int H, int* threads, int* vpt) {
     *vpt = (nv + t - 1) / t;
 }
 
-}  // namespace
+template <class Recv>
+cudaError_t launch_any(const DispatchParams& p, const Recv& rv, bool fp8, int sm_cap, int full_sms,
+                       cudaStream_t st) {
+    int threads, vpt;
+    shape_of(p.H, &threads, &vpt);
+    if (!fp8) {
+        if (vpt <= 1) return launch_rows(dispatch_bf16_kernel<1, Recv>, threads, sm_cap, full_sms, p, rv, st);
+        if (vpt <= 2) return launch_rows(dispatch_bf16_kernel<2, Recv>, threads, sm_cap, full_sms, p, rv, st);
+        if (vpt <= 4) return launch_rows(dispatch_bf16_kernel<4, Recv>, threads, sm_cap, full_sms, p, rv, st);
+        return launch_rows(dispatch_bf16_kernel<8, Recv>, threads, sm_cap, full_sms, p, rv, st);
+    }
+    if (vpt <= 1) return launch_rows(dispatch_fp8_kernel<1, Recv>, threads, sm_cap, full_sms, p, rv, st);
+    if (vpt <= 2) return launch_rows(dispatch_fp8_kernel<2, Recv>, threads, sm_cap, full_sms, p, rv, st);
+    if (vpt <= 4) return launch_rows(dispatch_fp8_kernel<4, Recv>, threads, sm_cap, full_sms, p, rv, st);
+    return launch_rows(dispatch_fp8_kernel<8, Recv>, threads, sm_cap, full_sms, p, rv, st);
+}
 
-cudaError_t launch_dispatch(const ep_buffer& b, int T, const void* x, cudaStream_t st) {
+DispatchParams params_of(const ep_buffer& b, int64_t N, const void* x) {
     const ep_config_t& c = b.cfg;
     DispatchParams p{};
-    p.N = (int64_t)c.num_ranks * T;
+    p.N = N;
     p.K = c.topk;
     p.H = c.hidden;
     p.m_max = b.m_max;
     p.x = static_cast<const uint8_t*>(x);
     p.dst_row = b.dst_row;
     p.topk_w = b.topk_w;
-    p.recv_x = static_cast<uint8_t*>(b.recv_x);
-    p.recv_scale = b.recv_scale;
-    p.recv_src = b.recv_src;
-    p.recv_w = b.recv_w;
     p.err = b.err;
+    return p;
+}
+
+int sm_cap_of(const ep_buffer& b) {
+    const ep_config_t& c = b.cfg;
+    return (c.num_sms > 0 && c.num_sms < b.sm_count) ? c.num_sms : b.sm_count;
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const ep_buffer& b, int T, const void* x, cudaStream_t st) {
+    const DispatchParams p = params_of(b, (int64_t)b.cfg.num_ranks * T, x);
     if (p.N == 0) return cudaSuccess;
-    const int sm_cap = (c.num_sms > 0 && c.num_sms < b.sm_count) ? c.num_sms : b.sm_count;
-    int threads, vpt;
-    shape_of(p.H, &threads, &vpt);
-    if (!(c.flags & EP_FLAG_FP8)) {
-        if (vpt <= 1) return launch_rows(dispatch_bf16_kernel<1>, threads, sm_cap, b.sm_count, p, st);
-        if (vpt <= 2) return launch_rows(dispatch_bf16_kernel<2>, threads, sm_cap, b.sm_count, p, st);
-        if (vpt <= 4) return launch_rows(dispatch_bf16_kernel<4>, threads, sm_cap, b.sm_count, p, st);
-        return launch_rows(dispatch_bf16_kernel<8>, threads, sm_cap, b.sm_count, p, st);
+    LocalRecv rv{static_cast<uint8_t*>(b.recv_x), b.recv_scale, b.recv_src, b.recv_w};
+    return launch_any(p, rv, (b.cfg.flags & EP_FLAG_FP8) != 0, sm_cap_of(b), b.sm_count, st);
+}
+
+cudaError_t launch_shard_dispatch(const ep_buffer& b, int rank, int T, const void* x, void* const* peer_x,
+                                  float* const* peer_scale, int32_t* const* peer_src, float* const* peer_w,
+                                  cudaStream_t st) {
+    DispatchParams p = params_of(b, T, x);
+    if (p.N == 0) return cudaSuccess;
+    p.dst_rank = b.dst_rank;
+    p.num_peers = b.cfg.num_ranks;
+    p.g_base = (int64_t)rank * T;
+    PeerRecv rv{};
+    for (int d = 0; d < b.cfg.num_ranks; ++d) {
+        rv.x[d] = static_cast<uint8_t*>(peer_x[d]);
+        rv.scale[d] = peer_scale ? peer_scale[d] : nullptr;
+        rv.src[d] = peer_src[d];
+        rv.w[d] = peer_w[d];
     }
-    if (vpt <= 1) return launch_rows(dispatch_fp8_kernel<1>, threads, sm_cap, b.sm_count, p, st);
-    if (vpt <= 2) return launch_rows(dispatch_fp8_kernel<2>, threads, sm_cap, b.sm_count, p, st);
-    if (vpt <= 4) return launch_rows(dispatch_fp8_kernel<4>, threads, sm_cap, b.sm_count, p, st);
-    return launch_rows(dispatch_fp8_kernel<8>, threads, sm_cap, b.sm_count, p, st);
+    return launch_any(p, rv, (b.cfg.flags & EP_FLAG_FP8) != 0, sm_cap_of(b), b.sm_count, st);
 }
 
 }  // namespace ep

@@ -1,6 +1,7 @@
 // C ABI of libep (declared in include/ep.h): argument validation, worst-case
 // buffer sizing and partitioning, and the launches. Host code only. Every
-// device computation happens in layout.cu, dispatch.cu and combine.cu.
+// device computation happens in layout.cu, dispatch.cu, combine.cu, dedup.cu
+// and shard.cu.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdarg.h>
@@ -55,8 +56,10 @@ ep_status_t validate(const ep_config_t* c) {
         if (c->topk > c->topk_groups * gs) return fail(EP_ERR_INVALID, "topk exceeds the experts of the kept groups");
     }
     if (c->num_sms < 0) return fail(EP_ERR_INVALID, "num_sms must be >= 0");
-    if (c->flags & ~(EP_FLAG_FP8 | EP_FLAG_LOW_LATENCY | EP_FLAG_DEDUP))
+    if (c->flags & ~(EP_FLAG_FP8 | EP_FLAG_LOW_LATENCY | EP_FLAG_DEDUP | EP_FLAG_SHARD))
         return fail(EP_ERR_INVALID, "unknown flag bits");
+    if ((c->flags & EP_FLAG_SHARD) && (c->flags & (EP_FLAG_LOW_LATENCY | EP_FLAG_DEDUP)))
+        return fail(EP_ERR_UNSUPPORTED, "EP_FLAG_SHARD does not combine with EP_FLAG_LOW_LATENCY or EP_FLAG_DEDUP");
     const int64_t m_max = (int64_t)c->num_ranks * c->max_tokens_per_rank * c->topk;
     if (m_max >= (int64_t)1 << 31) return fail(EP_ERR_UNSUPPORTED, "R*T_max*K must be < 2^31 (int32 row ids)");
     if ((c->flags & EP_FLAG_LOW_LATENCY) &&
@@ -75,26 +78,32 @@ enum {
     R_TOPK_IDX, R_TOPK_W, R_ITR, R_NTPR, R_CNT, R_NTPE, R_EOFF, R_ROFF, R_SOFF, R_DST,
     R_SCRATCH, R_ERR, R_RECV_X, R_RECV_SCALE, R_RECV_SRC, R_RECV_W,
     R_TOK_ROW, R_RANK_ROW_OFF, R_RANK_SRC_OFF, R_DD_X, R_DD_SCALE, R_DD_SRC, R_DD_TOPK_IDX, R_DD_TOPK_W, R_PARTIAL,
+    R_CNT_ALL, R_DST_RANK, R_RECV_COUNT, R_RECV_OFF,
     R_COUNT
 };
 
 Plan plan_of(const ep_config_t* c, int64_t* n_max, int64_t* m_max, int64_t* nc_max) {
     const int64_t R = c->num_ranks, T = c->max_tokens_per_rank, H = c->hidden, E = c->num_experts,
                   K = c->topk;
-    const int64_t N = R * T;
-    const int64_t M = (c->flags & EP_FLAG_LOW_LATENCY) ? E * R * T : N * K;
+    // one rank per GPU: the buffer holds this rank's T_max tokens, one source
+    // row of counts, and receive rows for the worst case (every slot of every
+    // rank lands here)
+    const bool sh = (c->flags & EP_FLAG_SHARD) != 0;
+    const int64_t S = sh ? 1 : R;  // source ranks whose tokens the buffer routes
+    const int64_t N = S * T;
+    const int64_t M = (c->flags & EP_FLAG_LOW_LATENCY) ? E * R * T : R * T * K;
     const int64_t scratch = ep::layout_scratch_ints(*c, ep::kMaxLayoutCtas);
     const bool fp8 = (c->flags & EP_FLAG_FP8) != 0;
     size_t sz[R_COUNT];
     sz[R_TOPK_IDX] = 4 * N * K;
     sz[R_TOPK_W] = 4 * N * K;
     sz[R_ITR] = N * R;
-    sz[R_NTPR] = 4 * R * R;
-    sz[R_CNT] = 4 * R * E;
+    sz[R_NTPR] = 4 * S * R;
+    sz[R_CNT] = 4 * S * E;
     sz[R_NTPE] = 4 * E;
     sz[R_EOFF] = 4 * (E + 1);
     sz[R_ROFF] = 4 * (R + 1);
-    sz[R_SOFF] = 4 * E * R;
+    sz[R_SOFF] = 4 * E * S;
     sz[R_DST] = 4 * N * K;
     sz[R_SCRATCH] = 4 * scratch;
     sz[R_ERR] = 16;
@@ -113,6 +122,11 @@ Plan plan_of(const ep_config_t* c, int64_t* n_max, int64_t* m_max, int64_t* nc_m
     sz[R_DD_TOPK_IDX] = 4 * D * K;
     sz[R_DD_TOPK_W] = 4 * D * K;
     sz[R_PARTIAL] = (size_t)D * H * 2;
+    const int64_t L = E / R;
+    sz[R_CNT_ALL] = sh ? 4 * R * E : 0;
+    sz[R_DST_RANK] = sh ? N * K : 0;
+    sz[R_RECV_COUNT] = sh ? 4 * L : 0;
+    sz[R_RECV_OFF] = sh ? 4 * (L + 1) : 0;
     Plan p{};
     size_t cur = 0;
     for (int i = 0; i < R_COUNT; ++i) {
@@ -237,6 +251,13 @@ ep_status_t ep_buffer_create(const ep_config_t* cfg, void* d_workspace, size_t b
     b->dd_topk_idx = dd ? reinterpret_cast<int32_t*>(w + p.off[R_DD_TOPK_IDX]) : nullptr;
     b->dd_topk_w = dd ? reinterpret_cast<float*>(w + p.off[R_DD_TOPK_W]) : nullptr;
     b->partial = dd ? reinterpret_cast<uint16_t*>(w + p.off[R_PARTIAL]) : nullptr;
+    const bool sh = (cfg->flags & EP_FLAG_SHARD) != 0;
+    b->cnt_all = sh ? reinterpret_cast<int32_t*>(w + p.off[R_CNT_ALL]) : nullptr;
+    b->dst_rank = sh ? w + p.off[R_DST_RANK] : nullptr;
+    b->recv_count = sh ? reinterpret_cast<int32_t*>(w + p.off[R_RECV_COUNT]) : nullptr;
+    b->recv_off = sh ? reinterpret_cast<int32_t*>(w + p.off[R_RECV_OFF]) : nullptr;
+    b->shard_rank = -1;
+    b->placed = false;
     int prev = 0;
     cudaGetDevice(&prev);
     if (prev != dev) cudaSetDevice(dev);
@@ -293,9 +314,9 @@ ep_status_t ep_buffer_recv(const ep_buffer_t* b, void** recv_x, float** recv_sca
     return ok();
 }
 
-ep_status_t ep_get_layout(ep_buffer_t* b, int T, const float* d_logits, const int32_t* d_topk_idx,
-                          const float* d_topk_w, int route, uint64_t mask_seed, float mask_frac, void* stream) {
-    if (ep_status_t st = check_buf(b)) return st;
+static ep_status_t layout_args(const ep_buffer_t* b, int T, const float* d_logits, const int32_t* d_topk_idx,
+                               const float* d_topk_w, int route, uint64_t mask_seed, float mask_frac,
+                               ep::LayoutArgs* a) {
     if (T < 0) return fail(EP_ERR_INVALID, "T must be >= 0");
     if (T > b->cfg.max_tokens_per_rank)
         return fail(EP_ERR_CAPACITY, "T=%d exceeds max_tokens_per_rank=%d", T, b->cfg.max_tokens_per_rank);
@@ -309,16 +330,32 @@ ep_status_t ep_get_layout(ep_buffer_t* b, int T, const float* d_logits, const in
         b->cfg.topk > b->cfg.topk_groups * (b->cfg.num_experts / b->cfg.num_groups))
         return fail(EP_ERR_INVALID, "topk exceeds the experts of the kept groups");
     if (!(mask_frac >= 0.0f && mask_frac <= 1.0f)) return fail(EP_ERR_INVALID, "mask_frac must be in [0, 1]");
-    ep::LayoutArgs a{};
-    a.T = T;
-    a.logits = d_logits;
-    a.in_idx = d_topk_idx;
-    a.in_w = d_topk_w;
-    a.route = route;
-    a.mask_seed = mask_seed;
+    *a = ep::LayoutArgs{};
+    a->T = T;
+    a->logits = d_logits;
+    a->in_idx = d_topk_idx;
+    a->in_w = d_topk_w;
+    a->route = route;
+    a->mask_seed = mask_seed;
     double thr = floor((double)mask_frac * 4294967296.0);
-    a.mask_threshold = (uint64_t)thr;
-    a.m_max = b->m_max;
+    a->mask_threshold = (uint64_t)thr;
+    a->m_max = b->m_max;
+    return EP_OK;
+}
+
+static ep_status_t check_single(const ep_buffer_t* b) {
+    if (ep_status_t st = check_buf(b)) return st;
+    if (b->cfg.flags & EP_FLAG_SHARD)
+        return fail(EP_ERR_INVALID, "buffer was created with EP_FLAG_SHARD: use the ep_shard_* calls");
+    return EP_OK;
+}
+
+ep_status_t ep_get_layout(ep_buffer_t* b, int T, const float* d_logits, const int32_t* d_topk_idx,
+                          const float* d_topk_w, int route, uint64_t mask_seed, float mask_frac, void* stream) {
+    if (ep_status_t st = check_single(b)) return st;
+    ep::LayoutArgs a;
+    if (ep_status_t st = layout_args(b, T, d_logits, d_topk_idx, d_topk_w, route, mask_seed, mask_frac, &a))
+        return st;
     cudaError_t e = ep::launch_layout(*b, a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "layout launch");
     b->last_T = T;
@@ -326,7 +363,7 @@ ep_status_t ep_get_layout(ep_buffer_t* b, int T, const float* d_logits, const in
 }
 
 ep_status_t ep_dispatch(ep_buffer_t* b, int T, const void* d_x, void* stream) {
-    if (ep_status_t st = check_buf(b)) return st;
+    if (ep_status_t st = check_single(b)) return st;
     if (T != b->last_T) return fail(EP_ERR_INVALID, "T=%d does not match the last ep_get_layout (T=%d)", T, b->last_T);
     if (T > 0 && !d_x) return fail(EP_ERR_INVALID, "d_x is NULL");
     if ((uintptr_t)d_x % 32 != 0) return fail(EP_ERR_INVALID, "d_x must be 32-byte aligned");
@@ -336,7 +373,7 @@ ep_status_t ep_dispatch(ep_buffer_t* b, int T, const void* d_x, void* stream) {
 }
 
 ep_status_t ep_combine(ep_buffer_t* b, int T, const void* d_y, const float* d_y_scale, void* d_out, void* stream) {
-    if (ep_status_t st = check_buf(b)) return st;
+    if (ep_status_t st = check_single(b)) return st;
     if (T != b->last_T) return fail(EP_ERR_INVALID, "T=%d does not match the last ep_get_layout (T=%d)", T, b->last_T);
     if (T > 0 && (!d_y || !d_out)) return fail(EP_ERR_INVALID, "d_y and d_out must be non-NULL");
     if ((uintptr_t)d_y % 32 != 0 || (uintptr_t)d_out % 32 != 0)
@@ -404,6 +441,104 @@ ep_status_t ep_combine_dedup(ep_buffer_t* b, int T, void* d_out, void* stream) {
     if ((uintptr_t)d_out % 32 != 0) return fail(EP_ERR_INVALID, "d_out must be 32-byte aligned");
     cudaError_t e = ep::launch_combine_dedup(*b, T, d_out, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "combine_dedup launch");
+    return ok();
+}
+
+/* ---- one rank per GPU (EP_FLAG_SHARD) ------------------------------------ */
+
+static ep_status_t check_shard(const ep_buffer_t* b) {
+    if (ep_status_t st = check_buf(b)) return st;
+    if (!(b->cfg.flags & EP_FLAG_SHARD)) return fail(EP_ERR_INVALID, "buffer was created without EP_FLAG_SHARD");
+    return EP_OK;
+}
+
+static ep_status_t check_shard_step(const ep_buffer_t* b, int rank, int T, bool need_placed) {
+    if (ep_status_t st = check_shard(b)) return st;
+    if (b->shard_rank < 0) return fail(EP_ERR_INVALID, "no ep_shard_layout on this buffer yet");
+    if (rank != b->shard_rank)
+        return fail(EP_ERR_INVALID, "rank=%d does not match the last ep_shard_layout (rank=%d)", rank, b->shard_rank);
+    if (T != b->last_T) return fail(EP_ERR_INVALID, "T=%d does not match the last ep_shard_layout (T=%d)", T, b->last_T);
+    if (need_placed && !b->placed) return fail(EP_ERR_INVALID, "call ep_shard_place after ep_shard_layout first");
+    return EP_OK;
+}
+
+ep_status_t ep_buffer_shard(const ep_buffer_t* b, int32_t** cnt_row, int32_t** cnt_all, uint8_t** dst_rank,
+                            int32_t** recv_count, int32_t** recv_off) {
+    if (ep_status_t st = check_shard(b)) return st;
+    if (cnt_row) *cnt_row = b->cnt;
+    if (cnt_all) *cnt_all = b->cnt_all;
+    if (dst_rank) *dst_rank = b->dst_rank;
+    if (recv_count) *recv_count = b->recv_count;
+    if (recv_off) *recv_off = b->recv_off;
+    return ok();
+}
+
+ep_status_t ep_shard_layout(ep_buffer_t* b, int rank, int T, const float* d_logits, const int32_t* d_topk_idx,
+                            const float* d_topk_w, int route, uint64_t mask_seed, float mask_frac, void* stream) {
+    if (ep_status_t st = check_shard(b)) return st;
+    if (rank < 0 || rank >= b->cfg.num_ranks)
+        return fail(EP_ERR_INVALID, "rank=%d outside [0, %d)", rank, b->cfg.num_ranks);
+    ep::LayoutArgs a;
+    if (ep_status_t st = layout_args(b, T, d_logits, d_topk_idx, d_topk_w, route, mask_seed, mask_frac, &a))
+        return st;
+    a.S = 1;
+    a.g_base = (int64_t)rank * T;
+    cudaError_t e = ep::launch_layout(*b, a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "shard layout launch");
+    b->last_T = T;
+    b->shard_rank = rank;
+    b->placed = false;
+    return ok();
+}
+
+ep_status_t ep_shard_place(ep_buffer_t* b, int rank, int T, void* stream) {
+    if (ep_status_t st = check_shard_step(b, rank, T, false)) return st;
+    if (b->placed) return fail(EP_ERR_INVALID, "ep_shard_place already ran for this ep_shard_layout");
+    cudaError_t e = ep::launch_shard_place(*b, rank, T, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "shard place launch");
+    b->placed = true;
+    return ok();
+}
+
+ep_status_t ep_shard_dispatch(ep_buffer_t* b, int rank, int T, const void* d_x, void* const* peer_recv_x,
+                              float* const* peer_recv_scale, int32_t* const* peer_recv_src,
+                              float* const* peer_recv_w, void* stream) {
+    if (ep_status_t st = check_shard_step(b, rank, T, true)) return st;
+    if (T > 0 && !d_x) return fail(EP_ERR_INVALID, "d_x is NULL");
+    if ((uintptr_t)d_x % 32 != 0) return fail(EP_ERR_INVALID, "d_x must be 32-byte aligned");
+    if (!peer_recv_x || !peer_recv_src || !peer_recv_w)
+        return fail(EP_ERR_INVALID, "peer_recv_x, peer_recv_src and peer_recv_w must be non-NULL");
+    const bool fp8 = (b->cfg.flags & EP_FLAG_FP8) != 0;
+    if (fp8 && !peer_recv_scale) return fail(EP_ERR_INVALID, "EP_FLAG_FP8 needs peer_recv_scale");
+    for (int d = 0; d < b->cfg.num_ranks; ++d) {
+        if (!peer_recv_x[d] || !peer_recv_src[d] || !peer_recv_w[d] || (fp8 && !peer_recv_scale[d]))
+            return fail(EP_ERR_INVALID, "peer table entry %d is NULL", d);
+        if ((uintptr_t)peer_recv_x[d] % 32 != 0) return fail(EP_ERR_INVALID, "peer_recv_x[%d] must be 32-byte aligned", d);
+        if ((uintptr_t)peer_recv_src[d] % 4 != 0 || (uintptr_t)peer_recv_w[d] % 4 != 0 ||
+            (fp8 && (uintptr_t)peer_recv_scale[d] % 4 != 0))
+            return fail(EP_ERR_INVALID, "peer table entry %d must be 4-byte aligned", d);
+    }
+    cudaError_t e = ep::launch_shard_dispatch(*b, rank, T, d_x, peer_recv_x, fp8 ? peer_recv_scale : nullptr,
+                                              peer_recv_src, peer_recv_w, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "shard dispatch launch");
+    return ok();
+}
+
+ep_status_t ep_shard_combine(ep_buffer_t* b, int rank, int T, const void* const* peer_y,
+                             const float* const* peer_y_scale, void* d_out, void* stream) {
+    if (ep_status_t st = check_shard_step(b, rank, T, true)) return st;
+    if (T > 0 && !d_out) return fail(EP_ERR_INVALID, "d_out is NULL");
+    if ((uintptr_t)d_out % 32 != 0) return fail(EP_ERR_INVALID, "d_out must be 32-byte aligned");
+    if (!peer_y) return fail(EP_ERR_INVALID, "peer_y is NULL");
+    for (int d = 0; d < b->cfg.num_ranks; ++d) {
+        if (!peer_y[d] || (peer_y_scale && !peer_y_scale[d]))
+            return fail(EP_ERR_INVALID, "peer table entry %d is NULL", d);
+        if ((uintptr_t)peer_y[d] % 32 != 0) return fail(EP_ERR_INVALID, "peer_y[%d] must be 32-byte aligned", d);
+        if (peer_y_scale && (uintptr_t)peer_y_scale[d] % 4 != 0)
+            return fail(EP_ERR_INVALID, "peer_y_scale[%d] must be 4-byte aligned", d);
+    }
+    cudaError_t e = ep::launch_shard_combine(*b, T, peer_y, peer_y_scale, d_out, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "shard combine launch");
     return ok();
 }
 

@@ -39,6 +39,13 @@ struct ep_buffer {
     int32_t* dd_topk_idx;   // [d_max, K]
     float* dd_topk_w;       // [d_max, K]
     uint16_t* partial;      // [d_max, H] bf16
+    // one rank per GPU (EP_FLAG_SHARD; device unless stated)
+    int32_t* cnt_all;     // [R, E]: every rank's count row, filled by the caller's all-gather
+    uint8_t* dst_rank;    // [T_max, K]: destination rank of each slot
+    int32_t* recv_count;  // [E/R]: receive rows of each of this rank's experts
+    int32_t* recv_off;    // [E/R + 1]: their exclusive prefix; recv_off[E/R] = rows received
+    int shard_rank;       // host: rank of the last ep_shard_layout (-1 = none)
+    bool placed;          // host: ep_shard_place ran after the last ep_shard_layout
     uint32_t* err;  // device error word
     // receive buffers (device)
     void* recv_x;
@@ -55,6 +62,8 @@ void set_last_error(const char* msg);
 // Layout grid cap (CTAs = chunks) and the control words at the head of the
 // layout scratch (two barrier counters, zero between launches).
 constexpr int kMaxLayoutCtas = 1024;
+// Ranks a peer-pointer table holds (the num_ranks limit).
+constexpr int kMaxPeers = 32;
 constexpr int kLayoutControlInts = 64;
 
 struct LayoutArgs {
@@ -68,6 +77,8 @@ struct LayoutArgs {
     int64_t m_max;            // rows the receive side holds (bound check)
     int low_latency;          // fixed (expert, source rank) regions of T_max rows
     int T_max;                // region size in low-latency mode
+    int S = 0;                        // source ranks routed (0 = all R); 1 = one rank's own tokens
+    int64_t g_base = 0;               // global id of the first token (slot-mask hash)
     int32_t* tok_row = nullptr;       // dedup outputs (NULL: not wanted)
     int32_t* rank_row_off = nullptr;
     int32_t* rank_src_off = nullptr;
@@ -95,5 +106,15 @@ cudaError_t launch_local_reduce(const ep_buffer& b, int T, const void* y, const 
 cudaError_t launch_combine_dedup(const ep_buffer& b, int T, void* out, cudaStream_t stream);
 cudaError_t launch_combine(const ep_buffer& b, int T, const void* y, const float* y_scale, void* out,
                            cudaStream_t stream);
+
+// One rank per GPU (EP_FLAG_SHARD): placement from the gathered count rows,
+// then dispatch into / combine from every rank's arrays through tables of
+// num_ranks device pointers.
+cudaError_t launch_shard_place(const ep_buffer& b, int rank, int T, cudaStream_t stream);
+cudaError_t launch_shard_dispatch(const ep_buffer& b, int rank, int T, const void* x, void* const* peer_x,
+                                  float* const* peer_scale, int32_t* const* peer_src, float* const* peer_w,
+                                  cudaStream_t stream);
+cudaError_t launch_shard_combine(const ep_buffer& b, int T, const void* const* peer_y,
+                                 const float* const* peer_scale, void* out, cudaStream_t stream);
 
 }  // namespace ep

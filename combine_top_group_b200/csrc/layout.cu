@@ -45,6 +45,8 @@ constexpr int kThreads = kWarps * 32;
 
 struct LayoutParams {
     int R, T, E, K, L, G, KG, J;  // J = E + R histogram columns
+    int S;                        // source ranks whose tokens this launch routes: R, or 1 (one rank's own)
+    int64_t g_base;               // global id of local token 0 (the slot mask hashes global ids)
     uint32_t l_magic;             // e / L == __umulhi(e, l_magic) for 0 <= e < 2^16
     int nb;                       // CTAs (one resident wave)
     int ncpr, nc;                 // chunks per rank, chunks (nc <= nb)
@@ -322,56 +324,12 @@ __device__ __forceinline__ void route_token(const LayoutParams& p, int64_t g, in
     }
     // slot mask
     if (lane < p.K && p.mask_thr != 0ull) {
-        const uint64_t h = splitmix64(p.mask_seed ^ (uint64_t)(g * p.K + lane));
+        const uint64_t h = splitmix64(p.mask_seed ^ (uint64_t)((p.g_base + g) * p.K + lane));
         if ((h >> 32) < p.mask_thr) {
             my_e = -1;
             my_w = 0.0f;
         }
     }
-}
-
-// Exclusive scan of n <= 4 * blockDim.x values in[j * stride] into out[0..n],
-// with out[n] = total. Called by every thread of the block.
-__device__ void block_exclusive_scan(const int32_t* in, int stride, int n, int* out, int* warp_tot) {
-    const int t = threadIdx.x;
-    const int lane = t & 31, warp = t >> 5, nw = blockDim.x >> 5;
-    int v[4];
-    int local = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int j = 4 * t + i;
-        v[i] = (j < n) ? in[(int64_t)j * stride] : 0;
-        local += v[i];
-    }
-    int incl = local;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int o = __shfl_up_sync(FULL, incl, off);
-        if (lane >= off) incl += o;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        const int wv = (lane < nw) ? warp_tot[lane] : 0;
-        int wi = wv;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int o = __shfl_up_sync(FULL, wi, off);
-            if (lane >= off) wi += o;
-        }
-        if (lane < nw) warp_tot[lane] = wi - wv;
-        if (lane == nw - 1) warp_tot[32] = wi;
-    }
-    __syncthreads();
-    int run = warp_tot[warp] + incl - local;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int j = 4 * t + i;
-        if (j < n) out[j] = run;
-        run += v[i];
-    }
-    if (t == 0) out[n] = warp_tot[32];
-    __syncthreads();
 }
 
 template <int EPL>
@@ -442,16 +400,16 @@ __global__ void __launch_bounds__(kThreads, 2) layout_kernel(LayoutParams p) {
         block_exclusive_scan(colp, 1, p.nc, eoff, warp_tot);  // eoff: scratch here, [nc + 1]
         for (int cc = threadIdx.x; cc < p.nc; cc += kThreads) colp[cc] = eoff[cc];
         // prefix at each rank's first chunk; eoff[nc] is the column total
-        if (threadIdx.x < p.R) {
-            const int r = threadIdx.x;
+        if (threadIdx.x < p.S) {
+            const int r = threadIdx.x;  // source rank
             const int a = (p.nc > 0) ? eoff[r * p.ncpr] : 0;
-            const int b = (p.nc > 0) ? eoff[(r + 1) * p.ncpr] : 0;  // (R * ncpr = nc) -> total
+            const int b = (p.nc > 0) ? eoff[(r + 1) * p.ncpr] : 0;  // (S * ncpr = nc) -> total
             if (col < p.E) {
-                p.src_off[(int64_t)col * p.R + r] = a;
+                p.src_off[(int64_t)col * p.S + r] = a;
                 p.cnt[(int64_t)r * p.E + col] = b - a;
             } else {
                 p.ntpr[(int64_t)r * p.R + (col - p.E)] = b - a;
-                if (p.dedup) p.rank_src_off[(int64_t)(col - p.E) * p.R + r] = a;
+                if (p.dedup) p.rank_src_off[(int64_t)(col - p.E) * p.S + r] = a;
             }
         }
         if (threadIdx.x == 0) {
@@ -618,14 +576,14 @@ cudaError_t launch_epl(LayoutParams& p, int dev, int sm_count, int max_ctas, cud
     int nb = per_sm * sm_count;
     if (nb > max_ctas) nb = max_ctas;
     // small batches: about one token per warp, so the grid barriers stay cheap
-    const int64_t want = ((int64_t)p.R * p.T + kWarps - 1) / kWarps;
-    if (want < nb) nb = (int)(want > p.R ? want : p.R);
-    if (nb < p.R) return cudaErrorInvalidConfiguration;  // every rank needs a chunk
+    const int64_t want = ((int64_t)p.S * p.T + kWarps - 1) / kWarps;
+    if (want < nb) nb = (int)(want > p.S ? want : p.S);
+    if (nb < p.S) return cudaErrorInvalidConfiguration;  // every source rank needs a chunk
     p.nb = nb;
-    int ncpr = nb / p.R;
+    int ncpr = nb / p.S;
     if (ncpr > p.T) ncpr = p.T;
     p.ncpr = ncpr > 0 ? ncpr : 1;
-    p.nc = (p.T > 0) ? p.R * ncpr : 0;
+    p.nc = (p.T > 0) ? p.S * ncpr : 0;
     void* args[] = {&p};
     e = cudaLaunchCooperativeKernel((const void*)kern, dim3(nb), dim3(kThreads), args, smem, st);
     if (e != cudaSuccess) return e;
@@ -656,6 +614,8 @@ cudaError_t launch_layout_raw(const ep_config_t& c, const LayoutArgs& a, const e
     p.G = c.num_groups;
     p.KG = c.topk_groups;
     p.J = p.E + p.R;
+    p.S = a.S > 0 ? a.S : p.R;
+    p.g_base = a.g_base;
     p.route = a.route;
     p.logits = a.logits;
     p.vec_logits = (a.logits != nullptr && (p.E % 4 == 0) && ((uintptr_t)a.logits % 16 == 0)) ? 1 : 0;

@@ -28,6 +28,7 @@ EP_DEVERR_EXPERT_ID, EP_DEVERR_ROW_BOUNDS, EP_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 EP_FLAG_FP8 = 0x1
 EP_FLAG_LOW_LATENCY = 0x2
 EP_FLAG_DEDUP = 0x4
+EP_FLAG_SHARD = 0x8
 EP_ROUTE_SOFTMAX, EP_ROUTE_SOFTMAX_RENORM, EP_ROUTE_GROUP_SIGMOID = 0, 1, 2
 
 
@@ -88,13 +89,25 @@ _lib.ep_combine_dedup.argtypes = [_P, ctypes.c_int, _P, _P]
 _lib.ep_combine_dedup.restype = _st
 _lib.ep_selftest_wait_timeout.argtypes = [_P, ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint32), _P]
 _lib.ep_selftest_wait_timeout.restype = _st
+_lib.ep_buffer_shard.argtypes = [_P] + [ctypes.POINTER(_P)] * 5
+_lib.ep_buffer_shard.restype = _st
+_lib.ep_shard_layout.argtypes = [_P, ctypes.c_int, ctypes.c_int, _P, _P, _P, ctypes.c_int, ctypes.c_uint64,
+                                 ctypes.c_float, _P]
+_lib.ep_shard_layout.restype = _st
+_lib.ep_shard_place.argtypes = [_P, ctypes.c_int, ctypes.c_int, _P]
+_lib.ep_shard_place.restype = _st
+_lib.ep_shard_dispatch.argtypes = [_P, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _P, _P]
+_lib.ep_shard_dispatch.restype = _st
+_lib.ep_shard_combine.argtypes = [_P, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P]
+_lib.ep_shard_combine.restype = _st
 
 EXPORTED = ("ep_abi_version", "ep_status_string", "ep_last_error_message", "ep_default_config",
             "ep_buffer_workspace_bytes", "ep_buffer_create", "ep_buffer_destroy", "ep_buffer_set_num_sms",
             "ep_buffer_layout",
             "ep_buffer_recv", "ep_get_layout", "ep_dispatch", "ep_combine", "ep_check_errors",
             "ep_get_layout_noalloc", "ep_selftest_wait_timeout", "ep_buffer_dedup", "ep_dispatch_dedup",
-            "ep_permute", "ep_local_reduce", "ep_combine_dedup")
+            "ep_permute", "ep_local_reduce", "ep_combine_dedup", "ep_buffer_shard", "ep_shard_layout",
+            "ep_shard_place", "ep_shard_dispatch", "ep_shard_combine")
 
 
 class EpError(RuntimeError):
@@ -136,6 +149,10 @@ class EpBuffer:
     @property
     def fp8(self) -> bool:
         return bool(self.cfg.flags & EP_FLAG_FP8)
+
+    @property
+    def shard(self) -> bool:
+        return bool(self.cfg.flags & EP_FLAG_SHARD)
 
     def _view(self, ptr: int, dtype: torch.dtype, shape) -> torch.Tensor:
         off = ptr - self.workspace.data_ptr()
@@ -200,21 +217,24 @@ def ep_buffer_set_num_sms(buf: EpBuffer, num_sms: int) -> None:
 
 
 def ep_buffer_layout(buf: EpBuffer, T: int) -> dict:
-    """torch views of the layout arrays for T tokens per rank."""
+    """torch views of the layout arrays for T tokens per rank (one source rank,
+    N = T, for an EP_FLAG_SHARD buffer)."""
     lay = EpLayout()
     _check(_lib.ep_buffer_layout(buf.handle, ctypes.byref(lay)), "ep_buffer_layout")
     c = buf.cfg
-    R, E, K, N = c.num_ranks, c.num_experts, c.topk, c.num_ranks * T
+    R, E, K = c.num_ranks, c.num_experts, c.topk
+    S = 1 if buf.shard else R
+    N = S * T
     return dict(
         topk_idx=buf._view(lay.topk_idx, torch.int32, (N, K)),
         topk_w=buf._view(lay.topk_w, torch.float32, (N, K)),
         is_token_in_rank=buf._view(lay.is_token_in_rank, torch.uint8, (N, R)),
-        num_tokens_per_rank=buf._view(lay.num_tokens_per_rank, torch.int32, (R, R)),
-        cnt=buf._view(lay.cnt_src_expert, torch.int32, (R, E)),
+        num_tokens_per_rank=buf._view(lay.num_tokens_per_rank, torch.int32, (S, R)),
+        cnt=buf._view(lay.cnt_src_expert, torch.int32, (S, E)),
         num_tokens_per_expert=buf._view(lay.num_tokens_per_expert, torch.int32, (E,)),
         expert_off=buf._view(lay.expert_off, torch.int32, (E + 1,)),
         rank_off=buf._view(lay.rank_off, torch.int32, (R + 1,)),
-        src_off=buf._view(lay.src_off, torch.int32, (E, R)),
+        src_off=buf._view(lay.src_off, torch.int32, (E, S)),
         dst_row=buf._view(lay.dst_row, torch.int32, (N, K)),
     )
 
@@ -327,3 +347,56 @@ def ep_get_layout_noalloc(cfg: EpConfig, T: int, out: dict, error_word, logits=N
     _check(_lib.ep_get_layout_noalloc(ctypes.byref(cfg), T, _ptr(logits), _ptr(topk_idx), _ptr(topk_w), route,
                                       mask_seed & 0xFFFF_FFFF_FFFF_FFFF, mask_frac, ctypes.byref(lay),
                                       _ptr(error_word), _stream(stream)), "ep_get_layout_noalloc")
+
+
+# ---- one rank per GPU (EP_FLAG_SHARD) ------------------------------------------
+
+def _table(entries):
+    """Host array of device pointers (tensors or ints; None stays NULL)."""
+    if entries is None:
+        return None
+    arr = (_P * len(entries))(*[_ptr(t) for t in entries])
+    return arr
+
+
+def ep_buffer_shard(buf: EpBuffer, T: int) -> dict:
+    """torch views of the shard arrays: cnt_row [E], cnt_all [R, E],
+    dst_rank [T, K], recv_count [E/R], recv_off [E/R + 1]."""
+    ptrs = [_P() for _ in range(5)]
+    _check(_lib.ep_buffer_shard(buf.handle, *[ctypes.byref(p) for p in ptrs]), "ep_buffer_shard")
+    c = buf.cfg
+    R, E, K = c.num_ranks, c.num_experts, c.topk
+    L = E // R
+    return dict(cnt_row=buf._view(ptrs[0].value, torch.int32, (E,)),
+                cnt_all=buf._view(ptrs[1].value, torch.int32, (R, E)),
+                dst_rank=buf._view(ptrs[2].value, torch.uint8, (T, K)),
+                recv_count=buf._view(ptrs[3].value, torch.int32, (L,)),
+                recv_off=buf._view(ptrs[4].value, torch.int32, (L + 1,)))
+
+
+def ep_shard_layout(buf: EpBuffer, rank: int, T: int, logits=None, topk_idx=None, topk_w=None, route: int = 0,
+                    mask_seed: int = 0, mask_frac: float = 0.0, stream=None) -> None:
+    _check(_lib.ep_shard_layout(buf.handle, rank, T, _ptr(logits), _ptr(topk_idx), _ptr(topk_w), route,
+                                mask_seed & 0xFFFF_FFFF_FFFF_FFFF, mask_frac, _stream(stream)), "ep_shard_layout")
+
+
+def ep_shard_place(buf: EpBuffer, rank: int, T: int, stream=None) -> None:
+    _check(_lib.ep_shard_place(buf.handle, rank, T, _stream(stream)), "ep_shard_place")
+
+
+def ep_shard_dispatch(buf: EpBuffer, rank: int, T: int, x, peer_recv_x, peer_recv_scale, peer_recv_src,
+                      peer_recv_w, stream=None) -> None:
+    """peer_* are length-R lists of each rank's receive arrays (tensors or
+    device pointers); peer_recv_scale is None without FP8."""
+    tx, ts, tr, tw = (_table(peer_recv_x), _table(peer_recv_scale), _table(peer_recv_src),
+                      _table(peer_recv_w))
+    _check(_lib.ep_shard_dispatch(buf.handle, rank, T, _ptr(x), tx, ts, tr, tw, _stream(stream)),
+           "ep_shard_dispatch")
+
+
+def ep_shard_combine(buf: EpBuffer, rank: int, T: int, peer_y, peer_y_scale, out, stream=None) -> None:
+    """peer_y: length-R list of each rank's expert output (bf16, or e4m3 with
+    peer_y_scale for the fused dequantisation)."""
+    ty, ts = _table(peer_y), _table(peer_y_scale)
+    _check(_lib.ep_shard_combine(buf.handle, rank, T, ty, ts, _ptr(out), _stream(stream)), "ep_shard_combine")
+

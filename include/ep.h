@@ -40,7 +40,7 @@
 extern "C" {
 #endif
 
-#define EP_ABI_VERSION 1
+#define EP_ABI_VERSION 2
 
 typedef enum {
     EP_OK = 0,
@@ -76,6 +76,10 @@ typedef enum {
  * dedup layout (ep_buffer_dedup), and ep_dispatch_dedup, ep_permute,
  * ep_local_reduce and ep_combine_dedup become available. */
 #define EP_FLAG_DEDUP 0x4u
+/* One rank per GPU: the buffer belongs to ONE rank of R and holds its own
+ * T_max tokens' layout and its own receive rows (the ep_shard_* calls below).
+ * Not combinable with EP_FLAG_LOW_LATENCY or EP_FLAG_DEDUP. */
+#define EP_FLAG_SHARD 0x8u
 
 /* Routing rule applied by ep_get_layout to router logits. */
 typedef enum {
@@ -261,6 +265,106 @@ ep_status_t ep_local_reduce(ep_buffer_t *buf, int T, const void *d_y, const floa
  * partial[tok_row[g][r]] ); +0 for a token sent nowhere. d_out bf16 [N, H],
  * 32-byte aligned. */
 ep_status_t ep_combine_dedup(ep_buffer_t *buf, int T, void *d_out, void *stream);
+
+/* ---- one rank per GPU (EP_FLAG_SHARD) -------------------------------------
+ * The method as a node runs it: one process per GPU, each rank holding its own
+ * T tokens and the receive rows of its own E/R experts. Dispatch and combine
+ * then cross NVLink inside the node. The counts are exchanged first, and each
+ * rank writes its tokens straight into the receivers' buffers (DeepEP overlap
+ * notes, §节点内通信).
+ *
+ * A rank's buffer, created with EP_FLAG_SHARD and the same config on every
+ * rank, holds:
+ *  - the layout of the rank's own tokens, as ep_buffer_layout views with
+ *    N = T (one source rank):
+ *    - topk_idx, topk_w and dst_row [T, K], is_token_in_rank [T, R];
+ *    - num_tokens_per_rank [1, R] and cnt_src_expert [1, E]: this rank's row;
+ *  - cnt_all [R, E], dst_rank [T_max, K] and the receive counts
+ *    (ep_buffer_shard);
+ *  - receive rows for the worst case: M_max = R*T_max*K, every slot of every
+ *    rank on this rank (ep_buffer_recv).
+ *
+ * One step, on every rank s. Token g = s*T + t, with T the same on every rank:
+ *  1. ep_shard_layout: routing and the rank-local layout of s's T tokens. It
+ *     fills s's count row cnt[s][e].
+ *  2. The caller all-gathers the R count rows into every rank's cnt_all, for
+ *     example with an NCCL all-gather of R*E int32.
+ *  3. ep_shard_place: the row of each of s's slots on its destination rank
+ *     d = e / (E/R), and s's own receive counts.
+ *  4. The caller's barrier: every rank has finished reading its receive rows
+ *     from the step before.
+ *  5. ep_shard_dispatch: s's rows are stored into the destination ranks'
+ *     receive arrays, through tables of their device pointers. These are
+ *     peer-mapped pointers when the rank is another GPU.
+ *  6. The caller's barrier. Then expert work runs on each rank's own rows
+ *     [0, recv_off[E/R]).
+ *  7. ep_shard_combine: s's tokens are gathered from the ranks' expert
+ *     outputs, through pointer tables.
+ * There is no wait inside a kernel. The caller orders the ranks with
+ * collectives or barriers between the calls.
+ *
+ * Rank d's receive rows are rows [rank_off[d], rank_off[d+1]) of the
+ * single-buffer layout (ep_get_layout over all R*T tokens), shifted to start
+ * at 0: the same rows in the same order, (expert, source rank, token, slot).
+ * recv_src holds global token ids. dst_rank and dst_row index the
+ * destination's arrays. */
+
+/* Device views of the shard arrays:
+ *  cnt_row     int32 [E]: this rank's slots per expert (from ep_shard_layout),
+ *              the row to all-gather;
+ *  cnt_all     int32 [R, E]: the gathered rows; row s = rank s's cnt_row;
+ *  dst_rank    uint8 [T_max, K]: destination rank of each slot (after ep_shard_place);
+ *  recv_count  int32 [E/R]: rows this rank receives for each local expert;
+ *  recv_off    int32 [E/R + 1]: their exclusive prefix; recv_off[E/R] is
+ *              this rank's receive row count.
+ * Any out-pointer may be NULL. EP_ERR_INVALID without EP_FLAG_SHARD. */
+ep_status_t ep_buffer_shard(const ep_buffer_t *buf, int32_t **cnt_row, int32_t **cnt_all, uint8_t **dst_rank,
+                            int32_t **recv_count, int32_t **recv_off);
+
+/* Step 1: routing and the rank-local layout of rank `rank`'s T tokens. The
+ * inputs are as for ep_get_layout, but over [T, E] logits or [T, K] top-k.
+ * The slot mask hashes global ids (g = rank*T + t). Afterwards dst_row holds
+ * rank-local rows: this rank's exclusive expert offset plus the slot's
+ * position among the rank's earlier slots of that expert.
+ * Errors: as ep_get_layout, and EP_ERR_INVALID for a rank outside [0, R). */
+ep_status_t ep_shard_layout(ep_buffer_t *buf, int rank, int T, const float *d_logits,
+                            const int32_t *d_topk_idx, const float *d_topk_w, int route,
+                            uint64_t mask_seed, float mask_frac, void *stream);
+
+/* Step 3: reads cnt_all (the caller has filled it by step 2 on the same
+ * stream) and turns every slot's dst_row into its row on the destination
+ * rank, with that rank in dst_rank. Also writes this rank's recv_count and
+ * recv_off. Once per ep_shard_layout. rank and T must be those of the last
+ * ep_shard_layout. A row outside [0, M_max) sets EP_DEVERR_ROW_BOUNDS and
+ * becomes -1. */
+ep_status_t ep_shard_place(ep_buffer_t *buf, int rank, int T, void *stream);
+
+/* Step 5: for every unmasked slot (t,k) of this rank, destination d =
+ * dst_rank[t,k] and row r = dst_row[t,k]:
+ *  - peer_recv_x[d][r] = x[t], bf16 or cast to FP8 as in ep_dispatch;
+ *  - peer_recv_scale[d][r] = the FP8 scales;
+ *  - peer_recv_src[d][r] = rank*T + t;
+ *  - peer_recv_w[d][r] = topk_w[t,k].
+ * The peer_* arguments are HOST arrays of R device pointers: entry d is rank
+ * d's receive array (ep_buffer_recv on rank d). Pointers into other GPUs must
+ * be usable from this GPU: peer access enabled, or IPC or symmetric-memory
+ * mappings. Every entry is non-NULL. peer_recv_x entries are 32-byte aligned;
+ * peer_recv_scale may be NULL without EP_FLAG_FP8. d_x: bf16 [T, H], 32-byte
+ * aligned. Needs ep_shard_place first. Errors: EP_ERR_INVALID. */
+ep_status_t ep_shard_dispatch(ep_buffer_t *buf, int rank, int T, const void *d_x,
+                              void *const *peer_recv_x, float *const *peer_recv_scale,
+                              int32_t *const *peer_recv_src, float *const *peer_recv_w, void *stream);
+
+/* Step 7: out[t] = bf16_rne( sum over k ascending, unmasked, of
+ * w[t,k] * y_d[dst_row[t,k]] ), with d = dst_rank[t,k]. The sum is fp32 with
+ * one fused multiply-add per slot, as ep_combine computes it. peer_y is a
+ * HOST array of R device pointers to each rank's expert output: bf16
+ * [rows, H], or e4m3 [rows, H] with peer_y_scale (a host array of R fp32
+ * [rows, H/128] pointers) for the fused dequantisation. NULL peer_y_scale
+ * means bf16. d_out: bf16 [T, H]. peer_y entries and d_out are 32-byte
+ * aligned. Needs ep_shard_place first. Errors: EP_ERR_INVALID. */
+ep_status_t ep_shard_combine(ep_buffer_t *buf, int rank, int T, const void *const *peer_y,
+                             const float *const *peer_y_scale, void *d_out, void *stream);
 
 /* Diagnostic: proves that the library's bounded waits end. Runs the layout's
  * grid barrier on 2 CTAs with a target that can never be reached, and a limit

@@ -58,7 +58,7 @@ def test_binding_names_match_header():
 def test_host_only_entry_points():
     from combine_top_group_b200 import ep
     from combine_top_group_b200 import workloads as wl
-    assert ep.ep_abi_version() == 1
+    assert ep.ep_abi_version() == 2
     assert ep.ep_status_string(ep.EP_ERR_CAPACITY) == "EP_ERR_CAPACITY"
     cfg = ep.ep_default_config(8, 4096, 7168, 256, 8)
     assert (cfg.num_groups, cfg.topk_groups, cfg.num_sms, cfg.flags) == (1, 1, 0, 0)
@@ -81,7 +81,8 @@ def test_host_only_entry_points():
 @pytest.mark.parametrize("field,value,status", [
     ("num_ranks", 0, 5), ("num_ranks", 33, 5), ("hidden", 100, 5), ("num_experts", 2000, 5),
     ("num_experts", 30, 1), ("topk", 0, 1), ("topk", 33, 1), ("num_groups", 3, 1),
-    ("topk_groups", 9, 1), ("num_sms", -1, 1), ("flags", 8, 1), ("max_tokens_per_rank", 0, 1),
+    ("topk_groups", 9, 1), ("num_sms", -1, 1), ("flags", 16, 1), ("flags", 8 | 2, 5), ("flags", 8 | 4, 5),
+    ("max_tokens_per_rank", 0, 1),
 ])
 def test_config_validation(field, value, status):
     from combine_top_group_b200 import ep
@@ -100,3 +101,19 @@ def test_capacity_limit_int32_rows():
     with pytest.raises(ep.EpError) as ei:
         ep.ep_buffer_workspace_bytes(cfg)
     assert ei.value.status == ep.EP_ERR_UNSUPPORTED
+
+
+def test_shard_workspace_sizing():
+    """EP_FLAG_SHARD: the layout arrays cover one rank's T_max tokens, the
+    receive rows still cover the worst case (every slot of every rank)."""
+    from combine_top_group_b200 import ep
+    one = ep.ep_default_config(8, 4096, 7168, 256, 8)
+    full = ep.ep_buffer_workspace_bytes(one)
+    one.flags = ep.EP_FLAG_SHARD
+    sh = ep.ep_buffer_workspace_bytes(one)
+    M = 8 * 4096 * 8
+    assert sh >= M * 7168 * 2 + M * 8  # receive rows + recv_src + recv_w
+    # the single-buffer layout arrays for all 8 ranks (topk_idx, topk_w, dst_row,
+    # is_token_in_rank) shrink to one rank's, plus cnt_all and dst_rank
+    per_token = 8 * 12 + 8
+    assert full - sh >= 7 * 4096 * per_token - 8 * 256 * 4 - 4096 * 8 - 4096

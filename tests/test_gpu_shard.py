@@ -1,0 +1,168 @@
+"""One rank per GPU (EP_FLAG_SHARD): R ranks emulated on one device, each
+with its own buffer, checked against the oracle's single-buffer results.
+
+By definition of the split, rank d's receive rows are rows
+[rank_off[d], rank_off[d+1]) of the oracle's layout, shifted to start at 0;
+dst_rank = idx / L; a slot's row on its destination is its oracle row minus
+rank_off[dst_rank]; and each rank's combine output is the oracle's output for
+its tokens. Tolerances are those of the single-buffer parity tests.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from combine_top_group_b200 import workloads as wl
+from test_gpu_parity import _check_combine, _check_routing, _combine_expected, _oracle_route, _sample_rows, _to_host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from combine_top_group_b200 import ep, shard  # loads libep.so; fails loudly if missing
+    return ep, shard
+
+
+CASES = [("tiny", 0), ("tiny", 2), ("decode", 1), ("prefill", 0), ("skewed", 2)]
+
+
+@pytest.mark.parametrize("name,seed", CASES, ids=[f"{n}-s{s}" for n, s in CASES])
+def test_shard_parity(cuda, name, seed):
+    ep, shard = cuda
+    w = wl.WORKLOADS[name]
+    R, T, E, K, L, H = w.R, w.T, w.E, w.K, w.L, w.H
+    x = wl.make_x(w, seed)
+    logits = wl.make_logits(w, seed)
+    xt = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    lt = torch.from_numpy(np.ascontiguousarray(logits)).cuda()
+    out = torch.empty(w.N, H, dtype=torch.bfloat16, device="cuda")
+    em = shard.EmulatedRanks(w, xt, lt, out)
+
+    # ---- step 1: each rank's routing and rank-local counts
+    o_idx, o_w, margin = _oracle_route(w, logits)
+    em.layout()
+    assert em.check_errors() == 0
+    g_idx = np.concatenate([_to_host(ep.ep_buffer_layout(b, T)["topk_idx"]) for b in em.bufs])
+    g_w = np.concatenate([_to_host(ep.ep_buffer_layout(b, T)["topk_w"]) for b in em.bufs])
+    if _check_routing(w, o_idx, o_w, margin, g_idx, g_w):
+        em.layout(topk_idx=torch.from_numpy(o_idx).cuda(), topk_w=torch.from_numpy(o_w).cuda())
+    o_lay = oracle.layout(o_idx, R, T, E)
+    for s, b in enumerate(em.bufs):
+        lay = {k: _to_host(v) for k, v in ep.ep_buffer_layout(b, T).items()}
+        assert np.array_equal(lay["is_token_in_rank"], o_lay["is_token_in_rank"][s * T:(s + 1) * T])
+        assert np.array_equal(lay["num_tokens_per_rank"][0], o_lay["num_tokens_per_rank"][s])
+        assert np.array_equal(_to_host(em.sh[s]["cnt_row"]), o_lay["cnt"][s])
+
+    # ---- steps 2-3: exchange, placement on the destination ranks
+    em.exchange()
+    em.place()
+    assert em.check_errors() == 0
+    o_dst, o_eoff, o_roff = o_lay["dst_row"], o_lay["expert_off"], o_lay["rank_off"]
+    for s in range(R):
+        rows = slice(s * T, (s + 1) * T)
+        idx = o_idx[rows]
+        valid = idx >= 0
+        want_rank = np.where(valid, idx // L, 0)
+        want_row = np.where(valid, o_dst[rows] - o_roff[want_rank], -1)
+        assert np.array_equal(_to_host(em.sh[s]["dst_rank"]), want_rank.astype(np.uint8))
+        assert np.array_equal(_to_host(ep.ep_buffer_layout(em.bufs[s], T)["dst_row"]), want_row)
+        assert np.array_equal(_to_host(em.sh[s]["recv_count"]), o_lay["num_tokens_per_expert"][s * L:(s + 1) * L])
+        assert np.array_equal(_to_host(em.sh[s]["recv_off"]), o_eoff[s * L:(s + 1) * L + 1] - o_eoff[s * L])
+
+    # ---- step 5: dispatch into every rank's receive rows
+    em.dispatch()
+    assert em.check_errors() == 0
+    valid = o_dst >= 0
+    order = np.argsort(o_dst[valid])
+    gg = np.repeat(np.arange(w.N), K).reshape(w.N, K)
+    o_src = gg[valid][order].astype(np.int32)  # source token of every single-buffer row
+    o_rw = o_w[valid][order]
+    for d in range(R):
+        a, b = int(o_roff[d]), int(o_roff[d + 1])
+        rv = em.recv[d]
+        assert em.received_rows()[d] == b - a
+        assert np.array_equal(_to_host(rv["recv_src"][:b - a]), o_src[a:b])
+        g_rw = _to_host(rv["recv_w"][:b - a]).astype(np.float64)
+        assert (np.abs(g_rw - o_rw[a:b]) <= 2.0 ** -22 * np.abs(o_rw[a:b])).all()
+        n = b - a
+        pick = np.arange(n) if n * H <= 16 * 2 ** 20 else _sample_rows(n, o_eoff[d * L:(d + 1) * L + 1] - a, 500, seed)
+        g_rows = _to_host(rv["recv_x"].index_select(0, torch.from_numpy(pick).cuda()))
+        src = o_src[a:b][pick]
+        if not w.fp8:
+            assert np.array_equal(g_rows, x[src]), f"rank {d}"
+        else:
+            g_sc = _to_host(rv["recv_scale"].index_select(0, torch.from_numpy(pick).cuda()))
+            for i, g in enumerate(src):
+                q, sc = oracle.quant_fp8_row(x[g])
+                assert np.array_equal(g_rows[i], q) and np.array_equal(g_sc[i].view(np.uint32), sc.view(np.uint32))
+
+    # ---- step 7: combine from every rank's expert output
+    rng = np.random.default_rng(200 + seed)
+    tokens = np.arange(w.N) if w.N <= 1024 else np.unique(np.concatenate(
+        [rng.integers(0, w.N, 300), [0, w.N - 1], np.arange(1, R + 1) * T - 1, np.arange(R) * T]))
+    modes = ["bf16"] if not w.fp8 else ["fused", "fp8"]
+    for mode in modes:
+        if mode == "fp8":
+            em.identity_expert()
+        em.combine()
+        assert em.check_errors() == 0
+        got = _to_host(out.index_select(0, torch.from_numpy(tokens).cuda()))
+        _check_combine(got, _combine_expected(w, x, o_idx, o_w, tokens, mode))
+
+
+def test_shard_call_order_and_errors(cuda):
+    ep, shard = cuda
+    w = wl.WORKLOADS["tiny"]
+    T = w.T
+    from combine_top_group_b200 import runner
+    buf = ep.ep_buffer_create(shard.shard_config(w), device="cuda")
+    single = ep.ep_buffer_create(runner.make_config(w), device="cuda")
+    logits = torch.from_numpy(wl.make_logits(w, 0)[:T].copy()).cuda()
+    x = torch.zeros(T, w.H, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ep.EpError, match="created with EP_FLAG_SHARD"):
+        ep.ep_get_layout(buf, T, logits=logits)
+    with pytest.raises(ep.EpError, match="without EP_FLAG_SHARD"):
+        ep.ep_shard_layout(single, 0, T, logits=logits)
+    with pytest.raises(ep.EpError, match="no ep_shard_layout"):
+        ep.ep_shard_place(buf, 0, T)
+    with pytest.raises(ep.EpError, match="rank=9"):
+        ep.ep_shard_layout(buf, 9, T, logits=logits)
+    ep.ep_shard_layout(buf, 1, T, logits=logits)
+    rv = ep.ep_buffer_recv(buf)
+    tab = [rv["recv_x"]] * w.R
+    with pytest.raises(ep.EpError, match="ep_shard_place"):
+        ep.ep_shard_dispatch(buf, 1, T, x, tab, None, [rv["recv_src"]] * w.R, [rv["recv_w"]] * w.R)
+    with pytest.raises(ep.EpError, match="rank=0 does not match"):
+        ep.ep_shard_place(buf, 0, T)
+    sh = ep.ep_buffer_shard(buf, T)
+    sh["cnt_all"].zero_()
+    sh["cnt_all"][1].copy_(sh["cnt_row"])  # the only rank with tokens
+    ep.ep_shard_place(buf, 1, T)
+    with pytest.raises(ep.EpError, match="already ran"):
+        ep.ep_shard_place(buf, 1, T)
+    with pytest.raises(ep.EpError, match="entry 2 is NULL"):
+        ep.ep_shard_dispatch(buf, 1, T, x, tab[:2] + [0] + tab[3:], None, [rv["recv_src"]] * w.R,
+                             [rv["recv_w"]] * w.R)
+    assert ep.ep_check_errors(buf) == 0
+
+
+def test_shard_bad_counts_flag_rows(cuda):
+    """Counts that disagree with the rows they describe (a broken exchange)
+    cannot place a row outside the receive buffer: the row is dropped and the
+    error word says so."""
+    ep, shard = cuda
+    w = wl.WORKLOADS["tiny"]
+    T = w.T
+    buf = ep.ep_buffer_create(shard.shard_config(w), device="cuda")
+    logits = torch.from_numpy(wl.make_logits(w, 0)[:T].copy()).cuda()
+    ep.ep_shard_layout(buf, w.R - 1, T, logits=logits)
+    sh = ep.ep_buffer_shard(buf, T)
+    sh["cnt_all"].fill_(2 ** 27)  # a total far above M_max
+    ep.ep_shard_place(buf, w.R - 1, T)
+    word = ep.ep_check_errors(buf)
+    assert word & ep.EP_DEVERR_ROW_BOUNDS
+    dst = ep.ep_buffer_layout(buf, T)["dst_row"]
+    assert (dst.cpu() == -1).all()
