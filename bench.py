@@ -60,6 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--dedup", action="store_true",
                     help="also time the deduplicated-receive pipeline (dispatch_dedup, permute, local_reduce, "
                          "combine_dedup) on the same workload")
+    ap.add_argument("--graph", action="store_true",
+                    help="also time the step captured in a CUDA graph (one replay per step)")
     ap.add_argument("--shard", action="store_true",
                     help="also time the one-rank-per-GPU calls, R ranks emulated on this GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -254,8 +256,13 @@ def run_ours(args, w: wl.Workload, rank: int, world: int, local_rank: int):
         out["overlap"] = measure_overlap(pipe, w, dev, fused)
     if args.dedup:
         out["dedup"] = measure_dedup(w, rank, dev, fused, steps=min(args.steps, 10))
+    if args.graph:
+        t = time_graph(lambda: pipe.step(fused=fused), dev, flush, steps=args.steps)
+        out["graph"] = {"step_us": t * 1e6, "value": bytes_step / t / 1e9, "unit": "GB/s",
+                        "launches_per_step": 3, "steps": args.steps}
     if args.shard:
-        out["shard"] = (measure_shard(pipe, w, dev, fused, bytes_dispatch, bytes_combine, steps=min(args.steps, 10))
+        out["shard"] = (measure_shard(pipe, w, dev, fused, bytes_dispatch, bytes_combine, flush,
+                                      steps=min(args.steps, 10), graph=args.graph)
                         if world == 1 else {"skipped": "the emulated ranks run on one GPU (--gpus 1)"})
     ep.ep_buffer_set_num_sms(pipe.buf, args.num_sms)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -389,12 +396,44 @@ def measure_dedup(w, seed, dev, fused, steps):
     return res
 
 
-def measure_shard(pipe, w, dev, fused, bytes_dispatch, bytes_combine, steps):
+def time_graph(step, dev, flush, steps):
+    """Seconds per step of `step` captured once in a CUDA graph and replayed:
+    every launch of the step is enqueued by one graph launch, so host
+    overhead between kernels drops out. Events bracket each replay; the L2
+    flush (if any) runs between replays, outside them."""
+    import torch
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        step()  # warm-up on the capture stream's side
+    torch.cuda.current_stream(dev).wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in ev:
+        if flush is not None:
+            flush.fill_(1)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    t = sum(a.elapsed_time(b) for a, b in ev) / 1e3 / steps
+    del g
+    return t
+
+
+def measure_shard(pipe, w, dev, fused, bytes_dispatch, bytes_combine, flush, steps, graph=False):
     """The one-rank-per-GPU calls (EP_FLAG_SHARD) with all R ranks emulated on
     this GPU: per step R layouts, the count all-gather (device copies), R
     placements, R dispatches and R combines, each phase timed with events.
     The same rows move as in the single-buffer path, so the same algorithmic
-    bytes apply."""
+    bytes apply. Eagerly, the R small launches per phase are host-bound;
+    with graph=True the whole step is also timed as one CUDA graph replay."""
     import torch
 
     from combine_top_group_b200 import shard
@@ -412,6 +451,8 @@ def measure_shard(pipe, w, dev, fused, bytes_dispatch, bytes_combine, steps):
              lambda: em.dispatch(stream), lambda: em.combine(stream)]
     tot = [0.0] * len(calls)
     for _ in range(steps):
+        if flush is not None:
+            flush.fill_(1)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
         ev[0].record(stream)
         for i, c in enumerate(calls):
@@ -427,6 +468,8 @@ def measure_shard(pipe, w, dev, fused, bytes_dispatch, bytes_combine, steps):
     res["dispatch_gbs"] = bytes_dispatch / (tot[3] / steps) / 1e9
     res["combine_gbs"] = bytes_combine / (tot[4] / steps) / 1e9
     res["step_us"] = sum(tot) / steps * 1e6
+    if graph:
+        res["graph_step_us"] = time_graph(lambda: em.step(None), dev, flush, steps) * 1e6
     del em
     return res
 

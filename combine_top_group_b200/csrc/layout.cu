@@ -149,31 +149,36 @@ __device__ __forceinline__ uint32_t kept_groups(const LayoutParams& p, const uin
     if (gs % EPL == 0 && lpg <= 32 && (lpg & (lpg - 1)) == 0) {
         // each group spans lpg whole lanes: the lanes' top-2, then a butterfly
         top2_merge(a, b, lpg);
-        const int src = (lane < p.G) ? lane * lpg : 0;
+        // group g's score sits on its first lane, g * lpg; lanes in ascending
+        // order hold groups in ascending order
+        const bool leader = (lane & (lpg - 1)) == 0 && lane < p.G * lpg;
         const float s32 = sigmoid_f(key_value(a)) + sigmoid_f(key_value(b));
-        const float sc = __shfl_sync(FULL, s32, src);  // group `lane`'s fp32 score
-        for (int h = 0; h < p.G; ++h) {
-            const float sh = __shfl_sync(FULL, sc, h);
-            if (lane < p.G && (sh > sc || (sh == sc && h < lane))) ++rank;
+        // KG rounds of warp max over the scores' order keys (a score is > 0,
+        // so its key is never 0); equal scores go to the lower group
+        uint32_t sk = leader ? order_key(s32) : 0u;
+        uint32_t kept = 0u, last = 0u;
+        for (int r = 0; r < p.KG; ++r) {
+            const uint32_t m = __reduce_max_sync(FULL, sk);
+            const int win = __ffs(__ballot_sync(FULL, leader && sk == m)) - 1;
+            kept |= 1u << (win / lpg);
+            if (lane == win) sk = 0u;
+            last = m;
         }
         bool certain = true;
         if (p.KG < p.G) {
             // fp32 sigmoid error <= 3*2^-23 (expf <= 2 ulp, add and rcp 0.5 ulp each),
             // so a score errs by < 1e-6. A gap over 4e-6 decides as fp64 would.
-            const uint32_t m_last = __ballot_sync(FULL, lane < p.G && rank == p.KG - 1);
-            const uint32_t m_next = __ballot_sync(FULL, lane < p.G && rank == p.KG);
-            const float s_last = __shfl_sync(FULL, sc, __ffs(m_last) - 1);
-            const float s_next = __shfl_sync(FULL, sc, __ffs(m_next) - 1);
-            certain = (s_last - s_next) > 4e-6f;
+            const uint32_t next = __reduce_max_sync(FULL, sk);
+            certain = (key_value(last) - key_value(next)) > 4e-6f;
         }
-        if (!certain) {  // warp-uniform: decide in fp64
-            const double s64 = sigmoid_d((double)key_value(a)) + sigmoid_d((double)key_value(b));
-            const double sd = __shfl_sync(FULL, s64, src);
-            rank = 0;
-            for (int h = 0; h < p.G; ++h) {
-                const double sh = __shfl_sync(FULL, sd, h);
-                if (lane < p.G && (sh > sd || (sh == sd && h < lane))) ++rank;
-            }
+        if (certain) return kept;
+        // warp-uniform: decide in fp64
+        const int src = (lane < p.G) ? lane * lpg : 0;
+        const double s64 = sigmoid_d((double)key_value(a)) + sigmoid_d((double)key_value(b));
+        const double sd = __shfl_sync(FULL, s64, src);
+        for (int h = 0; h < p.G; ++h) {
+            const double sh = __shfl_sync(FULL, sd, h);
+            if (lane < p.G && (sh > sd || (sh == sd && h < lane))) ++rank;
         }
     } else {
         // generic layout of groups over lanes: one warp-wide top-2 per group, fp64
@@ -226,67 +231,63 @@ __device__ __forceinline__ void load_logits(const LayoutParams& p, int64_t g, in
     }
 }
 
-// Routes token g with one warp, from its logits vin (load_logits) when the
-// call routes logits. Lane k < K ends up holding slot k's expert id (-1 =
-// masked) and weight.
+// Per-warp staging of a group of B = 32 / K tokens: slot k of the group's
+// token j sits at index j*K + k, so the group's per-slot work (weights, mask,
+// writes, counts) runs once over all 32 lanes instead of once per token on K
+// lanes.
+struct WarpStage {
+    int32_t e[32];     // expert of each slot (-1: none)
+    uint32_t key[32];  // order key of the slot's logit
+    uint32_t mx[32];   // per token: key of its largest logit
+    double z[32];      // per token: sum over all experts of exp(l - max) (plain softmax)
+    double s[32];      // per slot: unnormalised weight
+    uint32_t rb[32];   // per slot: bit of its destination rank
+};
+
+// Selects token g's top-K with one warp from its logits vin (load_logits) and
+// stages slot k (expert, key) at st.e / st.key[j*K + k]. Ranking: logit
+// descending, then expert id ascending.
 template <int EPL>
-__device__ __forceinline__ void route_token(const LayoutParams& p, int64_t g, int lane, const float (&vin)[EPL],
-                                            int& my_e, float& my_w) {
-    my_e = -1;
-    my_w = 0.0f;
-    if (p.logits == nullptr) {
-        // caller-supplied top-k
-        if (lane < p.K) {
-            int e = p.in_idx[g * p.K + lane];
-            const float w = p.in_w[g * p.K + lane];
-            if (e < -1 || e >= p.E) {
-                set_error(p.err, EP_DEVERR_EXPERT_ID);
-                e = -1;
-            }
-            my_e = e;
-            my_w = w;
-        }
-    } else {
-        uint32_t key[EPL];
-        const int e0 = lane * EPL;
+__device__ __forceinline__ void select_token(const LayoutParams& p, int lane, const float (&vin)[EPL], int j,
+                                             WarpStage& st) {
+    uint32_t key[EPL];
+    const int e0 = lane * EPL;
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) key[j] = (e0 + j < p.E) ? order_key(vin[j]) : 0u;
+    for (int i = 0; i < EPL; ++i) key[i] = (e0 + i < p.E) ? order_key(vin[i]) : 0u;
 
-        // this lane's two best candidates; a lane rescans its list only when
-        // both have been taken
-        uint32_t a, b, taken = 0u;
-        int pa, pb;
-        top2_of<EPL>(key, 0u, a, pa, b, pb);
+    // this lane's two best candidates; a lane rescans its list only when
+    // both have been taken
+    uint32_t a, b, taken = 0u;
+    int pa, pb;
+    top2_of<EPL>(key, 0u, a, pa, b, pb);
 
-        if (p.route == EP_ROUTE_GROUP_SIGMOID && p.G > 1) {
-            const uint32_t kept = kept_groups<EPL>(p, key, a, b, lane);
-            const int gs = p.E / p.G;
-            if (gs % EPL == 0) {
-                // all of this lane's experts sit in group e0 / gs
-                if (!((kept >> (e0 / gs)) & 1u)) a = b = 0u;
-            } else {
+    if (p.route == EP_ROUTE_GROUP_SIGMOID && p.G > 1) {
+        const uint32_t kept = kept_groups<EPL>(p, key, a, b, lane);
+        const int gs = p.E / p.G;
+        if (gs % EPL == 0) {
+            // all of this lane's experts sit in group e0 / gs
+            if (!((kept >> (e0 / gs)) & 1u)) a = b = 0u;
+        } else {
 #pragma unroll
-                for (int j = 0; j < EPL; ++j) {
-                    const int e = e0 + j;
-                    if (e < p.E && !((kept >> (e / gs)) & 1u)) key[j] = 0u;
-                }
-                top2_of<EPL>(key, 0u, a, pa, b, pb);
+            for (int i = 0; i < EPL; ++i) {
+                const int e = e0 + i;
+                if (e < p.E && !((kept >> (e / gs)) & 1u)) key[i] = 0u;
             }
+            top2_of<EPL>(key, 0u, a, pa, b, pb);
         }
+    }
 
-        // top-K: K rounds of warp argmax on (logit desc, expert id asc)
-        uint32_t top_key = 0;
-        uint32_t my_key = 0;
-        for (int k = 0; k < p.K; ++k) {
-            const uint32_t wk = __reduce_max_sync(FULL, a);
-            const uint32_t cand = (a == wk && a != 0u) ? ~(uint32_t)(e0 + pa) : 0u;
-            const uint32_t wc = __reduce_max_sync(FULL, cand);
-            if (k == 0) top_key = wk;
-            if (lane == k) {
-                my_e = (wk != 0u) ? (int)~wc : -1;
-                my_key = wk;
-            }
-            if (cand != 0u && cand == wc) {  // this lane's head won: pop it
+    // top-K: K rounds of warp max. Equal keys go to the lowest lane, which
+    // holds the lowest expert ids; within a lane top2_of keeps id order.
+    const int base = j * p.K;
+    for (int k = 0; k < p.K; ++k) {
+        const uint32_t wk = __reduce_max_sync(FULL, a);
+        const int win = __ffs(__ballot_sync(FULL, a == wk)) - 1;
+        if (k == 0 && lane == 0) st.mx[j] = wk;
+        if (lane == win) {
+            st.e[base + k] = (wk != 0u) ? e0 + pa : -1;
+            st.key[base + k] = wk;
+            if (wk != 0u) {  // pop this lane's head
                 taken |= 1u << pa;
                 a = b;
                 pa = pb;
@@ -294,41 +295,103 @@ __device__ __forceinline__ void route_token(const LayoutParams& p, int64_t g, in
                 if (a == 0u) top2_of<EPL>(key, taken, a, pa, b, pb);
             }
         }
-        const float my_logit = key_value(my_key);
+    }
 
-        // weights, fp64
-        double wt = 0.0;
-        if (p.route == EP_ROUTE_GROUP_SIGMOID) {
-            const double s = (lane < p.K && my_e >= 0) ? sigmoid_d((double)my_logit) : 0.0;
-            double sum = 0.0;
-            for (int k = 0; k < p.K; ++k) sum += __shfl_sync(FULL, s, k);
-            wt = s / sum;
-        } else {
-            const double mx = (double)key_value(top_key);
-            double z = 0.0;
+    if (p.route == EP_ROUTE_SOFTMAX) {
+        // the normaliser of the plain softmax: every expert, fp64
+        __syncwarp();
+        const double mx = (double)key_value(st.mx[j]);
+        double z = 0.0;
 #pragma unroll
-            for (int j = 0; j < EPL; ++j)  // softmax routes never zero keys: key j is logit j
-                if (key[j] != 0u) z += exp((double)key_value(key[j]) - mx);
+        for (int i = 0; i < EPL; ++i)  // softmax routes never zero keys: key i is logit i
+            if (key[i] != 0u) z += exp((double)key_value(key[i]) - mx);
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(FULL, z, off);
-            const double pk = (lane < p.K && my_e >= 0) ? exp((double)my_logit - mx) / z : 0.0;
-            if (p.route == EP_ROUTE_SOFTMAX_RENORM) {
-                double sum = 0.0;
-                for (int k = 0; k < p.K; ++k) sum += __shfl_sync(FULL, pk, k);
-                wt = pk / sum;
-            } else {
-                wt = pk;
+        for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(FULL, z, off);
+        if (lane == 0) st.z[j] = z;
+    }
+}
+
+// Finishes the staged group: tokens g0 .. g0+nt-1 (global index g0 within
+// this launch), lane = j*K + k. Weights in fp64, rounded once to fp32:
+//  - group sigmoid: w_k = s_k / sum_k s_k, s = sigmoid(logit);
+//  - softmax: w_k = exp(l_k - max) / z;
+//  - renormalised softmax: w_k = p_k / sum_k p_k = exp(l_k - max) / sum_k exp(l_k - max)
+//    (z cancels).
+// The sums run over the token's slots in ascending k. Then the slot mask,
+// the topk_idx / topk_w writes (coalesced over the group), the per-warp
+// expert counts, is_token_in_rank and the per-warp rank counts.
+__device__ __forceinline__ void finish_group(const LayoutParams& p, int lane, int64_t g0, int nt, WarpStage& st,
+                                             int* my_hist) {
+    const int K = p.K;
+    const int jj = lane / K, k = lane - jj * K;
+    const bool act = jj < nt;
+    const int64_t g = g0 + jj;
+    int e = -1;
+    float w = 0.0f;
+    if (p.logits == nullptr) {
+        // caller-supplied top-k
+        if (act) {
+            e = p.in_idx[g * K + k];
+            w = p.in_w[g * K + k];
+            if (e < -1 || e >= p.E) {
+                set_error(p.err, EP_DEVERR_EXPERT_ID);
+                e = -1;
             }
         }
-        my_w = (lane < p.K) ? (float)wt : 0.0f;
+    } else {
+        __syncwarp();
+        e = act ? st.e[lane] : -1;
+        double sv = 0.0;
+        if (e >= 0) {
+            const double l = (double)key_value(st.key[lane]);
+            sv = (p.route == EP_ROUTE_GROUP_SIGMOID) ? sigmoid_d(l) : exp(l - (double)key_value(st.mx[jj]));
+        }
+        st.s[lane] = sv;
+        __syncwarp();
+        double den = 0.0;
+        if (p.route == EP_ROUTE_SOFTMAX) {
+            den = act ? st.z[jj] : 1.0;
+        } else if (act) {
+            for (int q = 0; q < K; ++q) den += st.s[jj * K + q];
+        }
+        w = (e >= 0) ? (float)(sv / den) : 0.0f;
     }
     // slot mask
-    if (lane < p.K && p.mask_thr != 0ull) {
-        const uint64_t h = splitmix64(p.mask_seed ^ (uint64_t)((p.g_base + g) * p.K + lane));
+    if (act && p.mask_thr != 0ull) {
+        const uint64_t h = splitmix64(p.mask_seed ^ (uint64_t)((p.g_base + g) * K + k));
         if ((h >> 32) < p.mask_thr) {
-            my_e = -1;
-            my_w = 0.0f;
+            e = -1;
+            w = 0.0f;
         }
+    }
+    if (act) {
+        p.topk_idx[g * K + k] = e;
+        p.topk_w[g * K + k] = w;
+        if (e >= 0) atomicAdd(&my_hist[e], 1);
+    }
+    st.rb[lane] = (e >= 0) ? (1u << (p.L == 1 ? (uint32_t)e : __umulhi((uint32_t)e, p.l_magic))) : 0u;
+    __syncwarp();
+    for (int i = lane; i < nt * p.R; i += 32) {
+        const int tj = i / p.R, r = i - tj * p.R;
+        uint32_t bits = 0u;
+        for (int q = 0; q < K; ++q) bits |= st.rb[tj * K + q];
+        const uint32_t in = (bits >> r) & 1u;
+        p.itr[(g0 + tj) * p.R + r] = (uint8_t)in;
+        if (in) atomicAdd(&my_hist[p.E + r], 1);
+    }
+    __syncwarp();  // the stage is refilled by the next group
+}
+
+// Outputs of column `col` for source rank r, whose chunks' exclusive prefix
+// starts at a and ends at b: src_off and cnt (expert columns), or
+// num_tokens_per_rank and the dedup rank offsets (rank columns).
+__device__ __forceinline__ void column_outputs(const LayoutParams& p, int col, int r, int a, int b) {
+    if (col < p.E) {
+        p.src_off[(int64_t)col * p.S + r] = a;
+        p.cnt[(int64_t)r * p.E + col] = b - a;
+    } else {
+        p.ntpr[(int64_t)r * p.R + (col - p.E)] = b - a;
+        if (p.dedup) p.rank_src_off[(int64_t)(col - p.E) * p.S + r] = a;
     }
 }
 
@@ -338,6 +401,7 @@ __global__ void __launch_bounds__(kThreads, 2) layout_kernel(LayoutParams p) {
     int* hist = sm;                      // [kWarps][J]: per-warp counts, later per-warp row bases
     int* eoff = sm + kWarps * p.J;       // [max(E, nc) + 1]: scan output
     __shared__ int warp_tot[33];
+    __shared__ WarpStage stage[kWarps];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int c = blockIdx.x;
@@ -353,35 +417,29 @@ __global__ void __launch_bounds__(kThreads, 2) layout_kernel(LayoutParams p) {
         w1 = t0 + (warp + 1) * n / kWarps;
     }
 
-    // ---- phase 1: route; per-warp expert and rank histograms
+    // ---- phase 1: route; per-warp expert and rank histograms. The warp
+    // selects B = 32 / K tokens one at a time, then finishes them together.
     for (int i = threadIdx.x; i < kWarps * p.J; i += kThreads) hist[i] = 0;
     __syncthreads();
     int* my_hist = hist + warp * p.J;
+    WarpStage& st = stage[warp];
+    const int B = 32 / p.K;
     float vnext[EPL];
     if (p.logits != nullptr && w0 < w1) load_logits<EPL>(p, (int64_t)s * p.T + w0, lane, vnext);
-    for (int t = w0; t < w1; ++t) {
-        const int64_t g = (int64_t)s * p.T + t;
-        float vcur[EPL];
+    for (int t0g = w0; t0g < w1; t0g += B) {
+        const int nt = min(B, w1 - t0g);
+        const int64_t g0 = (int64_t)s * p.T + t0g;
+        if (p.logits != nullptr) {
+            for (int j = 0; j < nt; ++j) {
+                const int t = t0g + j;
+                float vcur[EPL];
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) vcur[j] = vnext[j];
-        if (p.logits != nullptr && t + 1 < w1) load_logits<EPL>(p, g + 1, lane, vnext);  // prefetch
-        int e;
-        float w;
-        route_token<EPL>(p, g, lane, vcur, e, w);
-        if (lane < p.K) {
-            p.topk_idx[g * p.K + lane] = e;
-            p.topk_w[g * p.K + lane] = w;
-            if (e >= 0) atomicAdd(&my_hist[e], 1);
+                for (int i = 0; i < EPL; ++i) vcur[i] = vnext[i];
+                if (t + 1 < w1) load_logits<EPL>(p, g0 + j + 1, lane, vnext);  // prefetch
+                select_token<EPL>(p, lane, vcur, j, st);
+            }
         }
-        const uint32_t ranks =
-            __reduce_or_sync(FULL, (lane < p.K && e >= 0)
-                                       ? (1u << (p.L == 1 ? (uint32_t)e : __umulhi((uint32_t)e, p.l_magic)))
-                                       : 0u);
-        if (lane < p.R) {
-            const uint32_t in = (ranks >> lane) & 1u;
-            p.itr[g * p.R + lane] = (uint8_t)in;
-            my_hist[p.E + lane] += (int)in;
-        }
+        finish_group(p, lane, g0, nt, st, my_hist);
     }
     __syncthreads();
     if (has_chunk) {
@@ -394,30 +452,63 @@ __global__ void __launch_bounds__(kThreads, 2) layout_kernel(LayoutParams p) {
     }
     grid_barrier(p.bar, (uint32_t)p.nb, p.err);
 
-    // ---- phase 2: per-column exclusive scan over chunks (one CTA per column)
-    for (int col = blockIdx.x; col < p.J; col += p.nb) {
-        int32_t* colp = p.chunk + (int64_t)col * p.nc;
-        block_exclusive_scan(colp, 1, p.nc, eoff, warp_tot);  // eoff: scratch here, [nc + 1]
-        for (int cc = threadIdx.x; cc < p.nc; cc += kThreads) colp[cc] = eoff[cc];
-        // prefix at each rank's first chunk; eoff[nc] is the column total
-        if (threadIdx.x < p.S) {
-            const int r = threadIdx.x;  // source rank
-            const int a = (p.nc > 0) ? eoff[r * p.ncpr] : 0;
-            const int b = (p.nc > 0) ? eoff[(r + 1) * p.ncpr] : 0;  // (S * ncpr = nc) -> total
-            if (col < p.E) {
-                p.src_off[(int64_t)col * p.S + r] = a;
-                p.cnt[(int64_t)r * p.E + col] = b - a;
-            } else {
-                p.ntpr[(int64_t)r * p.R + (col - p.E)] = b - a;
-                if (p.dedup) p.rank_src_off[(int64_t)(col - p.E) * p.S + r] = a;
+    // ---- phase 2: per-column exclusive scan over chunks. Few chunks: one
+    // warp per column (4 chunks per lane). Otherwise one CTA per column.
+    if (p.nc <= 4 * 32) {
+        for (int col = blockIdx.x * kWarps + warp; col < p.J; col += p.nb * kWarps) {
+            int32_t* colp = p.chunk + (int64_t)col * p.nc;
+            int v[4];
+            int local = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int j = 4 * lane + i;
+                v[i] = (j < p.nc) ? colp[j] : 0;
+                local += v[i];
             }
+            int incl = local;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_up_sync(FULL, incl, off);
+                if (lane >= off) incl += o;
+            }
+            const int total = __shfl_sync(FULL, incl, 31);
+            int run = incl - local;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int j = 4 * lane + i;
+                if (j < p.nc) colp[j] = run;
+                run += v[i];
+            }
+            __syncwarp();  // the prefixes written above are read back by other lanes
+            if (lane < p.S) {
+                const int r = lane;  // source rank; S * ncpr = nc
+                const int a = (p.nc > 0) ? colp[r * p.ncpr] : 0;
+                const int b = (p.nc > 0 && r + 1 < p.S) ? colp[(r + 1) * p.ncpr] : total;
+                column_outputs(p, col, r, a, b);
+            }
+            if (lane == 0) {
+                p.tot[col] = total;
+                if (col < p.E) p.ntpe[col] = total;
+            }
+            __syncwarp();
         }
-        if (threadIdx.x == 0) {
-            const int total = (p.nc > 0) ? eoff[p.nc] : 0;
-            p.tot[col] = total;
-            if (col < p.E) p.ntpe[col] = total;
+    } else {
+        for (int col = blockIdx.x; col < p.J; col += p.nb) {
+            int32_t* colp = p.chunk + (int64_t)col * p.nc;
+            block_exclusive_scan(colp, 1, p.nc, eoff, warp_tot);  // eoff: scratch here, [nc + 1]
+            for (int cc = threadIdx.x; cc < p.nc; cc += kThreads) colp[cc] = eoff[cc];
+            // prefix at each rank's first chunk; eoff[nc] is the column total
+            if (threadIdx.x < p.S) {
+                const int r = threadIdx.x;  // source rank
+                column_outputs(p, col, r, eoff[r * p.ncpr], eoff[(r + 1) * p.ncpr]);
+            }
+            if (threadIdx.x == 0) {
+                const int total = eoff[p.nc];
+                p.tot[col] = total;
+                if (col < p.E) p.ntpe[col] = total;
+            }
+            __syncthreads();
         }
-        __syncthreads();
     }
     grid_barrier(p.bar, 2u * (uint32_t)p.nb, p.err);
 

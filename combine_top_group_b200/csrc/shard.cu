@@ -65,20 +65,26 @@ __global__ void __launch_bounds__(kPlaceThreads) shard_place_kernel(PlaceParams 
     // receive buffer (so the int32 prefix sums below cannot overflow)
     unsigned long long mine = 0ull;
     for (int e = threadIdx.x; e < p.E; e += kPlaceThreads) {
+        int v[kMaxPeers];
+#pragma unroll
+        for (int s = 0; s < kMaxPeers; ++s)  // all loads in flight at once
+            v[s] = (s < p.R) ? __ldg(p.cnt_all + (int64_t)s * p.E + e) : 0;
         long long tot = 0, before = 0;
         bool neg = false;
-        for (int s = 0; s < p.R; ++s) {
-            const int v = __ldg(p.cnt_all + (int64_t)s * p.E + e);
-            neg = neg || v < 0;
-            if (s < p.rank) before += v;
-            tot += v;
+#pragma unroll
+        for (int s = 0; s < kMaxPeers; ++s) {
+            neg = neg || v[s] < 0;
+            if (s < p.rank) before += v[s];
+            tot += v[s];
         }
         if (neg) s_bad = 1;
         mine += (unsigned long long)(tot < 0 ? 0 : tot);
         col[e] = (int)min(tot, (long long)p.m_max);
         pre[e] = (int)min(before, (long long)p.m_max);
     }
-    atomicAdd(&s_total, mine);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mine += __shfl_xor_sync(FULL, mine, off);
+    if ((threadIdx.x & 31) == 0) atomicAdd(&s_total, mine);  // one shared atomic per warp
     __syncthreads();
     const bool bad = s_bad || s_total > (unsigned long long)p.m_max;
     if (bad) {

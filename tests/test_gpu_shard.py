@@ -166,3 +166,51 @@ def test_shard_bad_counts_flag_rows(cuda):
     assert word & ep.EP_DEVERR_ROW_BOUNDS
     dst = ep.ep_buffer_layout(buf, T)["dst_row"]
     assert (dst.cpu() == -1).all()
+
+
+def test_shard_zero_tokens_and_ragged(cuda):
+    """T = 0 on every rank moves nothing; a T below T_max places rows with
+    global ids rank*T + t."""
+    ep, shard = cuda
+    from combine_top_group_b200 import runner
+    w = wl.WORKLOADS["tiny"]
+    cfg = shard.shard_config(w)
+    bufs = [ep.ep_buffer_create(cfg, device="cuda") for _ in range(w.R)]
+    for T in (0, 37):
+        lw = w.with_tokens(T)
+        logits = wl.make_logits(lw, 3)
+        x = wl.make_x(lw, 3)
+        lt = torch.from_numpy(np.ascontiguousarray(logits)).cuda() if T else torch.zeros(1, w.E, device="cuda")
+        xt = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+        out = torch.full((max(lw.N, 1), w.H), 7.0, dtype=torch.bfloat16, device="cuda")
+        for s, b in enumerate(bufs):
+            ep.ep_shard_layout(b, s, T, logits=lt[s * T:(s + 1) * T] if T else lt, route=runner.route_of(w))
+        rows = torch.stack([ep.ep_buffer_shard(b, T)["cnt_row"] for b in bufs])
+        for b in bufs:
+            ep.ep_buffer_shard(b, T)["cnt_all"].copy_(rows)
+        for s, b in enumerate(bufs):
+            ep.ep_shard_place(b, s, T)
+        recv = [ep.ep_buffer_recv(b) for b in bufs]
+        tabs = {k: [r[k] for r in recv] for k in ("recv_x", "recv_src", "recv_w")}
+        for s, b in enumerate(bufs):
+            ep.ep_shard_dispatch(b, s, T, xt[s * T:(s + 1) * T] if T else out, tabs["recv_x"], None,
+                                 tabs["recv_src"], tabs["recv_w"])
+        for s, b in enumerate(bufs):
+            ep.ep_shard_combine(b, s, T, tabs["recv_x"], None, out[s * T:(s + 1) * T] if T else out)
+        for b in bufs:
+            assert ep.ep_check_errors(b) == 0
+        got_rows = [int(ep.ep_buffer_shard(b, T)["recv_off"][-1].item()) for b in bufs]
+        o_idx, o_w, _ = _oracle_route(lw, logits)
+        o_lay = oracle.layout(o_idx, w.R, T, w.E)
+        assert got_rows == np.diff(o_lay["rank_off"]).tolist()
+        if T == 0:
+            assert (out.float() == 7.0).all()  # nothing written
+            continue
+        for d in range(w.R):
+            a, b_ = int(o_lay["rank_off"][d]), int(o_lay["rank_off"][d + 1])
+            valid = o_lay["dst_row"] >= 0
+            order = np.argsort(o_lay["dst_row"][valid])
+            src = np.repeat(np.arange(lw.N), w.K).reshape(lw.N, w.K)[valid][order]
+            assert np.array_equal(_to_host(recv[d]["recv_src"][:b_ - a]), src[a:b_].astype(np.int32))
+        got = _to_host(out[:lw.N])
+        _check_combine(got, _combine_expected(lw, x, o_idx, o_w, np.arange(lw.N), "bf16"))
