@@ -396,7 +396,7 @@ __device__ __forceinline__ void column_outputs(const LayoutParams& p, int col, i
 }
 
 template <int EPL>
-__global__ void __launch_bounds__(kThreads, 2) layout_kernel(LayoutParams p) {
+__global__ void __launch_bounds__(kThreads, EPL >= 16 ? 2 : 4) layout_kernel(LayoutParams p) {
     extern __shared__ int sm[];
     int* hist = sm;                      // [kWarps][J]: per-warp counts, later per-warp row bases
     int* eoff = sm + kWarps * p.J;       // [max(E, nc) + 1]: scan output
