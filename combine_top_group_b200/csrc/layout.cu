@@ -114,26 +114,31 @@ __device__ __forceinline__ void top2_merge(uint32_t& a, uint32_t& b, int span) {
     }
 }
 
-// This lane's two best candidates by (key desc, position asc), skipping
+// This lane's three best candidates by (key desc, position asc), skipping
 // taken positions and zero keys. Returns key 0 where there is none.
 template <int EPL>
-__device__ __forceinline__ void top2_of(const uint32_t (&key)[EPL], uint32_t taken, uint32_t& a, int& pa,
-                                        uint32_t& b, int& pb) {
-    a = 0u;
-    b = 0u;
-    pa = 0;
-    pb = 0;
+__device__ __forceinline__ void top3_of(const uint32_t (&key)[EPL], uint32_t taken, uint32_t& a, int& pa,
+                                        uint32_t& b, int& pb, uint32_t& c, int& pc) {
+    a = b = c = 0u;
+    pa = pb = pc = 0;
 #pragma unroll
     for (int j = 0; j < EPL; ++j) {
         const uint32_t k = ((taken >> j) & 1u) ? 0u : key[j];
         if (k > a) {  // strict: an equal key later in the list stays behind
+            c = b;
+            pc = pb;
             b = a;
             pb = pa;
             a = k;
             pa = j;
         } else if (k > b) {
+            c = b;
+            pc = pb;
             b = k;
             pb = j;
+        } else if (k > c) {
+            c = k;
+            pc = j;
         }
     }
 }
@@ -149,27 +154,47 @@ __device__ __forceinline__ uint32_t kept_groups(const LayoutParams& p, const uin
     if (gs % EPL == 0 && lpg <= 32 && (lpg & (lpg - 1)) == 0) {
         // each group spans lpg whole lanes: the lanes' top-2, then a butterfly
         top2_merge(a, b, lpg);
-        // group g's score sits on its first lane, g * lpg; lanes in ascending
-        // order hold groups in ascending order
-        const bool leader = (lane & (lpg - 1)) == 0 && lane < p.G * lpg;
+        // group g's fp32 score sits on lane g * lpg. A group's rank is the
+        // number of groups ahead of it: higher score, or equal score and lower
+        // id. Kept = rank < KG.
         const float s32 = sigmoid_f(key_value(a)) + sigmoid_f(key_value(b));
-        // KG rounds of warp max over the scores' order keys (a score is > 0,
-        // so its key is never 0); equal scores go to the lower group
-        uint32_t sk = leader ? order_key(s32) : 0u;
-        uint32_t kept = 0u, last = 0u;
-        for (int r = 0; r < p.KG; ++r) {
-            const uint32_t m = __reduce_max_sync(FULL, sk);
-            const int win = __ffs(__ballot_sync(FULL, leader && sk == m)) - 1;
-            kept |= 1u << (win / lpg);
-            if (lane == win) sk = 0u;
-            last = m;
+        float sg;   // score of group gq
+        int gq, rk;  // rank of group gq, on the lanes that report it
+        bool lead;  // this lane reports group gq
+        if (p.G <= 8) {
+            // all pairs at once: lane = 4*gq + q compares group gq with groups 2q, 2q+1
+            gq = lane >> 2;
+            const int q = lane & 3, h0 = 2 * q, h1 = 2 * q + 1;
+            sg = __shfl_sync(FULL, s32, (gq < p.G ? gq : 0) * lpg);
+            const float s0 = __shfl_sync(FULL, s32, (h0 < p.G ? h0 : 0) * lpg);
+            const float s1 = __shfl_sync(FULL, s32, (h1 < p.G ? h1 : 0) * lpg);
+            rk = (h0 < p.G && (s0 > sg || (s0 == sg && h0 < gq))) + (h1 < p.G && (s1 > sg || (s1 == sg && h1 < gq)));
+            rk += __shfl_xor_sync(FULL, rk, 1);
+            rk += __shfl_xor_sync(FULL, rk, 2);
+            lead = q == 0 && gq < p.G;
+        } else {
+            // lane g ranks group g against every group (independent shuffles)
+            gq = lane;
+            sg = __shfl_sync(FULL, s32, (lane < p.G ? lane : 0) * lpg);
+            rk = 0;
+            for (int h = 0; h < p.G; ++h) {
+                const float sh = __shfl_sync(FULL, sg, h);
+                rk += (sh > sg || (sh == sg && h < lane)) ? 1 : 0;
+            }
+            lead = lane < p.G;
         }
+        uint32_t kept = 0u;
+        for (uint32_t m = __ballot_sync(FULL, lead && rk < p.KG); m; m &= m - 1)
+            kept |= 1u << __shfl_sync(FULL, gq, __ffs(m) - 1);
         bool certain = true;
         if (p.KG < p.G) {
             // fp32 sigmoid error <= 3*2^-23 (expf <= 2 ulp, add and rcp 0.5 ulp each),
             // so a score errs by < 1e-6. A gap over 4e-6 decides as fp64 would.
-            const uint32_t next = __reduce_max_sync(FULL, sk);
-            certain = (key_value(last) - key_value(next)) > 4e-6f;
+            const uint32_t m_last = __ballot_sync(FULL, lead && rk == p.KG - 1);
+            const uint32_t m_next = __ballot_sync(FULL, lead && rk == p.KG);
+            const float s_last = __shfl_sync(FULL, sg, __ffs(m_last) - 1);
+            const float s_next = __shfl_sync(FULL, sg, __ffs(m_next) - 1);
+            certain = (s_last - s_next) > 4e-6f;
         }
         if (certain) return kept;
         // warp-uniform: decide in fp64
@@ -255,30 +280,30 @@ __device__ __forceinline__ void select_token(const LayoutParams& p, int lane, co
 #pragma unroll
     for (int i = 0; i < EPL; ++i) key[i] = (e0 + i < p.E) ? order_key(vin[i]) : 0u;
 
-    // this lane's two best candidates; a lane rescans its list only when
-    // both have been taken
-    uint32_t a, b, taken = 0u;
-    int pa, pb;
-    top2_of<EPL>(key, 0u, a, pa, b, pb);
+    // this lane's three best candidates; a lane rescans its list only when
+    // all three have been taken
+    uint32_t a, b, c, taken = 0u;
+    int pa, pb, pc;
+    top3_of<EPL>(key, 0u, a, pa, b, pb, c, pc);
 
     if (p.route == EP_ROUTE_GROUP_SIGMOID && p.G > 1) {
         const uint32_t kept = kept_groups<EPL>(p, key, a, b, lane);
         const int gs = p.E / p.G;
         if (gs % EPL == 0) {
             // all of this lane's experts sit in group e0 / gs
-            if (!((kept >> (e0 / gs)) & 1u)) a = b = 0u;
+            if (!((kept >> (e0 / gs)) & 1u)) a = b = c = 0u;
         } else {
 #pragma unroll
             for (int i = 0; i < EPL; ++i) {
                 const int e = e0 + i;
                 if (e < p.E && !((kept >> (e / gs)) & 1u)) key[i] = 0u;
             }
-            top2_of<EPL>(key, 0u, a, pa, b, pb);
+            top3_of<EPL>(key, 0u, a, pa, b, pb, c, pc);
         }
     }
 
     // top-K: K rounds of warp max. Equal keys go to the lowest lane, which
-    // holds the lowest expert ids; within a lane top2_of keeps id order.
+    // holds the lowest expert ids; within a lane top3_of keeps id order.
     const int base = j * p.K;
     for (int k = 0; k < p.K; ++k) {
         const uint32_t wk = __reduce_max_sync(FULL, a);
@@ -291,8 +316,10 @@ __device__ __forceinline__ void select_token(const LayoutParams& p, int lane, co
                 taken |= 1u << pa;
                 a = b;
                 pa = pb;
-                b = 0u;
-                if (a == 0u) top2_of<EPL>(key, taken, a, pa, b, pb);
+                b = c;
+                pb = pc;
+                c = 0u;
+                if (a == 0u) top3_of<EPL>(key, taken, a, pa, b, pb, c, pc);
             }
         }
     }

@@ -17,7 +17,7 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
 
-FALLBACK_HBM_GBS = 6650.0  # earlier measurement on this machine, used only without MEASURED_PEAKS.json
+FALLBACK_HBM_GBS = 6650.0  # an earlier B200 copy measurement, used only without MEASURED_PEAKS.json
 
 
 # ---- algorithmic bytes -------------------------------------------------------
@@ -66,7 +66,7 @@ def max_over_ranks(values, device=None):
 # ---- peaks -------------------------------------------------------------------
 
 def hbm_peak() -> tuple[float, str]:
-    """(GB/s, source): the measured copy bandwidth, else the fallback."""
+    """(GB/s, source): the measured copy bandwidth in MEASURED_PEAKS.json, else the fallback."""
     try:
         with open(PEAKS_FILE) as f:
             return float(json.load(f)["hbm_gbs"]), "measured"

@@ -48,7 +48,7 @@ typedef enum {
     EP_ERR_CAPACITY = 2,    /* more tokens than the buffer was sized for */
     EP_ERR_OOM = 3,         /* workspace smaller than ep_buffer_workspace_bytes */
     EP_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
-    EP_ERR_UNSUPPORTED = 5, /* valid shape this build does not handle */
+    EP_ERR_UNSUPPORTED = 5, /* a valid shape the library does not handle */
     EP_ERR_DEVICE = 6       /* ep_check_errors found device error bits */
 } ep_status_t;
 
