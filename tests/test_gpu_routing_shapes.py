@@ -1,0 +1,86 @@
+"""Routing + layout from logits on shapes the five workloads do not reach, so
+every branch of the routing kernel runs against the oracle:
+- experts per lane (EPL = E/32) of 3, 4, 16 and 32;
+- groups spanning several lanes, one lane, or not aligned to lanes;
+- more than 8 groups (the shuffle ranking) and at most 8 (the all-pairs ranking);
+- K = 32 (one token per finishing group), K not dividing 32, plain softmax
+  over 256 and 1024 experts, and the slot mask.
+Tolerances and near-tie handling are those of the workload parity tests."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from combine_top_group_b200 import workloads as wl
+from test_gpu_parity import _check_combine, _check_routing, _combine_expected, _oracle_route, _to_host
+
+pytestmark = pytest.mark.gpu
+
+S, R2 = wl.ROUTE_SOFTMAX, wl.ROUTE_SOFTMAX_RENORM
+G = wl.ROUTE_GROUP_SIGMOID
+SHAPES = [
+    wl.Workload("g32", R=2, T=50, H=128, E=256, K=8, G=32, KG=8, route=G),  # one lane per group, G > 8
+    wl.Workload("g3_unaligned", R=2, T=50, H=128, E=96, K=5, G=3, KG=2, route=G),  # EPL 3: groups split lanes
+    wl.Workload("g16_e512", R=4, T=40, H=128, E=512, K=8, G=16, KG=4, route=G),  # EPL 16, 2 lanes per group
+    wl.Workload("g4_e128", R=4, T=40, H=128, E=128, K=6, G=4, KG=2, route=G, mask_frac=0.2),  # EPL 4, G < 8
+    wl.Workload("softmax_e1024_k32", R=4, T=24, H=128, E=1024, K=32, route=S),  # EPL 32, K = 32
+    wl.Workload("softmax_e256", R=2, T=64, H=256, E=256, K=8, route=S),  # plain softmax z over 256
+    wl.Workload("renorm_e64_k3", R=4, T=33, H=128, E=64, K=3, route=R2, mask_frac=0.1),
+]
+
+
+@pytest.fixture(scope="module")
+def cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from combine_top_group_b200 import ep, runner  # loads libep.so; fails loudly if missing
+    return ep, runner
+
+
+@pytest.mark.parametrize("w", SHAPES, ids=[w.name for w in SHAPES])
+def test_routing_shapes(cuda, w):
+    ep, runner = cuda
+    x = wl.make_x(w, 7)
+    logits = wl.make_logits(w, 7)
+    pipe = runner.Pipeline(w, 7, x=x, logits=logits)
+    o_idx, o_w, margin = _oracle_route(w, logits)
+    pipe.layout()
+    assert pipe.check_errors() == 0
+    lay = {k: _to_host(v) for k, v in ep.ep_buffer_layout(pipe.buf, w.T).items()}
+    if _check_routing(w, o_idx, o_w, margin, lay["topk_idx"], lay["topk_w"]):
+        pipe.layout(topk_idx=torch.from_numpy(o_idx).cuda(), topk_w=torch.from_numpy(o_w).cuda())
+        lay = {k: _to_host(v) for k, v in ep.ep_buffer_layout(pipe.buf, w.T).items()}
+    o_lay = oracle.layout(o_idx, w.R, w.T, w.E)
+    for key in ("is_token_in_rank", "num_tokens_per_rank", "cnt", "num_tokens_per_expert", "expert_off",
+                "rank_off", "src_off", "dst_row"):
+        assert np.array_equal(lay[key], o_lay[key]), key
+    pipe.dispatch()
+    pipe.combine()
+    assert pipe.check_errors() == 0
+    tokens = np.arange(w.N)
+    _check_combine(_to_host(pipe.out), _combine_expected(w, x, o_idx, o_w, tokens, "bf16"))
+
+
+def test_group_score_ties_decide_by_lower_id(cuda):
+    """Groups with identical logits tie exactly in fp32: the kernel must fall
+    back to fp64 (still tied) and keep the lower group ids, then break the
+    expert ties by lower id too (reading 4), exactly as the oracle does.
+    Half the tokens tie all 8 groups; the other half tie groups 2 and 5 only."""
+    ep, runner = cuda
+    w = wl.Workload("ties", R=2, T=16, H=128, E=256, K=8, G=8, KG=4, route=G)
+    logits = wl.make_logits(w, 3)
+    half = w.N // 2
+    logits[:half] = np.tile(logits[:half, :32], (1, 8))
+    logits[half:, 160:192] = logits[half:, 64:96]
+    x = wl.make_x(w, 3)
+    pipe = runner.Pipeline(w, 3, x=x, logits=logits)
+    pipe.layout()
+    assert pipe.check_errors() == 0
+    lay = ep.ep_buffer_layout(pipe.buf, w.T)
+    o_idx, o_w, margin = _oracle_route(w, logits)
+    assert (margin[:half] == 0).all()  # exact ties on the all-equal tokens
+    assert np.array_equal(_to_host(lay["topk_idx"]), o_idx)
+    g_w = _to_host(lay["topk_w"]).astype(np.float64)
+    assert (np.abs(g_w - o_w) <= 2.0 ** -22 * np.abs(o_w)).all()
+    # all-equal tokens keep groups 0..3 only
+    assert (o_idx[:half] < 128).all()
