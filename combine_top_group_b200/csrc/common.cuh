@@ -1,6 +1,6 @@
-// Device helpers shared by the sm_100a kernels of libep: inline-PTX wrappers
-// for the bulk-copy (TMA) engine and mbarriers, number-format conversions,
-// and the bounded wait used by every spin in this library.
+// Device helpers shared by the sm_100a kernels of libep: 256-bit global
+// loads and stores, number-format conversions, the block scan, and the clock
+// behind the bounded wait of every spin in this library.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -14,104 +14,15 @@ namespace ep {
 constexpr unsigned FULL = 0xffffffffu;
 
 // A wait that has not finished after this long gives up and sets
-// EP_DEVERR_TIMEOUT. Every copy waited on is a local HBM -> shared-memory
-// copy that completes within microseconds, so reaching it means a bug.
+// EP_DEVERR_TIMEOUT. The only waits are the layout's grid barriers, whose
+// CTAs are all resident and finish their phase within microseconds, so
+// reaching it means a bug.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
-}
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// ---- mbarrier -------------------------------------------------------------
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-// Makes mbarrier initialisation visible to the async (bulk-copy) proxy.
-__device__ __forceinline__ void fence_mbar_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Waits for phase `parity` of `bar` to complete. Returns false (and the caller
-// must record EP_DEVERR_TIMEOUT) if it has not after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-    }
-    return true;
-}
-
-// ---- bulk copies (TMA engine, untiled, never multicast) -------------------
-
-// L2 policy: the streamed rows are touched once, so evict them first.
-__device__ __forceinline__ uint64_t l2_evict_first_policy() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
-// global -> shared, completion signalled on `bar` (bytes % 16 == 0, both
-// addresses 16-byte aligned).
-__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar,
-                                         uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(smem_dst)),
-        "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
-        : "memory");
-}
-
-// shared -> global, tracked by the issuing thread's bulk groups.
-__device__ __forceinline__ void bulk_s2g(void* gdst, const void* smem_src, uint32_t bytes, uint64_t policy) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(gdst),
-                 "r"(smem_u32(smem_src)), "r"(bytes), "l"(policy)
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-
-// Wait until at most N committed groups still read their shared-memory source.
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-
-// Wait until at most N committed groups are incomplete (writes done).
-template <int N>
-__device__ __forceinline__ void bulk_wait_all() {
-    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// Orders this thread's generic-proxy shared-memory writes before later
-// async-proxy (bulk copy) reads of them.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ---- 256-bit global loads and stores (sm_100) ------------------------------
@@ -132,12 +43,6 @@ __device__ __forceinline__ u32x8 ld256_stream(const void* p) {
 
 __device__ __forceinline__ void st256(void* p, const u32x8& a) {
     asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.v[0]), "r"(a.v[1]),
-                 "r"(a.v[2]), "r"(a.v[3]), "r"(a.v[4]), "r"(a.v[5]), "r"(a.v[6]), "r"(a.v[7])
-                 : "memory");
-}
-
-__device__ __forceinline__ void st256_stream(void* p, const u32x8& a) {
-    asm volatile("st.global.cs.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.v[0]), "r"(a.v[1]),
                  "r"(a.v[2]), "r"(a.v[3]), "r"(a.v[4]), "r"(a.v[5]), "r"(a.v[6]), "r"(a.v[7])
                  : "memory");
 }

@@ -85,8 +85,7 @@ struct LayoutArgs {
 };
 
 // int32 entries of layout scratch for a grid of at most max_ctas CTAs:
-// control words, per-chunk counts [E+R][max_ctas], totals [E+R], rank
-// prefixes [E+R][R+1].
+// control words, per-chunk counts [E+R][max_ctas], column totals [E+R].
 int64_t layout_scratch_ints(const ep_config_t& c, int max_ctas);
 
 // The layout kernel on caller-given outputs and scratch
