@@ -66,6 +66,8 @@ def parse_args(argv=None):
                     help="also time the one-rank-per-GPU calls, R ranks emulated on this GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-copy-streams", type=int, default=1,
+                    help="e2e: copy streams per direction (each copy split by rows)")
     return ap.parse_args(argv)
 
 
@@ -216,7 +218,8 @@ def run_ours(args, w: wl.Workload, rank: int, world: int, local_rank: int):
     # end to end through the C ABI from pinned host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps=max(K, 8), world=world)
+        e2e = measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps=max(K, 8), world=world,
+                          copy_streams=args.e2e_copy_streams)
 
     peak, peak_src = metrics.hbm_peak()
     d_avg, c_avg = t_disp / K, t_comb / K
@@ -474,15 +477,16 @@ def measure_shard(pipe, w, dev, fused, bytes_dispatch, bytes_combine, flush, ste
     return res
 
 
-def measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps, world):
+def measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps, world, copy_streams=1):
     """Same metric, through the C ABI, with the step's inputs copied in from
     pinned host memory and its result copied back, inside the timed region.
 
-    Steps are double-buffered: device x / logits / out have two slots, the
-    host-to-device copies run on one copy stream and the device-to-host copies
-    on another, so step i+1's inputs and step i-1's result cross PCIe (full
-    duplex) while step i computes. Every step still copies all of its inputs
-    in and its whole result out."""
+    Steps are double-buffered: device x / logits / out have two slots. The
+    host-to-device copies run on their own copy streams and the device-to-host
+    copies on others, so step i+1's inputs and step i-1's result cross PCIe
+    (full duplex) while step i computes. With copy_streams > 1 each copy is
+    split by rows over that many streams per direction. Every step still
+    copies all of its inputs in and its whole result out."""
     import torch
     import torch.distributed as dist
     x_h = pipe.x.cpu().pin_memory()
@@ -494,19 +498,31 @@ def measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps, world):
     ls = [pipe.logits, torch.empty_like(pipe.logits)]
     outs = [pipe.out, torch.empty_like(pipe.out)]
     keep = (pipe.x, pipe.logits, pipe.out)
-    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev = lambda: torch.cuda.Event()  # noqa: E731
-    in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    C = max(1, copy_streams)
+    s_in = [torch.cuda.Stream(dev) for _ in range(C)]
+    s_out = [torch.cuda.Stream(dev) for _ in range(C)]
+
+    def rows(t, c):  # row range c of C
+        n = t.shape[0]
+        return t[n * c // C:n * (c + 1) // C]
+
+    def ev():
+        return torch.cuda.Event()
+
+    in_done = [[ev() for _ in range(C)] for _ in range(2)]
+    out_done = [[ev() for _ in range(C)] for _ in range(2)]
+    comp_done = [ev(), ev()]
 
     def one(i):
         k = i % 2
-        s_in.wait_event(comp_done[k])  # step i-2 has finished reading slot k's inputs
-        with torch.cuda.stream(s_in):
-            xs[k].copy_(x_h, non_blocking=True)
-            ls[k].copy_(l_h, non_blocking=True)
-        in_done[k].record(s_in)
-        stream.wait_event(in_done[k])
-        stream.wait_event(out_done[k])  # step i-2's result has left slot k
+        for c in range(C):
+            s_in[c].wait_event(comp_done[k])  # step i-2 has finished reading slot k's inputs
+            with torch.cuda.stream(s_in[c]):
+                rows(xs[k], c).copy_(rows(x_h, c), non_blocking=True)
+                rows(ls[k], c).copy_(rows(l_h, c), non_blocking=True)
+            in_done[k][c].record(s_in[c])
+            stream.wait_event(in_done[k][c])
+            stream.wait_event(out_done[k][c])  # step i-2's result has left slot k
         pipe.x, pipe.logits, pipe.out = xs[k], ls[k], outs[k]
         pipe.layout(stream)
         pipe.dispatch(stream)
@@ -515,10 +531,11 @@ def measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps, world):
         else:
             pipe.combine(fused=fused, stream=stream)
         comp_done[k].record(stream)
-        s_out.wait_event(comp_done[k])
-        with torch.cuda.stream(s_out):
-            out_h.copy_(outs[k], non_blocking=True)
-        out_done[k].record(s_out)
+        for c in range(C):
+            s_out[c].wait_event(comp_done[k])
+            with torch.cuda.stream(s_out[c]):
+                rows(out_h, c).copy_(rows(outs[k], c), non_blocking=True)
+            out_done[k][c].record(s_out[c])
 
     try:
         for i in range(2):  # warm-up; records every event once
@@ -528,11 +545,13 @@ def measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps, world):
             dist.barrier()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record(stream)
-        s_in.wait_event(s)
+        for c in range(C):
+            s_in[c].wait_event(s)
         for i in range(steps):
             one(i)
-        stream.wait_event(out_done[(steps - 1) % 2])
-        stream.wait_event(out_done[steps % 2])
+        for k in range(2):
+            for c in range(C):
+                stream.wait_event(out_done[k][c])
         e.record(stream)
         torch.cuda.synchronize(dev)
     finally:
@@ -540,7 +559,7 @@ def measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps, world):
     t = metrics.max_over_ranks([s.elapsed_time(e) / 1e3], dev)[0]
     return {"value": world * bytes_step * steps / t / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": t / steps * 1e3,
-            "copies": "pinned host buffers; H2D and D2H on two copy streams, double-buffered across steps"}
+            "copies": f"pinned host buffers; H2D and D2H each on {C} copy stream(s), double-buffered across steps"}
 
 
 def main(argv=None):
