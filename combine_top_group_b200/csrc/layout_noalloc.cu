@@ -29,8 +29,8 @@
 namespace {
 
 // 2 MiB. The layout grid is capped so its chunk scratch fits:
-// (2 MiB/4 - 64 - (E+R)(R+2)) / (E+R) CTAs, e.g. all 1024 at E = 256, R = 8,
-// and about 460 at E = 1024, R = 32.
+// (2 MiB/4 - 64 - (E+R)) / (E+R) CTAs, e.g. all 1024 at E = 256, R = 8,
+// and 495 at E = 1024, R = 32.
 constexpr int64_t kNoAllocScratchInts = (2 << 20) / 4;
 
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchInts];

@@ -389,8 +389,8 @@ ep_status_t ep_selftest_wait_timeout(uint32_t *d_words, uint64_t limit_ns, uint3
  * counters, plus the per-chunk counts and their prefix sums. The call makes no
  * cudaMalloc, cudaFree or other allocating call.
  *  - Limit: the 2 MiB bound the layout grid (one CTA per chunk) to
- *    (524288 - 64 - (E+R)(R+2)) / (E+R) CTAs, at most 1024. All 1024 fit at
- *    E = 256, R = 8, and about 460 at E = 1024, R = 32. No valid config is
+ *    (524288 - 64 - (E+R)) / (E+R) CTAs, at most 1024. All 1024 fit at
+ *    E = 256, R = 8, and 495 at E = 1024, R = 32. No valid config is
  *    rejected; a smaller grid only means longer chunks.
  *  - d_error_word: a device uint32 that receives EP_DEVERR_* bits with
  *    atomicOr. The caller zeroes and reads it.
