@@ -8,7 +8,6 @@ import os
 import subprocess
 import sys
 
-import pytest
 import torch.multiprocessing as mp
 
 from combine_top_group_b200 import metrics
