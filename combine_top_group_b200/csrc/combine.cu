@@ -7,7 +7,7 @@
 // in fp32.
 //
 // One CTA per token (a grid-stride loop when num_sms caps the grid). Each
-// thread owns 16 channels of y: a 32-byte vector of
+// thread owns 16 channels of y at a time: a 32-byte vector of
 // bf16 (256-bit load) or a 16-byte vector of e4m3. It issues the K gathers of
 // that column before any arithmetic, so K loads are in flight per thread.
 // Loads use the streaming cache hint (y is read once). The 32 output bytes
@@ -25,7 +25,12 @@
 namespace ep {
 namespace {
 
-constexpr int kCombineThreads = 128;
+// Threads per CTA (one token per CTA). bf16 y: 4 warps, 4 CTAs per SM at 128
+// registers; 64, 192 and 256 threads were no faster on B200 over 1k-33k
+// tokens. e4m3 y (fused dequantisation, issue-bound): 2 warps, 12 CTAs per SM
+// at 80 registers; 1715 -> 1604 us against 4 warps on the large shape.
+constexpr int kBf16Threads = 128;
+constexpr int kFp8Threads = 64;
 
 struct CombineParams {
     int64_t N;
@@ -81,12 +86,12 @@ __device__ __forceinline__ void report_rows(const CombineParams& p, int64_t g) {
 }
 
 template <class Y>
-__global__ void __launch_bounds__(kCombineThreads) combine_bf16_kernel(CombineParams p, Y py) {
+__global__ void __launch_bounds__(kBf16Threads) combine_bf16_kernel(CombineParams p, Y py) {
     const int nvec = p.H / 16;  // 32-byte vectors: 16 bf16 channels
     const size_t rb = (size_t)p.H * 2;
     for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {  // grid-stride when num_sms caps the grid
         report_rows<Y>(p, g);
-        for (int v = threadIdx.x; v < nvec; v += kCombineThreads) {
+        for (int v = threadIdx.x; v < nvec; v += kBf16Threads) {
             float acc[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
@@ -127,13 +132,13 @@ __global__ void __launch_bounds__(kCombineThreads) combine_bf16_kernel(CombinePa
 }
 
 template <class Y>
-__global__ void __launch_bounds__(kCombineThreads) combine_fp8_kernel(CombineParams p, Y py) {
+__global__ void __launch_bounds__(kFp8Threads) combine_fp8_kernel(CombineParams p, Y py) {
     const int nvec = p.H / 16;  // 16 e4m3 channels (16 B) per vector
     const int nb = p.H / 128;
     const size_t rb = (size_t)p.H;
     for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {
         report_rows<Y>(p, g);
-        for (int v = threadIdx.x; v < nvec; v += kCombineThreads) {
+        for (int v = threadIdx.x; v < nvec; v += kFp8Threads) {
             float acc[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
@@ -193,19 +198,20 @@ __global__ void __launch_bounds__(kCombineThreads) combine_fp8_kernel(CombinePar
 template <class Y>
 cudaError_t launch_y(const ep_buffer& b, const CombineParams& p, const Y& py, bool fp8, cudaStream_t st) {
     auto kern = fp8 ? combine_fp8_kernel<Y> : combine_bf16_kernel<Y>;
+    const int threads = fp8 ? kFp8Threads : kBf16Threads;
     int64_t grid = p.N;
     const ep_config_t& c = b.cfg;
     const int sm_cap = (c.num_sms > 0 && c.num_sms < b.sm_count) ? c.num_sms : b.sm_count;
     if (sm_cap < b.sm_count) {
         // num_sms cap (Buffer.set_num_sms): a resident grid on sm_cap SMs' worth of CTAs
         int per_sm = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kCombineThreads, 0);
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);
         if (e != cudaSuccess) return e;
         grid = (int64_t)sm_cap * (per_sm > 0 ? per_sm : 1);
         if (grid > p.N) grid = p.N;
     }
     if (grid > 0x7fffffff) grid = 0x7fffffff;
-    kern<<<(unsigned)grid, kCombineThreads, 0, st>>>(p, py);
+    kern<<<(unsigned)grid, threads, 0, st>>>(p, py);
     return cudaGetLastError();
 }
 
