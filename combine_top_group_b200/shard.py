@@ -163,24 +163,35 @@ class DistributedRank:
     NCCL). The workspace is symmetric memory, so every rank can store into and
     load from every other rank's receive arrays.
 
-    Its host logic (count exchange, pointer tables) is tested on CPU ranks;
-    the repository has no multi-GPU test of it."""
+    Every call of a step runs on the current CUDA stream (or `stream`, made
+    current for the step), so the NCCL collectives (the count all-gather and
+    the barriers) are ordered after the kernels before them and before the
+    kernels after them.
 
-    def __init__(self, w: wl.Workload, device: torch.device, group=None, num_sms: int = 0):
+    `ep_lib` and `symm_mem_lib` default to the library binding and torch's
+    symmetric memory; the host logic (call order, count exchange, pointer
+    tables) is tested on CPU ranks with stand-ins for both. The repository has
+    no multi-GPU test of it."""
+
+    def __init__(self, w: wl.Workload, device: torch.device, group=None, num_sms: int = 0, ep_lib=None,
+                 symm_mem_lib=None):
         import torch.distributed as dist
-        from torch.distributed import _symmetric_memory as symm_mem
+        if symm_mem_lib is None:
+            from torch.distributed import _symmetric_memory as symm_mem_lib
+        self.ep = ep if ep_lib is None else ep_lib
         self.w = w
         self.group = group
         self.rank = dist.get_rank(group)
         if dist.get_world_size(group) != w.R:
             raise ValueError(f"world size {dist.get_world_size(group)} != R={w.R}")
         cfg = shard_config(w, num_sms)
-        nbytes = ep.ep_buffer_workspace_bytes(cfg)
-        self.workspace = symm_mem.empty(nbytes, dtype=torch.uint8, device=device)
-        self.handle = symm_mem.rendezvous(self.workspace, group=group if group is not None else dist.group.WORLD)
-        self.buf = ep.ep_buffer_create(cfg, workspace=self.workspace)
-        self.recv = ep.ep_buffer_recv(self.buf)
-        self.sh = ep.ep_buffer_shard(self.buf, w.T)
+        nbytes = self.ep.ep_buffer_workspace_bytes(cfg)
+        self.workspace = symm_mem_lib.empty(nbytes, dtype=torch.uint8, device=device)
+        self.handle = symm_mem_lib.rendezvous(self.workspace,
+                                              group=group if group is not None else dist.group.WORLD)
+        self.buf = self.ep.ep_buffer_create(cfg, workspace=self.workspace)
+        self.recv = self.ep.ep_buffer_recv(self.buf)
+        self.sh = self.ep.ep_buffer_shard(self.buf, w.T)
         self.peers = peer_tables(self.workspace.data_ptr(), list(self.handle.buffer_ptrs),
                                  {k: self.recv[k] for k in ("recv_x", "recv_scale", "recv_src", "recv_w")})
 
@@ -191,16 +202,19 @@ class DistributedRank:
     def step(self, x: torch.Tensor, logits: torch.Tensor, out: torch.Tensor, expert=None, stream=None):
         """One step for this rank's T tokens. `expert(recv_x, recv_scale, rows)`
         may transform the received rows in place (identity when None)."""
-        w, s, b = self.w, self.rank, self.buf
-        ep.ep_shard_layout(b, s, w.T, logits=logits, route=route_of(w), mask_seed=w.mask_seed,
-                           mask_frac=w.mask_frac, stream=stream)
-        exchange_counts(self.sh["cnt_row"], self.sh["cnt_all"], self.group)
-        ep.ep_shard_place(b, s, w.T, stream=stream)
-        self.barrier()  # every rank is done reading the previous step's rows
-        p = self.peers
-        ep.ep_shard_dispatch(b, s, w.T, x, p["recv_x"], p["recv_scale"], p["recv_src"], p["recv_w"], stream=stream)
-        self.barrier()  # every rank's rows are written
-        if expert is not None:
-            expert(self.recv["recv_x"], self.recv["recv_scale"], int(self.sh["recv_off"][-1].item()))
-        self.barrier()  # every expert output is ready
-        ep.ep_shard_combine(b, s, w.T, p["recv_x"], p["recv_scale"] if w.fp8 else None, out, stream=stream)
+        import contextlib
+        w, s, b, lib = self.w, self.rank, self.buf, self.ep
+        ctx = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+        with ctx:
+            lib.ep_shard_layout(b, s, w.T, logits=logits, route=route_of(w), mask_seed=w.mask_seed,
+                                mask_frac=w.mask_frac)
+            exchange_counts(self.sh["cnt_row"], self.sh["cnt_all"], self.group)
+            lib.ep_shard_place(b, s, w.T)
+            self.barrier()  # every rank is done reading the previous step's rows
+            p = self.peers
+            lib.ep_shard_dispatch(b, s, w.T, x, p["recv_x"], p["recv_scale"], p["recv_src"], p["recv_w"])
+            self.barrier()  # every rank's rows are written
+            if expert is not None:
+                expert(self.recv["recv_x"], self.recv["recv_scale"], int(self.sh["recv_off"][-1].item()))
+            self.barrier()  # every expert output is ready
+            lib.ep_shard_combine(b, s, w.T, p["recv_x"], p["recv_scale"] if w.fp8 else None, out)

@@ -87,3 +87,122 @@ def test_peer_tables_keep_offsets():
     assert t["recv_scale"] is None
     assert t["recv_src"] == [p + (1 << 30) for p in peers]
     assert t["recv_x"][1] == base + 4096  # this rank's own entry is its local pointer
+
+
+class _FakeSymmMem:
+    """Stand-in for torch symmetric memory on CPU ranks: a plain workspace,
+    and made-up per-rank base addresses as the peer mappings."""
+
+    def __init__(self, R):
+        self.bases = [0x7000_0000_0000 + d * 0x10_0000_0000 for d in range(R)]
+
+    def empty(self, n, dtype, device):
+        return torch.zeros(n, dtype=dtype)
+
+    def rendezvous(self, t, group):
+        class H:
+            pass
+        h = H()
+        h.buffer_ptrs = list(self.bases)
+        return h
+
+
+class _FakeEp:
+    """Stand-in for the library binding: records the calls, routes with the
+    oracle, and lays the receive arrays out inside the workspace so that the
+    peer tables can be checked."""
+
+    def __init__(self, w):
+        self.w = w
+        self.calls = []
+        self.ws = None
+
+    def ep_buffer_workspace_bytes(self, cfg):
+        assert cfg.flags & 0x8  # EP_FLAG_SHARD
+        return 1 << 16
+
+    def ep_buffer_create(self, cfg, workspace):
+        self.ws = workspace
+        return "buf"
+
+    def ep_buffer_recv(self, buf):
+        return {"recv_x": self.ws[256:4096], "recv_scale": None, "recv_src": self.ws[4096:8192],
+                "recv_w": self.ws[8192:12288]}
+
+    def ep_buffer_shard(self, buf, T):
+        w = self.w
+        self.sh = {"cnt_row": torch.zeros(w.E, dtype=torch.int32),
+                   "cnt_all": torch.zeros(w.R, w.E, dtype=torch.int32),
+                   "recv_off": torch.zeros(w.L + 1, dtype=torch.int32)}
+        return self.sh
+
+    def ep_shard_layout(self, b, s, T, logits, route, mask_seed, mask_frac):
+        import oracle
+        idx, _, _ = oracle.route(np.ascontiguousarray(logits.numpy()), self.w.K, route, self.w.G, self.w.KG)
+        self.sh["cnt_row"].copy_(torch.from_numpy(np.bincount(idx.ravel(), minlength=self.w.E).astype(np.int32)))
+        self.calls.append(("layout", s, T))
+
+    def ep_shard_place(self, b, s, T):
+        self.calls.append(("place", s, T, self.sh["cnt_all"].numpy().copy()))
+
+    def ep_shard_dispatch(self, b, s, T, x, tx, ts, tr, tw):
+        self.calls.append(("dispatch", s, T, list(tx), ts, list(tr), list(tw)))
+
+    def ep_shard_combine(self, b, s, T, ty, tys, out):
+        self.calls.append(("combine", s, T, list(ty), tys))
+
+
+W2 = wl.Workload("two_ranks_plain", R=2, T=64, H=128, E=16, K=4, route=wl.ROUTE_SOFTMAX)
+
+
+def _driver_rank_main(rank: int, world: int, port: int, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from combine_top_group_b200 import shard
+        fake = _FakeEp(W2)
+        drv = shard.DistributedRank(W2, torch.device("cpu"), ep_lib=fake, symm_mem_lib=_FakeSymmMem(world))
+        real_barrier = drv.barrier
+        drv.barrier = lambda: (fake.calls.append(("barrier",)), real_barrier())
+        logits = torch.from_numpy(wl.make_logits(W2, 0)[rank * W2.T:(rank + 1) * W2.T].copy())
+        drv.step(torch.zeros(W2.T, W2.H), logits, torch.zeros(W2.T, W2.H))
+        q.put((rank, fake.calls))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_distributed_driver_order_exchange_and_tables():
+    """DistributedRank on 2 gloo ranks, with stand-ins for the kernels and for
+    symmetric memory: the calls come in the method's order, the count rows
+    are exchanged before placement, and the peer tables point at the same
+    offset inside every rank's (stand-in) workspace."""
+    import oracle
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_driver_rank_main, args=(r, W2.R, port, q)) for r in range(W2.R)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in procs:
+        r, calls = q.get(timeout=120)
+        res[r] = calls
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    idx, _, _ = oracle.route(wl.make_logits(W2, 0), W2.K, W2.route)
+    want_cnt = oracle.layout(idx, W2.R, W2.T, W2.E)["cnt"]
+    bases = _FakeSymmMem(W2.R).bases
+    for r, calls in res.items():
+        kinds = [c[0] for c in calls]
+        # barriers: before dispatch (rows free), after it (rows written), after the experts
+        assert kinds == ["layout", "place", "barrier", "dispatch", "barrier", "barrier", "combine"]
+        layout, place, disp, comb = (c for c in calls if c[0] != "barrier")
+        assert layout[1] == r and place[1] == r and disp[1] == r and comb[1] == r
+        assert np.array_equal(place[3], want_cnt)  # all-gathered before placement
+        # recv_x sits 256 B into every workspace; recv_src 4096 B; recv_w 8192 B
+        assert disp[3] == [b + 256 for b in bases]
+        assert disp[5] == [b + 4096 for b in bases] and disp[6] == [b + 8192 for b in bases]
+        assert disp[4] is None and comb[4] is None  # bf16: no scale tables
+        assert comb[3] == [b + 256 for b in bases]  # combine reads every rank's rows
