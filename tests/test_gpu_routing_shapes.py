@@ -26,6 +26,11 @@ SHAPES = [
     wl.Workload("softmax_e1024_k32", R=4, T=24, H=128, E=1024, K=32, route=S),  # EPL 32, K = 32
     wl.Workload("softmax_e256", R=2, T=64, H=256, E=256, K=8, route=S),  # plain softmax z over 256
     wl.Workload("renorm_e64_k3", R=4, T=33, H=128, E=64, K=3, route=R2, mask_frac=0.1),
+    # limits: 32 ranks (a full 32-bit rank mask), the largest hidden size (dispatch with 8
+    # vectors per thread, combine looping 4096 vectors), bf16 and FP8
+    wl.Workload("ranks32", R=32, T=8, H=128, E=64, K=4, route=S),
+    wl.Workload("hidden65536_bf16", R=2, T=4, H=65536, E=4, K=2, route=S),
+    wl.Workload("hidden65536_fp8", R=2, T=4, H=65536, E=4, K=2, route=S, fp8=True),
 ]
 
 
@@ -55,10 +60,27 @@ def test_routing_shapes(cuda, w):
                 "rank_off", "src_off", "dst_row"):
         assert np.array_equal(lay[key], o_lay[key]), key
     pipe.dispatch()
-    pipe.combine()
+    mode = "bf16"
+    if w.fp8:
+        # the e4m3 rows against the oracle's cast, then the fused-dequant combine
+        M = int(o_lay["expert_off"][-1])
+        dst = o_lay["dst_row"]
+        src = np.repeat(np.arange(w.N), w.K).reshape(w.N, w.K)[dst >= 0][np.argsort(dst[dst >= 0])]
+        g_rows = _to_host(pipe.recv["recv_x"][:M])
+        g_sc = _to_host(pipe.recv["recv_scale"][:M])
+        for i, g in enumerate(src):
+            q, sc = oracle.quant_fp8_row(x[g])
+            assert np.array_equal(g_rows[i], q) and np.array_equal(g_sc[i].view(np.uint32), sc.view(np.uint32))
+        mode = "fused"
+    else:
+        M = int(o_lay["expert_off"][-1])
+        dst = o_lay["dst_row"]
+        src = np.repeat(np.arange(w.N), w.K).reshape(w.N, w.K)[dst >= 0][np.argsort(dst[dst >= 0])]
+        assert np.array_equal(_to_host(pipe.recv["recv_x"][:M]), x[src])
+    pipe.combine(fused=w.fp8)
     assert pipe.check_errors() == 0
     tokens = np.arange(w.N)
-    _check_combine(_to_host(pipe.out), _combine_expected(w, x, o_idx, o_w, tokens, "bf16"))
+    _check_combine(_to_host(pipe.out), _combine_expected(w, x, o_idx, o_w, tokens, mode))
 
 
 def test_group_score_ties_decide_by_lower_id(cuda):

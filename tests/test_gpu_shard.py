@@ -26,13 +26,14 @@ def cuda():
     return ep, shard
 
 
-CASES = [("tiny", 0), ("tiny", 2), ("decode", 1), ("prefill", 0), ("skewed", 2)]
+CASES = [("tiny", 0), ("tiny", 2), ("decode", 1), ("prefill", 0), ("skewed", 2), ("ranks32", 0)]
+EXTRA = {"ranks32": wl.Workload("ranks32", R=32, T=8, H=128, E=64, K=4, route=wl.ROUTE_SOFTMAX)}
 
 
 @pytest.mark.parametrize("name,seed", CASES, ids=[f"{n}-s{s}" for n, s in CASES])
 def test_shard_parity(cuda, name, seed):
     ep, shard = cuda
-    w = wl.WORKLOADS[name]
+    w = EXTRA[name] if name in EXTRA else wl.WORKLOADS[name]
     R, T, E, K, L, H = w.R, w.T, w.E, w.K, w.L, w.H
     x = wl.make_x(w, seed)
     logits = wl.make_logits(w, seed)
