@@ -13,6 +13,7 @@ import torch
 
 import oracle
 from combine_top_group_b200 import workloads as wl
+from shard_view import shard_view
 from test_gpu_parity import _check_combine, _check_routing, _combine_expected, _oracle_route, _sample_rows, _to_host
 
 pytestmark = pytest.mark.gpu
@@ -51,47 +52,41 @@ def test_shard_parity(cuda, name, seed):
     if _check_routing(w, o_idx, o_w, margin, g_idx, g_w):
         em.layout(topk_idx=torch.from_numpy(o_idx).cuda(), topk_w=torch.from_numpy(o_w).cuda())
     o_lay = oracle.layout(o_idx, R, T, E)
+    views = shard_view(o_idx, o_lay, R, T, E)
     for s, b in enumerate(em.bufs):
         lay = {k: _to_host(v) for k, v in ep.ep_buffer_layout(b, T).items()}
         assert np.array_equal(lay["is_token_in_rank"], o_lay["is_token_in_rank"][s * T:(s + 1) * T])
         assert np.array_equal(lay["num_tokens_per_rank"][0], o_lay["num_tokens_per_rank"][s])
-        assert np.array_equal(_to_host(em.sh[s]["cnt_row"]), o_lay["cnt"][s])
+        assert np.array_equal(_to_host(em.sh[s]["cnt_row"]), views[s]["cnt_row"])
+        assert np.array_equal(lay["dst_row"], views[s]["local_rows"])  # rank-local rows before placement
 
     # ---- steps 2-3: exchange, placement on the destination ranks
     em.exchange()
     em.place()
     assert em.check_errors() == 0
-    o_dst, o_eoff, o_roff = o_lay["dst_row"], o_lay["expert_off"], o_lay["rank_off"]
     for s in range(R):
-        rows = slice(s * T, (s + 1) * T)
-        idx = o_idx[rows]
-        valid = idx >= 0
-        want_rank = np.where(valid, idx // L, 0)
-        want_row = np.where(valid, o_dst[rows] - o_roff[want_rank], -1)
-        assert np.array_equal(_to_host(em.sh[s]["dst_rank"]), want_rank.astype(np.uint8))
-        assert np.array_equal(_to_host(ep.ep_buffer_layout(em.bufs[s], T)["dst_row"]), want_row)
-        assert np.array_equal(_to_host(em.sh[s]["recv_count"]), o_lay["num_tokens_per_expert"][s * L:(s + 1) * L])
-        assert np.array_equal(_to_host(em.sh[s]["recv_off"]), o_eoff[s * L:(s + 1) * L + 1] - o_eoff[s * L])
+        assert np.array_equal(_to_host(em.sh[s]["dst_rank"]), views[s]["dst_rank"])
+        assert np.array_equal(_to_host(ep.ep_buffer_layout(em.bufs[s], T)["dst_row"]), views[s]["dst_row"])
+        assert np.array_equal(_to_host(em.sh[s]["recv_count"]), views[s]["recv_count"])
+        assert np.array_equal(_to_host(em.sh[s]["recv_off"]), views[s]["recv_off"])
 
     # ---- step 5: dispatch into every rank's receive rows
     em.dispatch()
     assert em.check_errors() == 0
+    o_dst, o_eoff, o_roff = o_lay["dst_row"], o_lay["expert_off"], o_lay["rank_off"]
     valid = o_dst >= 0
-    order = np.argsort(o_dst[valid])
-    gg = np.repeat(np.arange(w.N), K).reshape(w.N, K)
-    o_src = gg[valid][order].astype(np.int32)  # source token of every single-buffer row
-    o_rw = o_w[valid][order]
+    o_rw = o_w[valid][np.argsort(o_dst[valid])]
     for d in range(R):
         a, b = int(o_roff[d]), int(o_roff[d + 1])
         rv = em.recv[d]
         assert em.received_rows()[d] == b - a
-        assert np.array_equal(_to_host(rv["recv_src"][:b - a]), o_src[a:b])
+        assert np.array_equal(_to_host(rv["recv_src"][:b - a]), views[d]["recv_src"])
         g_rw = _to_host(rv["recv_w"][:b - a]).astype(np.float64)
         assert (np.abs(g_rw - o_rw[a:b]) <= 2.0 ** -22 * np.abs(o_rw[a:b])).all()
         n = b - a
         pick = np.arange(n) if n * H <= 16 * 2 ** 20 else _sample_rows(n, o_eoff[d * L:(d + 1) * L + 1] - a, 500, seed)
         g_rows = _to_host(rv["recv_x"].index_select(0, torch.from_numpy(pick).cuda()))
-        src = o_src[a:b][pick]
+        src = views[d]["recv_src"][pick]
         if not w.fp8:
             assert np.array_equal(g_rows, x[src]), f"rank {d}"
         else:

@@ -206,3 +206,20 @@ def test_distributed_driver_order_exchange_and_tables():
         assert disp[5] == [b + 4096 for b in bases] and disp[6] == [b + 8192 for b in bases]
         assert disp[4] is None and comb[4] is None  # bf16: no scale tables
         assert comb[3] == [b + 256 for b in bases]  # combine reads every rank's rows
+
+
+def test_shard_view_matches_hand_worked_example(golden):
+    """The test-side derivation of every rank's view from the single-buffer
+    oracle (tests/shard_view.py, used by the GPU shard tests) against a
+    hand-worked example."""
+    import oracle
+    from shard_view import shard_view
+    g = golden("layout_example.txt")
+    R, T, E, K = int(g["R"][0]), int(g["T"][0]), int(g["E"][0]), int(g["K"][0])
+    idx = np.array([int(v) for v in g["topk_idx"]], dtype=np.int32).reshape(R * T, K)
+    lay = oracle.layout(idx, R, T, E)
+    want = golden("shard_example.txt")
+    for s, view in enumerate(shard_view(idx, lay, R, T, E)):
+        for key in ("local_rows", "dst_rank", "dst_row", "cnt_row", "recv_count", "recv_off", "recv_src"):
+            exp = np.array([int(v) for v in want[f"{key}_{s}"]])
+            assert np.array_equal(np.asarray(view[key]).ravel().astype(np.int64), exp), (key, s)
