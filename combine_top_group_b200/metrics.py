@@ -220,6 +220,8 @@ class ClockSampler:
         self.thread = None
         self.samples = []  # (t, sm_mhz, max_mhz, power_w or None, reasons)
         self._stop = None
+        self._read = None  # one NVML sample (the thread's body), also callable from the caller's thread
+        self._last = 0.0
 
     def start(self):
         try:
@@ -233,16 +235,21 @@ class ClockSampler:
             mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
             self._stop = threading.Event()
 
+            def read(with_power: bool):
+                try:
+                    sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0 if with_power else None
+                    self.samples.append((time.perf_counter(), sm, mx, pw, rs))
+                except Exception:  # noqa: BLE001 - sampling is best effort
+                    pass
+
+            self._read = read
+
             def run():
                 i = 0
                 while not self._stop.is_set():
-                    try:
-                        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
-                        rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
-                        pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0 if i % 10 == 0 else None
-                        self.samples.append((time.perf_counter(), sm, mx, pw, rs))
-                    except Exception:  # noqa: BLE001 - sampling is best effort
-                        pass
+                    read(i % 10 == 0)
                     i += 1
                     self._stop.wait(self.interval)
 
@@ -257,6 +264,19 @@ class ClockSampler:
         except OSError:
             self.proc = None
         return self
+
+    def sample_now(self, min_gap_s: float = 0.001) -> None:
+        """One sample from the caller's thread, at most every min_gap_s. The
+        bench calls it between step launches, so that the timed region holds
+        samples even when the host loop keeps the sampling thread off the
+        interpreter for its whole (short) duration."""
+        import time
+        if self._read is None:
+            return
+        now = time.perf_counter()
+        if now - self._last >= min_gap_s:
+            self._last = now
+            self._read(False)
 
     def stop(self, t0: float | None = None, t1: float | None = None) -> dict | None:
         """Stops sampling. Summarises the samples taken in [t0, t1] (host
