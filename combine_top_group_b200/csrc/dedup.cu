@@ -27,7 +27,8 @@ namespace ep {
 namespace {
 
 constexpr int kMaxRK = 32;
-constexpr int kThreads = 128;  // permute / reduce / combine
+constexpr int kThreads = 128;    // permute / reduce / combine
+constexpr int kReduceBatch = 4;  // local_reduce: gathers in flight per thread
 
 struct DedupParams {
     int64_t N;
@@ -218,10 +219,12 @@ __global__ void __launch_bounds__(512) permute_kernel(DedupParams p) {
 // ---------------------------------------------------------------------------
 // local_reduce: per (token, rank) weighted sum of that rank's expert outputs
 // ---------------------------------------------------------------------------
+template <bool FP8>
 __global__ void __launch_bounds__(kThreads) local_reduce_kernel(DedupParams p) {
     __shared__ int32_t s_d[kMaxRK];
-    __shared__ int32_t s_row[kMaxRK];
+    __shared__ int32_t s_row[kMaxRK];  // the row's local slots, compacted, k ascending
     __shared__ float s_w[kMaxRK];
+    __shared__ int s_nl;
     const int nvec = p.H / 16;  // 16 channels per thread: 32 B of bf16 y, or 16 B of e4m3 y
     const int nb = p.H / 128;
     for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {
@@ -230,40 +233,68 @@ __global__ void __launch_bounds__(kThreads) local_reduce_kernel(DedupParams p) {
         for (int r = 0; r < p.R; ++r) {
             const int32_t d = s_d[r];
             if (d < 0) continue;  // uniform
-            if (threadIdx.x < p.K) {
+            if (threadIdx.x < 32) {  // warp 0 compacts the row's local slots (K <= 32)
                 const int k = threadIdx.x;
-                const bool here = p.dd_topk_idx[(int64_t)d * p.K + k] >= 0;
-                s_row[k] = here ? checked(__ldg(p.dst_row + g * p.K + k), p.m_max, p.err) : -1;
-                s_w[k] = p.dd_topk_w[(int64_t)d * p.K + k];
+                int32_t row = -1;
+                if (k < p.K && p.dd_topk_idx[(int64_t)d * p.K + k] >= 0)
+                    row = checked(__ldg(p.dst_row + g * p.K + k), p.m_max, p.err);
+                const unsigned here = __ballot_sync(FULL, row >= 0);
+                if (row >= 0) {
+                    const int pos = __popc(here & ((1u << k) - 1u));
+                    s_row[pos] = row;
+                    s_w[pos] = p.dd_topk_w[(int64_t)d * p.K + k];
+                }
+                if (k == 0) s_nl = __popc(here);
             }
             __syncthreads();
+            const int nl = s_nl;
             for (int v = threadIdx.x; v < nvec; v += kThreads) {
                 float acc[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
-                for (int k = 0; k < p.K; ++k) {
-                    const int32_t row = s_row[k];
-                    if (row < 0) continue;
-                    const float w = s_w[k];
-                    if (p.y_scale == nullptr) {
-                        const u32x8 q = ld256_stream(p.y + (size_t)row * p.H * 2 + (size_t)v * 32);
+                // up to kReduceBatch gathers in flight per thread; the fma chain
+                // still runs over the slots in ascending k
+                for (int i0 = 0; i0 < nl; i0 += kReduceBatch) {
+                    if constexpr (!FP8) {
+                        u32x8 q[kReduceBatch];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            acc[2 * j] = __fmaf_rn(w, bf16lo(q.v[j]), acc[2 * j]);
-                            acc[2 * j + 1] = __fmaf_rn(w, bf16hi(q.v[j]), acc[2 * j + 1]);
+                        for (int i = 0; i < kReduceBatch; ++i)
+                            if (i0 + i < nl) q[i] = ld256_stream(p.y + (size_t)s_row[i0 + i] * p.H * 2 + (size_t)v * 32);
+#pragma unroll
+                        for (int i = 0; i < kReduceBatch; ++i) {
+                            if (i0 + i >= nl) break;
+                            const float w = s_w[i0 + i];
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                acc[2 * j] = __fmaf_rn(w, bf16lo(q[i].v[j]), acc[2 * j]);
+                                acc[2 * j + 1] = __fmaf_rn(w, bf16hi(q[i].v[j]), acc[2 * j + 1]);
+                            }
                         }
                     } else {
-                        const uint4 q = __ldcs(reinterpret_cast<const uint4*>(p.y + (size_t)row * p.H) + v);
-                        const float sc = __ldg(p.y_scale + (size_t)row * nb + v / 8);
-                        const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+                        uint4 q[kReduceBatch];
+                        float sc[kReduceBatch];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float2 a = unpack_e4m3x2(u[j] & 0xffffu);
-                            const float2 b = unpack_e4m3x2(u[j] >> 16);
-                            acc[4 * j + 0] = __fmaf_rn(w, __fmul_rn(a.x, sc), acc[4 * j + 0]);
-                            acc[4 * j + 1] = __fmaf_rn(w, __fmul_rn(a.y, sc), acc[4 * j + 1]);
-                            acc[4 * j + 2] = __fmaf_rn(w, __fmul_rn(b.x, sc), acc[4 * j + 2]);
-                            acc[4 * j + 3] = __fmaf_rn(w, __fmul_rn(b.y, sc), acc[4 * j + 3]);
+                        for (int i = 0; i < kReduceBatch; ++i) {
+                            if (i0 + i < nl) {
+                                const int32_t row = s_row[i0 + i];
+                                q[i] = __ldcs(reinterpret_cast<const uint4*>(p.y + (size_t)row * p.H) + v);
+                                sc[i] = __ldg(p.y_scale + (size_t)row * nb + v / 8);
+                            }
+                        }
+#pragma unroll
+                        for (int i = 0; i < kReduceBatch; ++i) {
+                            if (i0 + i >= nl) break;
+                            const float w = s_w[i0 + i];
+                            const uint32_t u[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const float2 a = unpack_e4m3x2(u[j] & 0xffffu);
+                                const float2 b = unpack_e4m3x2(u[j] >> 16);
+                                acc[4 * j + 0] = __fmaf_rn(w, __fmul_rn(a.x, sc[i]), acc[4 * j + 0]);
+                                acc[4 * j + 1] = __fmaf_rn(w, __fmul_rn(a.y, sc[i]), acc[4 * j + 1]);
+                                acc[4 * j + 2] = __fmaf_rn(w, __fmul_rn(b.x, sc[i]), acc[4 * j + 2]);
+                                acc[4 * j + 3] = __fmaf_rn(w, __fmul_rn(b.y, sc[i]), acc[4 * j + 3]);
+                            }
                         }
                     }
                 }
@@ -398,7 +429,8 @@ cudaError_t launch_local_reduce(const ep_buffer& b, int T, const void* y, const 
     p.y = static_cast<const uint8_t*>(y);
     p.y_scale = y_scale;
     if (p.N == 0) return cudaSuccess;
-    return launch_tokens(local_reduce_kernel, kThreads, b, p, st);
+    if (y_scale != nullptr) return launch_tokens(local_reduce_kernel<true>, kThreads, b, p, st);
+    return launch_tokens(local_reduce_kernel<false>, kThreads, b, p, st);
 }
 
 cudaError_t launch_combine_dedup(const ep_buffer& b, int T, void* out, cudaStream_t st) {
