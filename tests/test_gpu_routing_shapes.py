@@ -1,10 +1,13 @@
 """Routing + layout from logits on shapes the five workloads do not reach, so
 every branch of the routing kernel runs against the oracle:
-- experts per lane (EPL = E/32) of 3, 4, 16 and 32;
-- groups spanning several lanes, one lane, or not aligned to lanes;
-- more than 8 groups (the shuffle ranking) and at most 8 (the all-pairs ranking);
-- K = 32 (one token per finishing group), K not dividing 32, plain softmax
-  over 256 and 1024 experts, and the slot mask.
+- experts per lane (EPL: E/32 rounded up to a power of two) of 1, 2, 4, 8, 16
+  and 32, with lanes past E left empty;
+- groups spanning several lanes, one lane, or not aligned to lanes (the
+  generic group path);
+- more than 8 groups (the shuffle ranking, at EPL 8 and 16) and at most 8
+  (the all-pairs ranking);
+- K = 32 (one token per finishing group), K = 16, K not dividing 32, plain
+  softmax over 256 and 1024 experts, and the slot mask.
 Tolerances and near-tie handling are those of the workload parity tests."""
 import numpy as np
 import pytest
@@ -20,11 +23,15 @@ S, R2 = wl.ROUTE_SOFTMAX, wl.ROUTE_SOFTMAX_RENORM
 G = wl.ROUTE_GROUP_SIGMOID
 SHAPES = [
     wl.Workload("g32", R=2, T=50, H=128, E=256, K=8, G=32, KG=8, route=G),  # one lane per group, G > 8
-    wl.Workload("g3_unaligned", R=2, T=50, H=128, E=96, K=5, G=3, KG=2, route=G),  # EPL 3: groups split lanes
+    wl.Workload("g3_e96", R=2, T=50, H=128, E=96, K=5, G=3, KG=2, route=G),  # EPL 4, 24 of 32 lanes used
     wl.Workload("g16_e512", R=4, T=40, H=128, E=512, K=8, G=16, KG=4, route=G),  # EPL 16, 2 lanes per group
     wl.Workload("g4_e128", R=4, T=40, H=128, E=128, K=6, G=4, KG=2, route=G, mask_frac=0.2),  # EPL 4, G < 8
     wl.Workload("softmax_e1024_k32", R=4, T=24, H=128, E=1024, K=32, route=S),  # EPL 32, K = 32
     wl.Workload("softmax_e256", R=2, T=64, H=256, E=256, K=8, route=S),  # plain softmax z over 256
+    wl.Workload("g3_e300_generic", R=4, T=30, H=128, E=300, K=5, G=3, KG=2, route=G),  # EPL 16: groups of 100 split lanes
+    wl.Workload("g4_e64", R=2, T=51, H=128, E=64, K=6, G=4, KG=2, route=G),  # EPL 2, 8 lanes per group
+    wl.Workload("g16_e256", R=2, T=41, H=128, E=256, K=8, G=16, KG=4, route=G),  # EPL 8, G > 8, 2 lanes per group
+    wl.Workload("softmax_e128_k16", R=4, T=27, H=128, E=128, K=16, route=S),  # EPL 4, K = 16
     wl.Workload("renorm_e64_k3", R=4, T=33, H=128, E=64, K=3, route=R2, mask_frac=0.1),
     # limits: 32 ranks (a full 32-bit rank mask), the largest hidden size (dispatch with 8
     # vectors per thread, combine looping 4096 vectors), bf16 and FP8
