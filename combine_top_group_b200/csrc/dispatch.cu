@@ -28,6 +28,8 @@
 // memory over NVLink on a multi-GPU node).
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -210,13 +212,12 @@ cudaError_t launch_rows(void (*kernel)(DispatchParams, Recv), int threads, int s
 }
 
 // Threads per CTA, a multiple of 32 and at most 512, and VPT 16-channel
-// vectors per thread: one vector per thread for bf16 rows, two for FP8 rows
-// (the cast gives each thread enough work to hide the load; measured on B200,
-// FP8 dispatch 1569 -> 1522 us on the large shape, 174.5 -> 168.4 us on skewed;
-// bf16 prefill is fastest at one).
-void shape_of(int H, bool fp8, int* threads, int* vpt) {
+// vectors per thread, for a target of `per` vectors per thread: one for bf16
+// rows, two for FP8 rows (the cast gives each thread enough work to hide the
+// load; measured on B200, FP8 dispatch 1569 -> 1522 us on the large shape,
+// 174.5 -> 168.4 us on skewed; bf16 prefill is fastest at one).
+void shape_of(int H, int per, int* threads, int* vpt) {
     const int nv = H / 16;
-    const int per = fp8 ? 2 : 1;
     int t = (nv + per - 1) / per;
     t = t < 512 ? t : 512;
     t = (t + 31) / 32 * 32;
@@ -224,21 +225,72 @@ void shape_of(int H, bool fp8, int* threads, int* vpt) {
     *vpt = (nv + t - 1) / t;
 }
 
+// Resident CTAs per SM of a kernel at a block size (queried once per pair).
+cudaError_t per_sm_of(const void* fn, int threads, int* per_sm) {
+    static std::mutex mu;
+    static const void* fns[64] = {};
+    static int thr[64] = {}, val[64] = {};
+    static int n = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; ++i)
+        if (fns[i] == fn && thr[i] == threads) {
+            *per_sm = val[i];
+            return cudaSuccess;
+        }
+    int v = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, fn, threads, 0);
+    if (e != cudaSuccess) return e;
+    if (v < 1) v = 1;
+    if (n < 64) {
+        fns[n] = fn;
+        thr[n] = threads;
+        val[n] = v;
+        ++n;
+    }
+    *per_sm = v;
+    return cudaSuccess;
+}
+
+template <class Recv>
+void (*fp8_kernel_of(int vpt))(DispatchParams, Recv) {
+    if (vpt <= 1) return dispatch_fp8_kernel<1, Recv>;
+    if (vpt <= 2) return dispatch_fp8_kernel<2, Recv>;
+    if (vpt <= 4) return dispatch_fp8_kernel<4, Recv>;
+    return dispatch_fp8_kernel<8, Recv>;
+}
+
 template <class Recv>
 cudaError_t launch_any(const DispatchParams& p, const Recv& rv, bool fp8, int sm_cap, int full_sms,
                        cudaStream_t st) {
     int threads, vpt;
-    shape_of(p.H, fp8, &threads, &vpt);
+    shape_of(p.H, fp8 ? 2 : 1, &threads, &vpt);
     if (!fp8) {
         if (vpt <= 1) return launch_rows(dispatch_bf16_kernel<1, Recv>, threads, sm_cap, full_sms, p, rv, st);
         if (vpt <= 2) return launch_rows(dispatch_bf16_kernel<2, Recv>, threads, sm_cap, full_sms, p, rv, st);
         if (vpt <= 4) return launch_rows(dispatch_bf16_kernel<4, Recv>, threads, sm_cap, full_sms, p, rv, st);
         return launch_rows(dispatch_bf16_kernel<8, Recv>, threads, sm_cap, full_sms, p, rv, st);
     }
-    if (vpt <= 1) return launch_rows(dispatch_fp8_kernel<1, Recv>, threads, sm_cap, full_sms, p, rv, st);
-    if (vpt <= 2) return launch_rows(dispatch_fp8_kernel<2, Recv>, threads, sm_cap, full_sms, p, rv, st);
-    if (vpt <= 4) return launch_rows(dispatch_fp8_kernel<4, Recv>, threads, sm_cap, full_sms, p, rv, st);
-    return launch_rows(dispatch_fp8_kernel<8, Recv>, threads, sm_cap, full_sms, p, rv, st);
+    auto kern = fp8_kernel_of<Recv>(vpt);
+    if (sm_cap == full_sms) {
+        // A batch a little over one wave of CTAs (decode: 1024 tokens against
+        // 888 resident CTAs of 224 threads) would leave a short second wave
+        // running alone. Half as many threads with twice the vectors each fit
+        // it in one wave when they can.
+        int per_sm = 0;
+        cudaError_t e = per_sm_of((const void*)kern, threads, &per_sm);
+        if (e != cudaSuccess) return e;
+        const int64_t wave = (int64_t)per_sm * full_sms;
+        if (p.N > wave && p.N <= 2 * wave) {
+            int t4, v4;
+            shape_of(p.H, 4, &t4, &v4);
+            auto k4 = fp8_kernel_of<Recv>(v4);
+            int per4 = 0;
+            e = per_sm_of((const void*)k4, t4, &per4);
+            if (e != cudaSuccess) return e;
+            if (p.N <= (int64_t)per4 * full_sms) return launch_rows(k4, t4, sm_cap, full_sms, p, rv, st);
+        }
+    }
+    return launch_rows(kern, threads, sm_cap, full_sms, p, rv, st);
 }
 
 DispatchParams params_of(const ep_buffer& b, int64_t N, const void* x) {
