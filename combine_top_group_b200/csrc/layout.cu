@@ -183,9 +183,7 @@ __device__ __forceinline__ uint32_t kept_groups(const LayoutParams& p, const uin
             }
             lead = lane < p.G;
         }
-        uint32_t kept = 0u;
-        for (uint32_t m = __ballot_sync(FULL, lead && rk < p.KG); m; m &= m - 1)
-            kept |= 1u << __shfl_sync(FULL, gq, __ffs(m) - 1);
+        const uint32_t kept = __reduce_or_sync(FULL, (lead && rk < p.KG) ? 1u << gq : 0u);  // gq < G <= 32
         bool certain = true;
         if (p.KG < p.G) {
             // fp32 sigmoid error <= 3*2^-23 (expf <= 2 ulp, add and rcp 0.5 ulp each),
