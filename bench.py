@@ -100,32 +100,70 @@ def oracle_step(ws: wl.Workload, x, logits):
     return dt, metrics.layout_bytes(ws) + metrics.dispatch_bytes(ws, M) + metrics.combine_bytes(ws, M)
 
 
+def host_cpu() -> dict:
+    """The host's CPU model and logical core count."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu": model, "nproc": os.cpu_count()}
+
+
+class OneCore:
+    """Pins this process to one core of its allowed set while the oracle is
+    timed (single-threaded C), then restores the previous set."""
+
+    def __enter__(self):
+        self.prev = None
+        if hasattr(os, "sched_getaffinity"):
+            try:
+                self.prev = os.sched_getaffinity(0)
+                os.sched_setaffinity(0, {min(self.prev)})
+            except OSError:
+                self.prev = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.prev is not None:
+            os.sched_setaffinity(0, self.prev)
+        return False
+
+
 def cpu_baseline(w: wl.Workload) -> dict:
-    """The oracle on the host, repeated over the sample until CPU_BASELINE_MIN_S
-    of work has been timed."""
+    """The oracle on the host, pinned to one core, repeated over the sample
+    until CPU_BASELINE_MIN_S of work has been timed."""
     ws, x, logits = oracle_sample(w)
     tot_t, tot_b, reps = 0.0, 0, 0
-    while tot_t < CPU_BASELINE_MIN_S:
-        dt, nb = oracle_step(ws, x, logits)
-        tot_t += dt
-        tot_b += nb
-        reps += 1
+    with OneCore():
+        while tot_t < CPU_BASELINE_MIN_S:
+            dt, nb = oracle_step(ws, x, logits)
+            tot_t += dt
+            tot_b += nb
+            reps += 1
     return {"value": tot_b / tot_t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"{reps} passes of the whole path (route, layout, dispatch, identity expert, combine) "
-                      f"over {ws.R}x{ws.T} tokens of the same shape; {tot_t:.1f} s single-threaded C"}
+                      f"over {ws.R}x{ws.T} tokens of the same shape; {tot_t:.1f} s single-threaded C, "
+                      f"pinned to one core",
+            "host": host_cpu()}
 
 
 def run_reference(args, w: wl.Workload, rank: int, world: int):
     if rank != 0:
         return
     ws, x, logits = oracle_sample(w)
-    for _ in range(args.warmup):
-        oracle_step(ws, x, logits)
     tot_t, tot_b = 0.0, 0
-    for _ in range(args.steps):
-        dt, nb = oracle_step(ws, x, logits)
-        tot_t += dt
-        tot_b += nb
+    with OneCore():
+        for _ in range(args.warmup):
+            oracle_step(ws, x, logits)
+        for _ in range(args.steps):
+            dt, nb = oracle_step(ws, x, logits)
+            tot_t += dt
+            tot_b += nb
     value = tot_b / tot_t / 1e9
     line = {
         "impl": "reference", "metric": "routing+layout+dispatch+combine achieved HBM GB/s (algorithmic bytes / time)",
@@ -135,7 +173,8 @@ def run_reference(args, w: wl.Workload, rank: int, world: int):
         "config": workload_desc(w),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": f"each step: the whole path over {ws.R}x{ws.T} tokens of the same shape "
-                                   f"(single-threaded C)"},
+                                   f"(single-threaded C, pinned to one core)",
+                         "host": host_cpu()},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

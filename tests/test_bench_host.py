@@ -83,6 +83,17 @@ def test_reference_arm_json_line():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "GB/s"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["cpu_baseline"]["cores"] == 1 and line["cpu_baseline"]["host"]["nproc"] >= 1
+
+
+def test_one_core_pin_is_restored():
+    import bench
+    if not hasattr(os, "sched_getaffinity"):
+        return
+    before = os.sched_getaffinity(0)
+    with bench.OneCore():
+        assert len(os.sched_getaffinity(0)) == 1
+    assert os.sched_getaffinity(0) == before
 
 
 def test_reference_arm_other_ranks_exit_quietly():
