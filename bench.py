@@ -89,12 +89,13 @@ def oracle_sample(w: wl.Workload, seed: int = 0):
     return ws, wl.make_x(ws, seed), wl.make_logits(ws, seed)
 
 
-def oracle_step(ws: wl.Workload, x, logits):
+def oracle_step(ws: wl.Workload, x, logits, phases: dict | None = None):
     """One oracle pass (route, layout, dispatch, identity expert, combine) over
-    the sample. Returns (seconds, algorithmic bytes)."""
+    the sample. Returns (seconds, algorithmic bytes); `phases` accumulates the
+    seconds of each phase."""
     import oracle  # test infrastructure: only the CPU legs of the bench run it
     t0 = time.perf_counter()
-    res = oracle.run_path(x, logits, ws)
+    res = oracle.run_path(x, logits, ws, timings=phases)
     dt = time.perf_counter() - t0
     M = res["M"]
     return dt, metrics.layout_bytes(ws) + metrics.dispatch_bytes(ws, M) + metrics.combine_bytes(ws, M)
@@ -139,9 +140,10 @@ def cpu_baseline(w: wl.Workload) -> dict:
     until CPU_BASELINE_MIN_S of work has been timed."""
     ws, x, logits = oracle_sample(w)
     tot_t, tot_b, reps = 0.0, 0, 0
+    phases: dict = {}
     with OneCore():
         while tot_t < CPU_BASELINE_MIN_S:
-            dt, nb = oracle_step(ws, x, logits)
+            dt, nb = oracle_step(ws, x, logits, phases)
             tot_t += dt
             tot_b += nb
             reps += 1
@@ -149,6 +151,7 @@ def cpu_baseline(w: wl.Workload) -> dict:
             "sample": f"{reps} passes of the whole path (route, layout, dispatch, identity expert, combine) "
                       f"over {ws.R}x{ws.T} tokens of the same shape; {tot_t:.1f} s single-threaded C, "
                       f"pinned to one core",
+            "phase_ms_per_pass": {k: v / reps * 1e3 for k, v in phases.items()},
             "host": host_cpu()}
 
 
@@ -157,11 +160,12 @@ def run_reference(args, w: wl.Workload, rank: int, world: int):
         return
     ws, x, logits = oracle_sample(w)
     tot_t, tot_b = 0.0, 0
+    phases: dict = {}
     with OneCore():
         for _ in range(args.warmup):
             oracle_step(ws, x, logits)
         for _ in range(args.steps):
-            dt, nb = oracle_step(ws, x, logits)
+            dt, nb = oracle_step(ws, x, logits, phases)
             tot_t += dt
             tot_b += nb
     value = tot_b / tot_t / 1e9
@@ -174,6 +178,7 @@ def run_reference(args, w: wl.Workload, rank: int, world: int):
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": f"each step: the whole path over {ws.R}x{ws.T} tokens of the same shape "
                                    f"(single-threaded C, pinned to one core)",
+                         "phase_ms_per_pass": {k: v / args.steps * 1e3 for k, v in phases.items()},
                          "host": host_cpu()},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

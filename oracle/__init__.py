@@ -13,6 +13,8 @@ import ctypes
 import os
 import subprocess
 
+import time
+
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -311,26 +313,41 @@ def combine(y: np.ndarray, y_scale: np.ndarray | None, dst_row: np.ndarray, topk
 
 
 def run_path(x: np.ndarray, logits: np.ndarray | None, w, topk_idx=None, topk_w=None,
-             combine_tokens=None, fp8_combine_fused: bool = False):
+             combine_tokens=None, fp8_combine_fused: bool = False, timings: dict | None = None):
     """Whole path on the CPU for workload w: routing (or the given top-k),
-    mask, layout, dispatch, identity expert and combine. Returns a dict."""
+    mask, layout, dispatch, identity expert and combine. Returns a dict.
+    `timings`, if given, receives the seconds each phase took (keys route,
+    layout, dispatch, expert, combine)."""
+    clock = [time.perf_counter()]
+
+    def lap(name):
+        now = time.perf_counter()
+        if timings is not None:
+            timings[name] = timings.get(name, 0.0) + now - clock[0]
+        clock[0] = now
+
     if topk_idx is None:
         idx, tw, margin = route(logits, w.K, w.route, w.G, w.KG)
         if w.mask_frac:
             apply_mask(idx, tw, w.mask_seed, w.mask_frac)
     else:
         idx, tw, margin = np.array(topk_idx, dtype=np.int32), np.array(topk_w, dtype=np.float32), None
+    lap("route")
     lay = layout(idx, w.R, w.T, w.E)
     M = int(lay["expert_off"][-1])
     if getattr(w, "low_latency", False):
         # fixed (expert, source rank) regions of T_max rows; the counts stay the same
         lay["dst_row"], _ = layout_ll(idx, w.R, w.T, w.T, w.E)
         M = w.E * w.R * w.T
+    lap("layout")
     recv_x, recv_scale, recv_src, recv_w = dispatch(x, lay["dst_row"], tw, M, w.fp8)
+    lap("dispatch")
     if w.fp8 and not fp8_combine_fused:
         y, ys = identity_expert_fp8(recv_x, recv_scale), None
     else:
         y, ys = recv_x, recv_scale
+    lap("expert")
     out = combine(y, ys, lay["dst_row"], tw, combine_tokens)
+    lap("combine")
     return dict(topk_idx=idx, topk_w=tw, margin=margin, M=M, recv_x=recv_x,
                 recv_scale=recv_scale, recv_src=recv_src, recv_w=recv_w, y=y, out=out, **lay)
