@@ -107,10 +107,37 @@ __device__ __forceinline__ void stage_rows(const DispatchParams& p, const Recv& 
     }
 }
 
+// The order in which the CTA writes the token's K rows: ascending
+// (destination rank, row), masked rows last; s_ord[i] = the i-th slot. CTAs
+// in flight hold consecutive tokens, whose rows for one expert are adjacent,
+// so in this order their writes meet in fewer places at a time (measured on
+// B200: prefill dispatch 687 -> 678 us). Threads t < K, after s_row / s_rank
+// are visible.
+template <class Recv>
+__device__ __forceinline__ void order_rows(int K, const int32_t* s_row, const int32_t* s_rank, int32_t* s_ord) {
+    const int t = threadIdx.x;
+    if (t < K) {
+        auto key = [&](int q) -> uint64_t {
+            const int32_t r = s_row[q];
+            if (r < 0) return ~0ull;
+            const uint64_t d = Recv::kPeer ? (uint64_t)(uint32_t)s_rank[q] : 0ull;
+            return (d << 32) | (uint32_t)r;
+        };
+        const uint64_t me = key(t);
+        int pos = 0;
+        for (int q = 0; q < K; ++q) {
+            const uint64_t o = key(q);
+            pos += (o < me || (o == me && q < t)) ? 1 : 0;
+        }
+        s_ord[pos] = t;
+    }
+}
+
 template <int VPT, class Recv>
 __global__ void __launch_bounds__(512) dispatch_bf16_kernel(DispatchParams p, Recv rv) {
     __shared__ int32_t s_row[kMaxK];
     __shared__ int32_t s_rank[Recv::kPeer ? kMaxK : 1];
+    __shared__ int32_t s_ord[kMaxK];
     const int nv = p.H / 16;  // 32-byte vectors per bf16 row
     const size_t rb = (size_t)p.H * 2;
     for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {
@@ -122,7 +149,10 @@ __global__ void __launch_bounds__(512) dispatch_bf16_kernel(DispatchParams p, Re
             if (c < nv) v[j] = ld256_stream(p.x + g * rb + (size_t)c * 32);
         }
         __syncthreads();
-        for (int k = 0; k < p.K; ++k) {
+        order_rows<Recv>(p.K, s_row, s_rank, s_ord);
+        __syncthreads();
+        for (int i = 0; i < p.K; ++i) {
+            const int k = s_ord[i];
             const int32_t r = s_row[k];
             if (r < 0) continue;
             uint8_t* dst = rv.x_of(Recv::kPeer ? s_rank[k] : 0) + (size_t)r * rb;
@@ -140,6 +170,7 @@ template <int VPT, class Recv>
 __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchParams p, Recv rv) {
     __shared__ int32_t s_row[kMaxK];
     __shared__ int32_t s_rank[Recv::kPeer ? kMaxK : 1];
+    __shared__ int32_t s_ord[kMaxK];
     const int nv = p.H / 16;  // 16-channel vectors per row: 32 B in, 16 B out
     const int nb = p.H / 128;
     const size_t rb_in = (size_t)p.H * 2;
@@ -175,7 +206,10 @@ __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchParams p, Rec
             sc[j] = __fdiv_rn(amax, 448.0f);
         }
         __syncthreads();
-        for (int k = 0; k < p.K; ++k) {
+        order_rows<Recv>(p.K, s_row, s_rank, s_ord);
+        __syncthreads();
+        for (int i = 0; i < p.K; ++i) {
+            const int k = s_ord[i];
             const int32_t r = s_row[k];
             if (r < 0) continue;
             const int d = Recv::kPeer ? s_rank[k] : 0;
