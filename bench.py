@@ -38,6 +38,8 @@ from combine_top_group_b200 import metrics  # noqa: E402
 from combine_top_group_b200 import workloads as wl  # noqa: E402
 
 ORACLE_SAMPLE_T = 1024  # tokens per rank in the CPU oracle's bounded sample
+# One metric string for both arms, so their lines compare directly.
+METRIC = "routing+layout+dispatch+combine achieved HBM GB/s (algorithmic bytes / time)"
 CPU_BASELINE_MIN_S = 10.0  # seconds of oracle work behind cpu_baseline
 
 
@@ -170,11 +172,14 @@ def run_reference(args, w: wl.Workload, rank: int, world: int):
             tot_b += nb
     value = tot_b / tot_t / 1e9
     line = {
-        "impl": "reference", "metric": "routing+layout+dispatch+combine achieved HBM GB/s (algorithmic bytes / time)",
+        "impl": "reference", "metric": METRIC,
         "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if not w.fp8 else "fp8_e4m3", "data": "synthetic",
-        "config": workload_desc(w),
+        "config": {**workload_desc(w), "parallelism": "1 host core", "combine_input": "bf16",
+                   "sample_tokens_per_rank": ws.T,
+                   "sample": f"each step runs the whole path over {ws.R}x{ws.T} of the workload's "
+                             f"{w.R}x{w.T} tokens"},
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": f"each step: the whole path over {ws.R}x{ws.T} tokens of the same shape "
                                    f"(single-threaded C, pinned to one core)",
@@ -275,7 +280,7 @@ def run_ours(args, w: wl.Workload, rank: int, world: int, local_rank: int):
     achieved = k_bytes / k_time / 1e9
     traffic = metrics.stored_traffic(kern, w.name)
     out = {
-        "metric": "routing+layout+dispatch+combine achieved HBM GB/s (algorithmic bytes / device time)",
+        "metric": METRIC,
         "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": t_total / K * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp8_e4m3" if w.fp8 else "bf16", "data": "synthetic",

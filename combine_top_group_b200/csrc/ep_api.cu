@@ -343,6 +343,24 @@ static ep_status_t layout_args(const ep_buffer_t* b, int T, const float* d_logit
     return EP_OK;
 }
 
+// True if [p, p + 1) lies inside the n bytes at base.
+static bool points_into(const void* p, const void* base, size_t n) {
+    const uintptr_t a = (uintptr_t)p, lo = (uintptr_t)base;
+    return base != nullptr && a >= lo && a - lo < n;
+}
+
+// An FP8 buffer's e4m3 rows hold 1 byte per channel. Read as bf16 y (no
+// scale given), rows of 2*H bytes would run past the end of the array, so
+// that call is refused.
+static ep_status_t check_y_not_e4m3_rows(const ep_buffer_t* b, const void* d_y, const float* d_y_scale) {
+    if (!(b->cfg.flags & EP_FLAG_FP8) || d_y_scale) return EP_OK;
+    const size_t H = (size_t)b->cfg.hidden;
+    if (points_into(d_y, b->recv_x, (size_t)b->m_max * H) || points_into(d_y, b->dd_x, (size_t)b->d_max * H))
+        return fail(EP_ERR_INVALID, "d_y points into the buffer's e4m3 rows: pass d_y_scale (fused dequant) "
+                                    "or a bf16 expert output");
+    return EP_OK;
+}
+
 static ep_status_t check_single(const ep_buffer_t* b) {
     if (ep_status_t st = check_buf(b)) return st;
     if (b->cfg.flags & EP_FLAG_SHARD)
@@ -379,6 +397,7 @@ ep_status_t ep_combine(ep_buffer_t* b, int T, const void* d_y, const float* d_y_
     if ((uintptr_t)d_y % 32 != 0 || (uintptr_t)d_out % 32 != 0)
         return fail(EP_ERR_INVALID, "d_y and d_out must be 32-byte aligned");
     if (d_y_scale && (uintptr_t)d_y_scale % 4 != 0) return fail(EP_ERR_INVALID, "d_y_scale must be 4-byte aligned");
+    if (ep_status_t st = check_y_not_e4m3_rows(b, d_y, d_y_scale)) return st;
     cudaError_t e = ep::launch_combine(*b, T, d_y, d_y_scale, d_out, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "combine launch");
     return ok();
@@ -430,6 +449,7 @@ ep_status_t ep_local_reduce(ep_buffer_t* b, int T, const void* d_y, const float*
     if (T > 0 && !d_y) return fail(EP_ERR_INVALID, "d_y is NULL");
     if ((uintptr_t)d_y % 32 != 0) return fail(EP_ERR_INVALID, "d_y must be 32-byte aligned");
     if (d_y_scale && (uintptr_t)d_y_scale % 4 != 0) return fail(EP_ERR_INVALID, "d_y_scale must be 4-byte aligned");
+    if (ep_status_t st = check_y_not_e4m3_rows(b, d_y, d_y_scale)) return st;
     cudaError_t e = ep::launch_local_reduce(*b, T, d_y, d_y_scale, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "local_reduce launch");
     return ok();

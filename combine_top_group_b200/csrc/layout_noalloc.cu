@@ -37,27 +37,65 @@ static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchInts];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-int32_t* g_scratch_ptr[kMaxDevices] = {};  // device address of g_noalloc_scratch, per device
+// Device address of g_noalloc_scratch per device, and the id of the context
+// it was looked up in. A context created anew (cudaDeviceReset) loads the
+// module again, and the array may then sit at another address.
+int32_t* g_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
 
 ep_status_t fail(ep_status_t st, const char* msg) {
     ep::set_last_error(msg);
     return st;
 }
 
-// Once per device, with that device current: the device address of the
-// scratch array. In host code the symbol itself is only a host-side stand-in,
-// so a kernel must never be given &g_noalloc_scratch directly.
+// The driver's unique id of the current context (cuCtxGetCurrent +
+// cuCtxGetId, reached through the runtime's driver entry points, so the
+// library needs no link to libcuda). Ids are never reused within a process.
+cudaError_t current_context_id(unsigned long long* id) {
+    using get_current_t = int (*)(void**);
+    using get_id_t = int (*)(void*, unsigned long long*);
+    static get_current_t get_current = nullptr;
+    static get_id_t get_id = nullptr;
+    if (!get_current || !get_id) {
+        void* f1 = nullptr;
+        void* f2 = nullptr;
+        cudaDriverEntryPointQueryResult q1, q2;
+        cudaError_t e = cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f1, 12000, cudaEnableDefault, &q1);
+        if (e == cudaSuccess)
+            e = cudaGetDriverEntryPointByVersion("cuCtxGetId", &f2, 12000, cudaEnableDefault, &q2);
+        if (e != cudaSuccess) return e;
+        if (q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess || !f1 || !f2)
+            return cudaErrorSymbolNotFound;
+        get_current = reinterpret_cast<get_current_t>(f1);
+        get_id = reinterpret_cast<get_id_t>(f2);
+    }
+    void* ctx = nullptr;
+    if (get_current(&ctx) != 0 || !ctx) return cudaErrorDeviceUninitialized;
+    if (get_id(ctx, id) != 0) return cudaErrorDeviceUninitialized;
+    return cudaSuccess;
+}
+
+// With the device current: the device address of the scratch array, looked
+// up once per device and context. In host code the symbol itself is only a
+// host-side stand-in, so a kernel must never be given &g_noalloc_scratch
+// directly.
 cudaError_t scratch_for_current_device(int32_t** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    unsigned long long ctx = 0;
+    // fails when this host thread has no current context yet
+    const bool have_ctx = current_context_id(&ctx) == cudaSuccess;
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
+    if (!have_ctx || !g_scratch_ptr[dev] || g_scratch_ctx[dev] != ctx) {
         void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // makes the device's primary context current
+        if (e != cudaSuccess) return e;
+        e = current_context_id(&ctx);
         if (e != cudaSuccess) return e;
         g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+        g_scratch_ctx[dev] = ctx;
     }
     *out = g_scratch_ptr[dev];
     return cudaSuccess;
@@ -72,6 +110,9 @@ extern "C" ep_status_t ep_get_layout_noalloc(const ep_config_t* cfg, int T, cons
     size_t ignored = 0;
     ep_status_t st = ep_buffer_workspace_bytes(cfg, &ignored);  // validates the config
     if (st != EP_OK) return st;
+    if (cfg->flags & (EP_FLAG_DEDUP | EP_FLAG_SHARD))
+        return fail(EP_ERR_UNSUPPORTED, "EP_FLAG_DEDUP and EP_FLAG_SHARD layouts need a buffer: use ep_get_layout "
+                                        "or ep_shard_layout");
     if (!out || !d_error_word) return fail(EP_ERR_INVALID, "out and d_error_word must be non-NULL");
     if (!out->topk_idx || !out->topk_w || !out->is_token_in_rank || !out->num_tokens_per_rank ||
         !out->cnt_src_expert || !out->num_tokens_per_expert || !out->expert_off || !out->rank_off ||

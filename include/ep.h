@@ -212,7 +212,9 @@ ep_status_t ep_dispatch(ep_buffer_t *buf, int T, const void *d_x, void *stream);
  * in the kernel as e4m3 * d_y_scale[row, h/128] (fp32) before the fma.
  * rows >= expert_off[E]. d_out: bf16 [N, H]. d_y and d_out 32-byte aligned.
  * T must equal the T of the last ep_get_layout. A token whose slots are all
- * masked gets +0. Errors: EP_ERR_INVALID. */
+ * masked gets +0. Errors: EP_ERR_INVALID, also when the buffer has
+ * EP_FLAG_FP8, d_y_scale is NULL and d_y points into the buffer's own e4m3
+ * rows (read as bf16 they would run past the end of the array). */
 ep_status_t ep_combine(ep_buffer_t *buf, int T, const void *d_y, const float *d_y_scale,
                        void *d_out, void *stream);
 
@@ -258,7 +260,8 @@ ep_status_t ep_permute(ep_buffer_t *buf, int T, void *stream);
 
 /* Local reduce: partial[d] = bf16( sum over the row's local slots k
  * ascending, fp32 fma, of w * y[dst_row[g][k]] ). y as for ep_combine (bf16,
- * or e4m3 + d_y_scale), 32-byte aligned. */
+ * or e4m3 + d_y_scale), 32-byte aligned. Errors: EP_ERR_INVALID, also for
+ * the buffer's own e4m3 rows (recv_x or dd_x) passed without d_y_scale. */
 ep_status_t ep_local_reduce(ep_buffer_t *buf, int T, const void *d_y, const float *d_y_scale, void *stream);
 
 /* Dedup combine: out[g] = bf16( sum over ranks r ascending, fp32, of
@@ -394,10 +397,15 @@ ep_status_t ep_selftest_wait_timeout(uint32_t *d_words, uint64_t limit_ns, uint3
  *    rejected; a smaller grid only means longer chunks.
  *  - d_error_word: a device uint32 that receives EP_DEVERR_* bits with
  *    atomicOr. The caller zeroes and reads it.
+ *  - cfg: the layout's shape, as for ep_buffer_workspace_bytes. EP_FLAG_FP8
+ *    does not change the layout and is ignored; EP_FLAG_LOW_LATENCY gives the
+ *    low-latency dst_row. EP_FLAG_DEDUP and EP_FLAG_SHARD are refused with
+ *    EP_ERR_UNSUPPORTED: their extra arrays have no place in ep_layout_t.
  *  - Runs on the current device. `stream` must belong to it.
- *  - Set-up: the first call on each device looks up the device address of
- *    the static scratch (cudaGetSymbolAddress). Make that first call before
- *    any stream capture.
+ *  - Set-up: the first call on each device, and the first call after that
+ *    device's context was created anew (after cudaDeviceReset), looks up the
+ *    device address of the static scratch (cudaGetSymbolAddress). Make those
+ *    calls before any stream capture.
  *  - Every call on a device shares the one scratch array and leaves its
  *    contents behind. Each call first zeroes the barrier counters with a
  *    stream-ordered cudaMemsetAsync of 256 bytes (not an allocation). The

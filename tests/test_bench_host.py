@@ -84,6 +84,11 @@ def test_reference_arm_json_line():
     assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "GB/s"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["cpu_baseline"]["cores"] == 1 and line["cpu_baseline"]["host"]["nproc"] >= 1
+    # both arms print the same metric, so their values compare directly
+    import bench
+    assert line["metric"] == bench.METRIC and line["higher_is_better"] is True
+    # the line names the sample it timed
+    assert line["config"]["sample_tokens_per_rank"] == min(wl.WORKLOADS["tiny"].T, bench.ORACLE_SAMPLE_T)
 
 
 def test_one_core_pin_is_restored():

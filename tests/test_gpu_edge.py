@@ -216,6 +216,29 @@ def test_host_errors(cuda):
     assert ei.value.status == ep.EP_ERR_INVALID
 
 
+def test_e4m3_rows_refused_as_bf16_y(cuda):
+    """An FP8 buffer's own e4m3 rows passed as y without scales would be read
+    as bf16 rows of twice the width, past the end of the array: refused on
+    the host. With the scales the same rows are the fused-dequant input."""
+    ep, runner = cuda
+    w = wl.WORKLOADS["decode"]
+    pipe = runner.Pipeline(w, 0, dedup=True)
+    pipe.layout()
+    pipe.dispatch()
+    with pytest.raises(ep.EpError) as ei:
+        ep.ep_combine(pipe.buf, w.T, pipe.recv["recv_x"], None, pipe.out)
+    assert ei.value.status == ep.EP_ERR_INVALID
+    with pytest.raises(ep.EpError) as ei:  # a row inside the array, not just its start
+        ep.ep_combine(pipe.buf, w.T, pipe.recv["recv_x"][64:], None, pipe.out)
+    assert ei.value.status == ep.EP_ERR_INVALID
+    for y in (pipe.recv["recv_x"], pipe.dd["dd_x"]):
+        with pytest.raises(ep.EpError) as ei:
+            ep.ep_local_reduce(pipe.buf, w.T, y, None)
+        assert ei.value.status == ep.EP_ERR_INVALID
+    ep.ep_combine(pipe.buf, w.T, pipe.recv["recv_x"], pipe.recv["recv_scale"], pipe.out)
+    assert pipe.check_errors() == 0
+
+
 def test_guard_bands_and_rows_beyond_M_untouched(cuda):
     """Canary bytes after the workspace and receive rows beyond M stay
     intact after a full step."""

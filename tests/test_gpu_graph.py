@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from combine_top_group_b200 import workloads as wl
-from test_gpu_parity import _check_combine, _combine_expected, _oracle_route, _to_host
+from parity_util import check_combine, combine_expected, oracle_route, to_host
 
 pytestmark = pytest.mark.gpu
 
@@ -63,10 +63,10 @@ def test_graph_replay_matches_eager(cuda, name):
         assert torch.equal(ep.ep_buffer_layout(pipe.buf, w.T)["dst_row"], got_dst)
         assert torch.equal(pipe.out.view(torch.int16), got_out.view(torch.int16))
     # the last replay ran on seed 1: spot-check it against the oracle
-    o_idx, o_w, _ = _oracle_route(w, l1)
+    o_idx, o_w, _ = oracle_route(w, l1)
     tokens = np.unique(np.concatenate([np.arange(0, w.N, max(1, w.N // 64)), [w.N - 1]]))
-    got = _to_host(got_out.index_select(0, torch.from_numpy(tokens).cuda()))
-    _check_combine(got, _combine_expected(w, x1, o_idx, o_w, tokens, "fused" if fused else "bf16"))
+    got = to_host(got_out.index_select(0, torch.from_numpy(tokens).cuda()))
+    check_combine(got, combine_expected(w, x1, o_idx, o_w, tokens, "fused" if fused else "bf16"))
 
 
 def test_graph_replay_emulated_ranks(cuda):

@@ -15,7 +15,7 @@ import torch
 
 import oracle
 from combine_top_group_b200 import workloads as wl
-from test_gpu_parity import _check_combine, _check_routing, _combine_expected, _oracle_route, _to_host
+from parity_util import check_combine, check_routing, combine_expected, oracle_route, to_host
 
 pytestmark = pytest.mark.gpu
 
@@ -55,13 +55,13 @@ def test_routing_shapes(cuda, w):
     x = wl.make_x(w, 7)
     logits = wl.make_logits(w, 7)
     pipe = runner.Pipeline(w, 7, x=x, logits=logits)
-    o_idx, o_w, margin = _oracle_route(w, logits)
+    o_idx, o_w, margin = oracle_route(w, logits)
     pipe.layout()
     assert pipe.check_errors() == 0
-    lay = {k: _to_host(v) for k, v in ep.ep_buffer_layout(pipe.buf, w.T).items()}
-    if _check_routing(w, o_idx, o_w, margin, lay["topk_idx"], lay["topk_w"]):
+    lay = {k: to_host(v) for k, v in ep.ep_buffer_layout(pipe.buf, w.T).items()}
+    if check_routing(w, o_idx, o_w, margin, lay["topk_idx"], lay["topk_w"]):
         pipe.layout(topk_idx=torch.from_numpy(o_idx).cuda(), topk_w=torch.from_numpy(o_w).cuda())
-        lay = {k: _to_host(v) for k, v in ep.ep_buffer_layout(pipe.buf, w.T).items()}
+        lay = {k: to_host(v) for k, v in ep.ep_buffer_layout(pipe.buf, w.T).items()}
     o_lay = oracle.layout(o_idx, w.R, w.T, w.E)
     for key in ("is_token_in_rank", "num_tokens_per_rank", "cnt", "num_tokens_per_expert", "expert_off",
                 "rank_off", "src_off", "dst_row"):
@@ -73,8 +73,8 @@ def test_routing_shapes(cuda, w):
         M = int(o_lay["expert_off"][-1])
         dst = o_lay["dst_row"]
         src = np.repeat(np.arange(w.N), w.K).reshape(w.N, w.K)[dst >= 0][np.argsort(dst[dst >= 0])]
-        g_rows = _to_host(pipe.recv["recv_x"][:M])
-        g_sc = _to_host(pipe.recv["recv_scale"][:M])
+        g_rows = to_host(pipe.recv["recv_x"][:M])
+        g_sc = to_host(pipe.recv["recv_scale"][:M])
         for i, g in enumerate(src):
             q, sc = oracle.quant_fp8_row(x[g])
             assert np.array_equal(g_rows[i], q) and np.array_equal(g_sc[i].view(np.uint32), sc.view(np.uint32))
@@ -83,11 +83,11 @@ def test_routing_shapes(cuda, w):
         M = int(o_lay["expert_off"][-1])
         dst = o_lay["dst_row"]
         src = np.repeat(np.arange(w.N), w.K).reshape(w.N, w.K)[dst >= 0][np.argsort(dst[dst >= 0])]
-        assert np.array_equal(_to_host(pipe.recv["recv_x"][:M]), x[src])
+        assert np.array_equal(to_host(pipe.recv["recv_x"][:M]), x[src])
     pipe.combine(fused=w.fp8)
     assert pipe.check_errors() == 0
     tokens = np.arange(w.N)
-    _check_combine(_to_host(pipe.out), _combine_expected(w, x, o_idx, o_w, tokens, mode))
+    check_combine(to_host(pipe.out), combine_expected(w, x, o_idx, o_w, tokens, mode))
 
 
 def test_group_score_ties_decide_by_lower_id(cuda):
@@ -106,10 +106,10 @@ def test_group_score_ties_decide_by_lower_id(cuda):
     pipe.layout()
     assert pipe.check_errors() == 0
     lay = ep.ep_buffer_layout(pipe.buf, w.T)
-    o_idx, o_w, margin = _oracle_route(w, logits)
+    o_idx, o_w, margin = oracle_route(w, logits)
     assert (margin[:half] == 0).all()  # exact ties on the all-equal tokens
-    assert np.array_equal(_to_host(lay["topk_idx"]), o_idx)
-    g_w = _to_host(lay["topk_w"]).astype(np.float64)
+    assert np.array_equal(to_host(lay["topk_idx"]), o_idx)
+    g_w = to_host(lay["topk_w"]).astype(np.float64)
     assert (np.abs(g_w - o_w) <= 2.0 ** -22 * np.abs(o_w)).all()
     # all-equal tokens keep groups 0..3 only
     assert (o_idx[:half] < 128).all()

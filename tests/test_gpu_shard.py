@@ -14,7 +14,8 @@ import torch
 import oracle
 from combine_top_group_b200 import workloads as wl
 from shard_view import shard_view
-from test_gpu_parity import _check_combine, _check_routing, _combine_expected, _oracle_route, _sample_rows, _to_host
+from parity_util import (check_combine, check_routing, check_rows, combine_expected, oracle_fp8_rows,
+                         oracle_route, to_host)
 
 pytestmark = pytest.mark.gpu
 
@@ -27,7 +28,8 @@ def cuda():
     return ep, shard
 
 
-CASES = [("tiny", 0), ("tiny", 2), ("decode", 1), ("prefill", 0), ("skewed", 2), ("ranks32", 0)]
+CASES = [("tiny", 0), ("tiny", 2), ("decode", 1), ("prefill", 0), ("prefill", 2), ("skewed", 1), ("skewed", 2),
+         ("ranks32", 0)]
 EXTRA = {"ranks32": wl.Workload("ranks32", R=32, T=8, H=128, E=64, K=4, route=wl.ROUTE_SOFTMAX)}
 
 
@@ -44,20 +46,20 @@ def test_shard_parity(cuda, name, seed):
     em = shard.EmulatedRanks(w, xt, lt, out)
 
     # ---- step 1: each rank's routing and rank-local counts
-    o_idx, o_w, margin = _oracle_route(w, logits)
+    o_idx, o_w, margin = oracle_route(w, logits)
     em.layout()
     assert em.check_errors() == 0
-    g_idx = np.concatenate([_to_host(ep.ep_buffer_layout(b, T)["topk_idx"]) for b in em.bufs])
-    g_w = np.concatenate([_to_host(ep.ep_buffer_layout(b, T)["topk_w"]) for b in em.bufs])
-    if _check_routing(w, o_idx, o_w, margin, g_idx, g_w):
+    g_idx = np.concatenate([to_host(ep.ep_buffer_layout(b, T)["topk_idx"]) for b in em.bufs])
+    g_w = np.concatenate([to_host(ep.ep_buffer_layout(b, T)["topk_w"]) for b in em.bufs])
+    if check_routing(w, o_idx, o_w, margin, g_idx, g_w):
         em.layout(topk_idx=torch.from_numpy(o_idx).cuda(), topk_w=torch.from_numpy(o_w).cuda())
     o_lay = oracle.layout(o_idx, R, T, E)
     views = shard_view(o_idx, o_lay, R, T, E)
     for s, b in enumerate(em.bufs):
-        lay = {k: _to_host(v) for k, v in ep.ep_buffer_layout(b, T).items()}
+        lay = {k: to_host(v) for k, v in ep.ep_buffer_layout(b, T).items()}
         assert np.array_equal(lay["is_token_in_rank"], o_lay["is_token_in_rank"][s * T:(s + 1) * T])
         assert np.array_equal(lay["num_tokens_per_rank"][0], o_lay["num_tokens_per_rank"][s])
-        assert np.array_equal(_to_host(em.sh[s]["cnt_row"]), views[s]["cnt_row"])
+        assert np.array_equal(to_host(em.sh[s]["cnt_row"]), views[s]["cnt_row"])
         assert np.array_equal(lay["dst_row"], views[s]["local_rows"])  # rank-local rows before placement
 
     # ---- steps 2-3: exchange, placement on the destination ranks
@@ -65,10 +67,10 @@ def test_shard_parity(cuda, name, seed):
     em.place()
     assert em.check_errors() == 0
     for s in range(R):
-        assert np.array_equal(_to_host(em.sh[s]["dst_rank"]), views[s]["dst_rank"])
-        assert np.array_equal(_to_host(ep.ep_buffer_layout(em.bufs[s], T)["dst_row"]), views[s]["dst_row"])
-        assert np.array_equal(_to_host(em.sh[s]["recv_count"]), views[s]["recv_count"])
-        assert np.array_equal(_to_host(em.sh[s]["recv_off"]), views[s]["recv_off"])
+        assert np.array_equal(to_host(em.sh[s]["dst_rank"]), views[s]["dst_rank"])
+        assert np.array_equal(to_host(ep.ep_buffer_layout(em.bufs[s], T)["dst_row"]), views[s]["dst_row"])
+        assert np.array_equal(to_host(em.sh[s]["recv_count"]), views[s]["recv_count"])
+        assert np.array_equal(to_host(em.sh[s]["recv_off"]), views[s]["recv_off"])
 
     # ---- step 5: dispatch into every rank's receive rows
     em.dispatch()
@@ -76,37 +78,34 @@ def test_shard_parity(cuda, name, seed):
     o_dst, o_eoff, o_roff = o_lay["dst_row"], o_lay["expert_off"], o_lay["rank_off"]
     valid = o_dst >= 0
     o_rw = o_w[valid][np.argsort(o_dst[valid])]
+    if not w.fp8:
+        table = torch.from_numpy(x.view(np.int16)).cuda()  # a fresh copy of the seeded input
+    else:
+        q, sc = oracle_fp8_rows(x)
+        table, stable = torch.from_numpy(q).cuda(), torch.from_numpy(sc).cuda()
     for d in range(R):
         a, b = int(o_roff[d]), int(o_roff[d + 1])
         rv = em.recv[d]
         assert em.received_rows()[d] == b - a
-        assert np.array_equal(_to_host(rv["recv_src"][:b - a]), views[d]["recv_src"])
-        g_rw = _to_host(rv["recv_w"][:b - a]).astype(np.float64)
+        assert np.array_equal(to_host(rv["recv_src"][:b - a]), views[d]["recv_src"])
+        g_rw = to_host(rv["recv_w"][:b - a]).astype(np.float64)
         assert (np.abs(g_rw - o_rw[a:b]) <= 2.0 ** -22 * np.abs(o_rw[a:b])).all()
-        n = b - a
-        pick = np.arange(n) if n * H <= 16 * 2 ** 20 else _sample_rows(n, o_eoff[d * L:(d + 1) * L + 1] - a, 500, seed)
-        g_rows = _to_host(rv["recv_x"].index_select(0, torch.from_numpy(pick).cuda()))
-        src = views[d]["recv_src"][pick]
-        if not w.fp8:
-            assert np.array_equal(g_rows, x[src]), f"rank {d}"
-        else:
-            g_sc = _to_host(rv["recv_scale"].index_select(0, torch.from_numpy(pick).cuda()))
-            for i, g in enumerate(src):
-                q, sc = oracle.quant_fp8_row(x[g])
-                assert np.array_equal(g_rows[i], q) and np.array_equal(g_sc[i].view(np.uint32), sc.view(np.uint32))
+        # every receive row of rank d against its source token's oracle row
+        rows_t = torch.arange(b - a, dtype=torch.int64, device="cuda")
+        src_t = torch.from_numpy(views[d]["recv_src"].astype(np.int64)).cuda()
+        check_rows(rv["recv_x"], rows_t, table, src_t, f"rank {d} rows")
+        if w.fp8:
+            check_rows(rv["recv_scale"], rows_t, stable, src_t, f"rank {d} scales")
+    del table
 
-    # ---- step 7: combine from every rank's expert output
-    rng = np.random.default_rng(200 + seed)
-    tokens = np.arange(w.N) if w.N <= 1024 else np.unique(np.concatenate(
-        [rng.integers(0, w.N, 300), [0, w.N - 1], np.arange(1, R + 1) * T - 1, np.arange(R) * T]))
+    # ---- step 7: combine from every rank's expert output, every token
     modes = ["bf16"] if not w.fp8 else ["fused", "fp8"]
     for mode in modes:
         if mode == "fp8":
             em.identity_expert()
         em.combine()
         assert em.check_errors() == 0
-        got = _to_host(out.index_select(0, torch.from_numpy(tokens).cuda()))
-        _check_combine(got, _combine_expected(w, x, o_idx, o_w, tokens, mode))
+        check_combine(to_host(out), combine_expected(w, x, o_idx, o_w, np.arange(w.N), mode))
 
 
 def test_shard_call_order_and_errors(cuda):
@@ -196,7 +195,7 @@ def test_shard_zero_tokens_and_ragged(cuda):
         for b in bufs:
             assert ep.ep_check_errors(b) == 0
         got_rows = [int(ep.ep_buffer_shard(b, T)["recv_off"][-1].item()) for b in bufs]
-        o_idx, o_w, _ = _oracle_route(lw, logits)
+        o_idx, o_w, _ = oracle_route(lw, logits)
         o_lay = oracle.layout(o_idx, w.R, T, w.E)
         assert got_rows == np.diff(o_lay["rank_off"]).tolist()
         if T == 0:
@@ -207,6 +206,6 @@ def test_shard_zero_tokens_and_ragged(cuda):
             valid = o_lay["dst_row"] >= 0
             order = np.argsort(o_lay["dst_row"][valid])
             src = np.repeat(np.arange(lw.N), w.K).reshape(lw.N, w.K)[valid][order]
-            assert np.array_equal(_to_host(recv[d]["recv_src"][:b_ - a]), src[a:b_].astype(np.int32))
-        got = _to_host(out[:lw.N])
-        _check_combine(got, _combine_expected(lw, x, o_idx, o_w, np.arange(lw.N), "bf16"))
+            assert np.array_equal(to_host(recv[d]["recv_src"][:b_ - a]), src[a:b_].astype(np.int32))
+        got = to_host(out[:lw.N])
+        check_combine(got, combine_expected(lw, x, o_idx, o_w, np.arange(lw.N), "bf16"))
