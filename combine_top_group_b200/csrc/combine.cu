@@ -139,9 +139,10 @@ __global__ void __launch_bounds__(kFp8Threads) combine_fp8_kernel(CombineParams 
     for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {
         report_rows<Y>(p, g);
         for (int v = threadIdx.x; v < nvec; v += kFp8Threads) {
-            float acc[16];
+            // acc[j] holds channels 2j and 2j+1 as an fp32 pair
+            uint64_t acc[8];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
+            for (int j = 0; j < 8; ++j) acc[j] = 0ull;
             for (int k0 = 0; k0 < p.K; k0 += kChunk) {
                 uint4 q[kChunk];
                 float sc[kChunk];
@@ -174,22 +175,28 @@ __global__ void __launch_bounds__(kFp8Threads) combine_fp8_kernel(CombineParams 
 #pragma unroll
                 for (int i = 0; i < kChunk; ++i) {
                     if (row[i] >= 0) {
+                        // per channel: acc = fma(w, e4m3 * scale, acc), each step rounded
+                        // as in the scalar chain, two channels per instruction
+                        const uint64_t w2 = f32x2_pack(w[i], w[i]);
+                        const uint64_t s2 = f32x2_pack(sc[i], sc[i]);
                         const uint32_t u[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             const float2 a = unpack_e4m3x2(u[j] & 0xffffu);
                             const float2 b = unpack_e4m3x2(u[j] >> 16);
-                            acc[4 * j + 0] = __fmaf_rn(w[i], __fmul_rn(a.x, sc[i]), acc[4 * j + 0]);
-                            acc[4 * j + 1] = __fmaf_rn(w[i], __fmul_rn(a.y, sc[i]), acc[4 * j + 1]);
-                            acc[4 * j + 2] = __fmaf_rn(w[i], __fmul_rn(b.x, sc[i]), acc[4 * j + 2]);
-                            acc[4 * j + 3] = __fmaf_rn(w[i], __fmul_rn(b.y, sc[i]), acc[4 * j + 3]);
+                            acc[2 * j] = f32x2_fma_rn(w2, f32x2_mul_rn(f32x2_pack(a.x, a.y), s2), acc[2 * j]);
+                            acc[2 * j + 1] =
+                                f32x2_fma_rn(w2, f32x2_mul_rn(f32x2_pack(b.x, b.y), s2), acc[2 * j + 1]);
                         }
                     }
                 }
             }
             u32x8 o;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) o.v[j] = pack_bf16x2(acc[2 * j], acc[2 * j + 1]);
+            for (int j = 0; j < 8; ++j) {
+                const float2 a = f32x2_unpack(acc[j]);
+                o.v[j] = pack_bf16x2(a.x, a.y);
+            }
             st256(p.out + (size_t)g * p.H * 2 + (size_t)v * 32, o);
         }
     }

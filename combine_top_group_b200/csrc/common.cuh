@@ -79,6 +79,33 @@ __device__ __forceinline__ float2 unpack_e4m3x2(uint32_t two_bytes) {
     return __half22float2(__half2(raw));
 }
 
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic) ---------------------------
+// A pair of fp32 values in one 64-bit register: `lo` in the low half. The
+// paired multiply and fused multiply-add round each lane on its own (RN), so
+// a pair op gives the same bits as two scalar __fmul_rn / __fmaf_rn.
+
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f32x2_unpack(uint64_t v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ uint64_t f32x2_mul_rn(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+// a * b + c per lane, one rounding.
+__device__ __forceinline__ uint64_t f32x2_fma_rn(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
 // Order-preserving map from a (non-NaN) float to uint32: a < b <=> key(a) <
 // key(b). -0 is folded into +0 first, so equal values get equal keys.
 // Key 0 is never produced, so 0 can mean "no candidate".

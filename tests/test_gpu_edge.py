@@ -169,6 +169,48 @@ def test_set_num_sms_changes_nothing_but_the_grid(cuda, num_sms):
         ep.ep_buffer_set_num_sms(pipe.buf, -1)
 
 
+@pytest.mark.parametrize("num_sms", [1, 20, 111])
+def test_capped_combine_prefill_shape(cuda, num_sms):
+    """Dispatch and bf16 combine under an SM budget at the prefill shape
+    (H = 7168, K = 8): receive rows and combine output equal the uncapped
+    run's, and the output is the oracle's (identity experts)."""
+    ep, runner = cuda
+    from parity_util import check_combine, combine_expected, oracle_route, to_host
+    w = wl.WORKLOADS["prefill"].with_tokens(64)
+    x, logits = wl.make_x(w, 5), wl.make_logits(w, 5)
+    pipe = runner.Pipeline(w, 5, x=x, logits=logits)
+    pipe.step()
+    M = pipe.num_rows()
+    ref = (pipe.recv["recv_x"][:M].clone(), pipe.out.clone())
+    ep.ep_buffer_set_num_sms(pipe.buf, num_sms)
+    pipe.recv["recv_x"][:M].zero_()
+    pipe.out.zero_()
+    pipe.step()
+    assert pipe.check_errors() == 0
+    assert torch.equal(pipe.recv["recv_x"][:M].view(torch.int16), ref[0].view(torch.int16))
+    assert torch.equal(pipe.out.view(torch.int16), ref[1].view(torch.int16))
+    o_idx, o_w, _ = oracle_route(w, logits)
+    check_combine(to_host(pipe.out), combine_expected(w, x, o_idx, o_w, np.arange(w.N), "bf16"))
+
+
+def test_capped_shard_combine_through_peer_tables(cuda):
+    """The one-rank-per-GPU combine (peer pointer tables) under an SM budget
+    gives the uncapped bytes."""
+    ep, runner = cuda
+    from combine_top_group_b200 import shard
+    w = wl.WORKLOADS["prefill"].with_tokens(32)
+    x = torch.from_numpy(wl.make_x(w, 6).view(np.int16)).view(torch.bfloat16).cuda()
+    lt = torch.from_numpy(np.ascontiguousarray(wl.make_logits(w, 6))).cuda()
+    outs = []
+    for num_sms in (0, 9):
+        out = torch.zeros(w.N, w.H, dtype=torch.bfloat16, device="cuda")
+        em = shard.EmulatedRanks(w, x, lt, out, num_sms=num_sms)
+        em.step()
+        assert em.check_errors() == 0
+        outs.append(out)
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+
+
 def test_deterministic_bytes(cuda):
     ep, runner = cuda
     w = wl.WORKLOADS["decode"]
