@@ -13,13 +13,21 @@ run back to back with no flush. For workloads that fit in L2 (--config tiny
 or decode) a 512 MB buffer is written between steps.
 
 value = the step's algorithmic HBM bytes (layout + dispatch + combine) / step
-time, in GB/s, summed over ranks. N > 1 runs N independent replicas (weak
-scaling), with no data-path collective. The timed region is K steps
-bracketed by a barrier and a device sync, and the time is the max over
-ranks. Rank 0 prints one JSON line.
+time, in GB/s, summed over ranks. The timed region is K steps bracketed by a
+barrier and a device sync, and the time is the max over ranks. Rank 0 prints
+one JSON line.
 
---impl reference times the CPU oracle (the only reference this path has)
-on rank 0, on a bounded sample of the same workload. Other ranks exit 0.
+N > 1 (under torchrun) runs the method one EP rank per GPU: R = N ranks, each
+with the workload's T tokens per rank (weak scaling), the count all-gather
+over NCCL, and dispatch / combine storing into and loading from the other
+GPUs' receive arrays over NVLink (workspaces mapped through CUDA IPC). An NCCL all-to-all-v of
+the same rows is timed beside it. --replicas runs N independent copies of the
+emulated single-GPU job instead. --one-rank-per-gpu takes the per-GPU path on
+one GPU too (R = 1).
+
+--impl reference times the CPU oracle (the only reference this path has) on
+all the host's cores, on rank 0, on a bounded sample of the same workload.
+Other ranks exit 0.
 """
 from __future__ import annotations
 
@@ -52,7 +60,7 @@ def parse_args(argv=None):
     ap.add_argument("--tokens", type=int, default=0,
                     help="tokens per rank (0 = the workload's own); smaller cases for profiling")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--num-sms", type=int, default=0, help="SM cap for dispatch (0 = all)")
+    ap.add_argument("--num-sms", type=int, default=0, help="SM cap for dispatch and combine (0 = all)")
     ap.add_argument("--fused-fp8-combine", action="store_true",
                     help="FP8 workloads: combine straight from the e4m3 rows (fused dequant)")
     ap.add_argument("--sweep-sms", action="store_true",
@@ -66,6 +74,10 @@ def parse_args(argv=None):
                     help="also time the step captured in a CUDA graph (one replay per step)")
     ap.add_argument("--shard", action="store_true",
                     help="also time the one-rank-per-GPU calls, R ranks emulated on this GPU")
+    ap.add_argument("--replicas", action="store_true",
+                    help="--gpus N > 1: run N independent replicas of the emulated job instead of one EP rank per GPU")
+    ap.add_argument("--one-rank-per-gpu", action="store_true",
+                    help="run the one-EP-rank-per-GPU path even on one GPU (R = 1); the default for --gpus N > 1")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-copy-streams", type=int, default=1,
@@ -91,13 +103,24 @@ def oracle_sample(w: wl.Workload, seed: int = 0):
     return ws, wl.make_x(ws, seed), wl.make_logits(ws, seed)
 
 
-def oracle_step(ws: wl.Workload, x, logits, phases: dict | None = None):
+def host_cores() -> int:
+    """Cores this process may run on."""
+    if hasattr(os, "sched_getaffinity"):
+        return len(os.sched_getaffinity(0))
+    return os.cpu_count() or 1
+
+
+def oracle_step(ws: wl.Workload, x, logits, phases: dict | None = None, threads: int = 1):
     """One oracle pass (route, layout, dispatch, identity expert, combine) over
-    the sample. Returns (seconds, algorithmic bytes); `phases` accumulates the
-    seconds of each phase."""
+    the sample: single-threaded, or over token chunks on `threads` host
+    threads (same C functions, identical outputs). Returns (seconds,
+    algorithmic bytes); `phases` accumulates the seconds of each phase."""
     import oracle  # test infrastructure: only the CPU legs of the bench run it
     t0 = time.perf_counter()
-    res = oracle.run_path(x, logits, ws, timings=phases)
+    if threads > 1:
+        res = oracle.run_path_parallel(x, logits, ws, threads, timings=phases)
+    else:
+        res = oracle.run_path(x, logits, ws, timings=phases)
     dt = time.perf_counter() - t0
     M = res["M"]
     return dt, metrics.layout_bytes(ws) + metrics.dispatch_bytes(ws, M) + metrics.combine_bytes(ws, M)
@@ -137,23 +160,35 @@ class OneCore:
         return False
 
 
-def cpu_baseline(w: wl.Workload) -> dict:
-    """The oracle on the host, pinned to one core, repeated over the sample
-    until CPU_BASELINE_MIN_S of work has been timed."""
-    ws, x, logits = oracle_sample(w)
+def _timed_oracle(ws, x, logits, threads: int, min_s: float):
     tot_t, tot_b, reps = 0.0, 0, 0
     phases: dict = {}
+    while tot_t < min_s:
+        dt, nb = oracle_step(ws, x, logits, phases, threads)
+        tot_t += dt
+        tot_b += nb
+        reps += 1
+    return tot_b / tot_t / 1e9, tot_t, reps, {k: v / reps * 1e3 for k, v in phases.items()}
+
+
+def cpu_baseline(w: wl.Workload) -> dict:
+    """The oracle on the host over the sample, repeated until CPU_BASELINE_MIN_S
+    of work has been timed: on all the host's cores (token chunks on threads),
+    and single-threaded pinned to one core."""
+    ws, x, logits = oracle_sample(w)
+    n = host_cores()
+    v_all, t_all, r_all, ph_all = _timed_oracle(ws, x, logits, n, CPU_BASELINE_MIN_S)
     with OneCore():
-        while tot_t < CPU_BASELINE_MIN_S:
-            dt, nb = oracle_step(ws, x, logits, phases)
-            tot_t += dt
-            tot_b += nb
-            reps += 1
-    return {"value": tot_b / tot_t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{reps} passes of the whole path (route, layout, dispatch, identity expert, combine) "
-                      f"over {ws.R}x{ws.T} tokens of the same shape; {tot_t:.1f} s single-threaded C, "
-                      f"pinned to one core",
-            "phase_ms_per_pass": {k: v / reps * 1e3 for k, v in phases.items()},
+        v_one, t_one, r_one, ph_one = _timed_oracle(ws, x, logits, 1, CPU_BASELINE_MIN_S)
+    what = f"the whole path (route, layout, dispatch, identity expert, combine) over {ws.R}x{ws.T} tokens of " \
+           f"the same shape"
+    return {"value": v_all, "unit": "GB/s", "cores": n, "kind": "oracle",
+            "sample": f"{r_all} passes of {what}; {t_all:.1f} s of C on {n} host threads (token chunks; "
+                      f"mask and layout scan serial)",
+            "phase_ms_per_pass": ph_all,
+            "single_core": {"value": v_one, "unit": "GB/s", "cores": 1,
+                            "sample": f"{r_one} passes, {t_one:.1f} s single-threaded, pinned to one core",
+                            "phase_ms_per_pass": ph_one},
             "host": host_cpu()}
 
 
@@ -163,26 +198,26 @@ def run_reference(args, w: wl.Workload, rank: int, world: int):
     ws, x, logits = oracle_sample(w)
     tot_t, tot_b = 0.0, 0
     phases: dict = {}
-    with OneCore():
-        for _ in range(args.warmup):
-            oracle_step(ws, x, logits)
-        for _ in range(args.steps):
-            dt, nb = oracle_step(ws, x, logits, phases)
-            tot_t += dt
-            tot_b += nb
+    n = host_cores()
+    for _ in range(args.warmup):
+        oracle_step(ws, x, logits, threads=n)
+    for _ in range(args.steps):
+        dt, nb = oracle_step(ws, x, logits, phases, threads=n)
+        tot_t += dt
+        tot_b += nb
     value = tot_b / tot_t / 1e9
     line = {
         "impl": "reference", "metric": METRIC,
         "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if not w.fp8 else "fp8_e4m3", "data": "synthetic",
-        "config": {**workload_desc(w), "parallelism": "1 host core", "combine_input": "bf16",
+        "config": {**workload_desc(w), "parallelism": f"{n} host threads", "combine_input": "bf16",
                    "sample_tokens_per_rank": ws.T,
                    "sample": f"each step runs the whole path over {ws.R}x{ws.T} of the workload's "
                              f"{w.R}x{w.T} tokens"},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": n, "kind": "oracle",
                          "sample": f"each step: the whole path over {ws.R}x{ws.T} tokens of the same shape "
-                                   f"(single-threaded C, pinned to one core)",
+                                   f"(C over token chunks on {n} host threads; mask and layout scan serial)",
                          "phase_ms_per_pass": {k: v / args.steps * 1e3 for k, v in phases.items()},
                          "host": host_cpu()},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -614,6 +649,247 @@ def measure_e2e(pipe, w, dev, stream, fused, bytes_step, steps, world, copy_stre
             "copies": f"pinned host buffers; H2D and D2H each on {C} copy stream(s), double-buffered across steps"}
 
 
+def free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def ep_workload(w: wl.Workload, world: int) -> wl.Workload:
+    """The workload as a node runs it: R = world ranks (one per GPU), the
+    same T tokens per rank, experts, routing and hidden size."""
+    import dataclasses
+    if w.low_latency:
+        raise SystemExit("the one-rank-per-GPU path uses the standard receive layout")
+    if w.E % world:
+        raise SystemExit(f"E={w.E} is not a multiple of {world} ranks")
+    return dataclasses.replace(w, R=world)
+
+
+def run_ep(args, w0: wl.Workload, rank: int, world: int, local_rank: int):
+    """One EP rank per GPU (shard.DistributedRank): this process routes its own
+    T tokens, all-gathers the count rows, and dispatch / combine store into and
+    load from every rank's receive arrays (peer memory over NVLink). Phases are
+    timed with events on the launching stream; the barriers between them are
+    stream-ordered NCCL all-reduces, included in the phase that waits on them.
+    FP8 workloads combine straight from the e4m3 rows (fused dequantisation)."""
+    import torch
+    import torch.distributed as dist
+
+    from combine_top_group_b200 import shard
+
+    w = ep_workload(w0, world)
+    T, H = w.T, w.H
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream(dev)
+    drv = shard.DistributedRank(w, dev, num_sms=args.num_sms)
+    xs = wl.make_x(w, 0, rows=slice(rank * T, (rank + 1) * T))
+    x = torch.from_numpy(xs.view(np.int16)).view(torch.bfloat16).to(dev)
+    logits = torch.from_numpy(np.ascontiguousarray(wl.make_logits(w, 0)[rank * T:(rank + 1) * T])).to(dev)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        drv.layout(logits)
+        drv.exchange()
+        drv.place()
+        if ev is not None:
+            ev[1].record(stream)
+        drv.barrier()  # every rank has finished reading the previous step's rows
+        drv.dispatch(x)
+        if ev is not None:
+            ev[2].record(stream)
+        drv.barrier()  # every rank's rows are written (identity experts)
+        drv.combine(out)
+        if ev is not None:
+            ev[3].record(stream)
+
+    step()
+    torch.cuda.synchronize(dev)
+    if drv.check_errors() != 0:
+        raise RuntimeError("device error word set during set-up")
+    check = ep_output_check(w, x, out, drv)
+    send, recv = drv.alltoallv_splits()
+    M_s = sum(send)  # rows this rank's tokens send
+    remote = M_s - send[rank]  # of which to other GPUs
+    b = 1 if w.fp8 else 2
+    row_b = H * b + ((H // 128) * 4 if w.fp8 else 0)
+    bytes_layout = metrics.layout_bytes(w, N=T)
+    bytes_dispatch = metrics.dispatch_bytes(w, M_s, N=T)
+    bytes_combine = metrics.combine_bytes(w, M_s, fused_fp8=w.fp8, N=T)
+    totals = metrics.sum_over_ranks([bytes_layout, bytes_dispatch, bytes_combine, remote * (row_b + 8),
+                                     remote * row_b], dev)
+    bytes_step = sum(totals[:3])
+
+    props = torch.cuda.get_device_properties(dev)
+    bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+    clk = metrics.ClockSampler(pci_bus_id=bus).start()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_host0 = time.perf_counter()
+    for i in range(K):
+        step(ev[i])
+        clk.sample_now()
+    clk.sample_now(0.0)
+    torch.cuda.synchronize(dev)
+    clk.sample_now(0.0)
+    t_host1 = time.perf_counter()
+    dist.barrier()
+    clocks = clk.stop(t_host0, t_host1)
+    if drv.check_errors() != 0:
+        raise RuntimeError("device error word set during the timed steps")
+    t_lay = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+    t_disp = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    t_comb = sum(e[2].elapsed_time(e[3]) for e in ev) / 1e3
+    t_total, t_lay, t_disp, t_comb = metrics.max_over_ranks([t_lay + t_disp + t_comb, t_lay, t_disp, t_comb], dev)
+    value = bytes_step * K / t_total / 1e9
+
+    nccl = nccl_alltoallv_baseline(drv, w, send, recv, dev, reps=max(3, min(K, 10)))
+    e2e = None if args.no_e2e else measure_e2e_ep(step, x, logits, out, dev, stream, bytes_step,
+                                                  steps=max(K, 5))
+    d_avg, c_avg = t_disp / K, t_comb / K
+    peak_hbm, peak_src = metrics.hbm_peak()
+    if world > 1:
+        # bound: the rows that cross NVLink, per direction per GPU, at the
+        # measured peer-copy bandwidth
+        nv_bytes = totals[3] / world
+        roof = {"bound": "nvlink", "kernel": "dispatch", "achieved": nv_bytes / d_avg / 1e9,
+                "peak": metrics.NVLINK_PEER_GBS, "unit": "GB/s",
+                "frac": nv_bytes / d_avg / 1e9 / metrics.NVLINK_PEER_GBS, "traffic": None,
+                "peak_source": "measured peer copy per direction (NVLink 5)"}
+    else:
+        roof = {"bound": "hbm", "kernel": "dispatch", "achieved": totals[1] / d_avg / 1e9, "peak": peak_hbm,
+                "unit": "GB/s", "frac": totals[1] / d_avg / 1e9 / peak_hbm, "traffic": None,
+                "peak_source": f"{peak_src} (hbm_gbs copy)"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": t_total / K * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8_e4m3" if w.fp8 else "bf16", "data": "synthetic",
+        "config": {**{k: v for k, v in workload_desc(w).items() if k != "ranks_emulated"}, "ep_ranks": world,
+                   "parallelism": f"ep{world}: one EP rank per GPU, peer stores/loads "
+                                                      f"through IPC-mapped workspaces, NCCL count all-gather",
+                   "num_sms": args.num_sms or "all", "combine_input": "fp8_fused" if w.fp8 else "bf16",
+                   "l2": "inputs larger than L2 (no flush)" if T * H * 2 * w.K > 2 * 126 * 2 ** 20 else
+                         "no flush (small per-rank batch)"},
+        "layout_us": t_lay / K * 1e6, "dispatch_us": d_avg * 1e6, "combine_us": c_avg * 1e6,
+        "dispatch_plus_combine_us": (d_avg + c_avg) * 1e6,
+        "phases": "layout = route + count all-gather + place; dispatch and combine each include the "
+                  "cross-rank barrier before them",
+        "dispatch_gbs": totals[1] / world / d_avg / 1e9, "combine_gbs": totals[2] / world / c_avg / 1e9,
+        "rows_sent_per_rank": M_s, "rows_to_other_gpus_per_rank": remote,
+        "nvlink_bytes_per_step": {"dispatch": totals[3], "combine": totals[4]},
+        "algorithmic_bytes": {"layout": totals[0], "dispatch": totals[1], "combine": totals[2]},
+        "roofline": roof, "nccl_alltoallv": nccl, "output_check": check,
+        "gpu_launches": 4 * K,  # layout, place, dispatch, combine per step (NCCL's own kernels not counted)
+        "clocks": clocks,
+    }
+    why = metrics.clocks_rejected(clocks)
+    if why:
+        line["clocks_rejected"] = why
+    if e2e is not None:
+        line["e2e"] = e2e
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def ep_output_check(w, x, out, drv) -> dict:
+    """A property that holds at any size, checked on the device after a step
+    with identity experts: each token's output is its input scaled by the sum
+    of its top-k weights, out[t] = x[t] * sum_k w[t,k], within the bf16
+    combine tolerance (2^-7 |ref| + 1e-3), or the FP8 round trip's (2^-4
+    relative, e4m3 having 3 mantissa bits). Rows lost or misplaced on the
+    way to another GPU and back break it."""
+    import torch
+    lay = drv.ep.ep_buffer_layout(drv.buf, w.T)
+    ref = x.float() * lay["topk_w"].sum(dim=1, keepdim=True)
+    err = (out.float() - ref).abs()
+    rel = 2.0 ** -4 + 2.0 ** -7 if w.fp8 else 2.0 ** -7
+    bad = int((err > rel * ref.abs() + 1e-3).sum().item())
+    ok = bad == 0
+    if not ok:
+        raise RuntimeError(f"output check failed on {bad} elements (max err {float(err.max()):.3g})")
+    return {"passed": True, "elements": int(out.numel()), "rule": "out = x * sum_k w within tolerance"}
+
+
+def nccl_alltoallv_baseline(drv, w, send, recv, dev, reps: int) -> dict:
+    """NCCL all-to-all-v moving the same rows between the ranks: this rank's
+    rows grouped by destination (split sizes from the exchanged counts), then
+    the reverse exchange for the combine. Only the collectives are timed: no
+    packing, no quantisation, no weighted sum."""
+    import torch
+    import torch.distributed as dist
+    dt = torch.uint8 if w.fp8 else torch.bfloat16
+    cols = w.H + (w.H // 128) * 4 if w.fp8 else w.H  # FP8 rows carry their scales
+    sbuf = torch.empty(max(sum(send), 1), cols, dtype=dt, device=dev)
+    rbuf = torch.empty(max(sum(recv), 1), cols, dtype=dt, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd():
+        dist.all_to_all_single(rbuf[:sum(recv)], sbuf[:sum(send)], recv, send)
+
+    def bwd():
+        dist.all_to_all_single(sbuf[:sum(send)], rbuf[:sum(recv)], send, recv)
+
+    fwd()
+    bwd()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record(stream)
+    for _ in range(reps):
+        fwd()
+    ev[1].record(stream)
+    for _ in range(reps):
+        bwd()
+    ev[2].record(stream)
+    torch.cuda.synchronize(dev)
+    t_f, t_b = metrics.max_over_ranks([ev[0].elapsed_time(ev[1]) / 1e3 / reps,
+                                       ev[1].elapsed_time(ev[2]) / 1e3 / reps], dev)
+    row_bytes = cols * (1 if w.fp8 else 2)
+    total = metrics.sum_over_ranks([sum(send) * row_bytes], dev)[0]
+    return {"dispatch_direction_us": t_f * 1e6, "combine_direction_us": t_b * 1e6,
+            "bytes_moved": total, "reps": reps,
+            "what": "torch.distributed.all_to_all_single (NCCL) of the same rows, split sizes from the "
+                    "exchanged counts; collectives only"}
+
+
+def measure_e2e_ep(step, x, logits, out, dev, stream, bytes_step, steps: int) -> dict:
+    """The EP step end to end through the public calls: every step copies
+    this rank's x and logits in from pinned host memory and its output back,
+    on the launching stream, inside the timed region."""
+    import torch
+    x_h = x.cpu().pin_memory()
+    l_h = logits.cpu().pin_memory()
+    o_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def one():
+        x.copy_(x_h, non_blocking=True)
+        logits.copy_(l_h, non_blocking=True)
+        step()
+        o_h.copy_(out, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(dev)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        one()
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    t = metrics.max_over_ranks([s.elapsed_time(e) / 1e3], dev)[0]
+    return {"value": bytes_step * steps / t / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": x_h.numel() * 2 + l_h.numel() * 4, "d2h_bytes_per_step": o_h.numel() * 2,
+            "steps": steps, "ms_per_step": t / steps * 1e3,
+            "copies": "pinned host buffers, copies on the launching stream (per rank)"}
+
+
 def main(argv=None):
     args = parse_args(argv)
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -629,14 +905,21 @@ def main(argv=None):
 
     import torch
     import torch.distributed as dist
-    if world > 1:
+    per_gpu = args.one_rank_per_gpu or (world > 1 and not args.replicas)
+    if world > 1 or per_gpu:
         torch.cuda.set_device(local_rank)
+        kw = {}
+        if world == 1 and "MASTER_ADDR" not in os.environ:
+            kw = dict(init_method=f"tcp://127.0.0.1:{free_port()}", rank=0, world_size=1)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
+                                device_id=torch.device("cuda", local_rank), **kw)
     try:
-        run_ours(args, w, rank, world, local_rank)
+        if per_gpu:
+            run_ep(args, w, rank, world, local_rank)
+        else:
+            run_ours(args, w, rank, world, local_rank)
     finally:
-        if world > 1:
+        if dist.is_initialized():
             dist.destroy_process_group()
 
 

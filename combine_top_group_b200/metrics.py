@@ -18,6 +18,7 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
 
 FALLBACK_HBM_GBS = 6650.0  # an earlier B200 copy measurement, used only without MEASURED_PEAKS.json
+NVLINK_PEER_GBS = 770.0  # measured B200 peer copy per direction over NVLink 5 (900 GB/s nominal)
 
 
 # ---- algorithmic bytes -------------------------------------------------------
@@ -60,6 +61,18 @@ def max_over_ranks(values, device=None):
         return [float(v) for v in values]
     t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def sum_over_ranks(values, device=None):
+    """Element-wise sum over the default process group (all ranks call it).
+    Single process: the values unchanged."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return t.tolist()
 
 
@@ -115,8 +128,10 @@ def source_hash(kernel: str | None = None) -> str:
 
 
 def stored_traffic(kernel: str, workload: str) -> float | None:
-    """dram read+write bytes per launch from the committed ncu summary, or
-    None if absent or captured from other sources."""
+    """dram read+write bytes per launch at the workload's full size, from the
+    committed ncu capture of a smaller case of the same workload scaled by
+    tokens (see record_traffic), or None if absent or captured from other
+    sources."""
     try:
         with open(TRAFFIC_FILE) as f:
             data = json.load(f)
@@ -173,20 +188,29 @@ def traffic_from_ncu(text: str) -> dict:
     return out
 
 
-def record_traffic(csv_path: str, workload: str, command: str, note: str) -> dict:
-    """Writes the per-kernel dram bytes of an ncu capture into the traffic file
-    under `workload`, stamped with each kernel's source hash."""
+def record_traffic(csv_path: str, workload: str, kernel: str, command: str, captured_tokens: int) -> dict:
+    """Writes one kernel's dram bytes from an ncu capture of a small case of
+    `workload` (captured_tokens tokens per rank) into the traffic file. The
+    capture is one kernel (-k) and one launch; the full-size figure scales it
+    by tokens, workload T / captured_tokens: every byte the kernels move
+    (token rows read or written, receive rows, logits, indices) grows in
+    proportion to the tokens at a fixed routing distribution. Stamped with
+    the kernel's source hash."""
     with open(csv_path) as f:
-        ent = traffic_from_ncu(f.read())
+        got = traffic_from_ncu(f.read())
+    if kernel not in got:
+        raise ValueError(f"no {kernel} launch with dram counters in {csv_path}")
+    k = got[kernel]
+    scale = wl.WORKLOADS[workload].T / captured_tokens
+    ent = {"dram_read": k["dram_read"], "dram_write": k["dram_write"], "captured_tokens_per_rank": captured_tokens,
+           "scale_to_workload": scale, "dram_bytes_per_launch": int(round((k["dram_read"] + k["dram_write"]) * scale)),
+           "source_hash": k["source_hash"], "command": command}
     try:
         with open(TRAFFIC_FILE) as f:
             data = json.load(f)
     except (OSError, ValueError):
         data = {}
-    slot = data.setdefault(workload, {})
-    slot.update(ent)
-    slot["command"] = command
-    slot["note"] = note
+    data.setdefault(workload, {})[kernel] = ent
     with open(TRAFFIC_FILE, "w") as f:
         json.dump(data, f, indent=1, sort_keys=False)
         f.write("\n")
@@ -372,10 +396,11 @@ def clocks_rejected(clk: dict | None) -> str | None:
 
 if __name__ == "__main__":
     import argparse
-    ap = argparse.ArgumentParser(description="record ncu dram traffic per kernel")
+    ap = argparse.ArgumentParser(description="record one kernel's ncu dram traffic, scaled to the full workload")
     ap.add_argument("csv")
     ap.add_argument("workload")
+    ap.add_argument("kernel", choices=sorted(NCU_NAMES))
+    ap.add_argument("--tokens", type=int, required=True, help="tokens per rank of the captured case")
     ap.add_argument("--command", required=True)
-    ap.add_argument("--note", default="")
     a = ap.parse_args()
-    print(json.dumps(record_traffic(a.csv, a.workload, a.command, a.note), indent=1))
+    print(json.dumps(record_traffic(a.csv, a.workload, a.kernel, a.command, a.tokens), indent=1))

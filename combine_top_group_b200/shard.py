@@ -13,8 +13,8 @@ Two drivers run the same C calls:
 - `DistributedRank`: this process is one rank of a torch.distributed job, one
   GPU per process.
   - The count exchange is an all-gather of R x E int32.
-  - The workspaces are torch symmetric memory, so every rank's receive arrays
-    have device pointers on every GPU.
+  - Every rank maps the others' workspaces through CUDA IPC handles, so
+    every rank's receive arrays have device pointers on every GPU.
   - Barriers order the steps: a rank's receive rows are written only after
     every rank has finished reading the last step's rows, and they are read
     only after every rank has finished writing them.
@@ -158,26 +158,77 @@ def peer_tables(local_base: int, peer_bases: list[int], arrays: dict) -> dict:
     return out
 
 
+class IpcPeerMemory:
+    """Workspaces that every rank of a node maps: each rank's workspace is an
+    ordinary device allocation, and the others open it through its CUDA IPC
+    handle (cudaIpcGetMemHandle / cudaIpcOpenMemHandle, through torch's CUDA
+    storage sharing), the create-shared-buffer scheme of vLLM's custom
+    all-reduce. The mappings are plain peer memory: no NVLink multicast object
+    is created, and the kernels only store and load through them.
+
+    Same interface as torch symmetric memory's empty / rendezvous:
+    rendezvous(t, group) is collective and returns a handle whose
+    buffer_ptrs[d] is rank d's copy of t as this GPU addresses it."""
+
+    def empty(self, n: int, dtype, device) -> torch.Tensor:
+        return torch.empty(n, dtype=dtype, device=device)
+
+    def rendezvous(self, t: torch.Tensor, group=None):
+        import torch.distributed as dist
+        storage = t.untyped_storage()
+        info = storage._share_cuda_()  # (device, handle, size, offset, ref counter..., event...)
+        off = t.data_ptr() - storage.data_ptr()
+        world, me = dist.get_world_size(group), dist.get_rank(group)
+        infos = [None] * world
+        dist.all_gather_object(infos, (info, off), group=group)
+
+        class Handle:
+            pass
+        h = Handle()
+        h.mapped = []  # the opened peer storages, kept alive with the handle
+        h.buffer_ptrs = []
+        for d, (inf, o) in enumerate(infos):
+            if d == me:
+                h.buffer_ptrs.append(t.data_ptr())
+                continue
+            peer = torch.UntypedStorage._new_shared_cuda(*inf)
+            h.mapped.append(peer)
+            h.buffer_ptrs.append(peer.data_ptr() + o)
+        return h
+
+
+def alltoallv_splits(cnt_all: torch.Tensor, rank: int, L: int) -> tuple[list[int], list[int]]:
+    """Rows each rank pair exchanges, from the gathered counts cnt_all [R, E]
+    (expert e lives on rank e // L): (rows this rank sends to each rank,
+    rows it receives from each rank). The split sizes an all-to-all-v of the
+    same rows takes."""
+    R = cnt_all.shape[0]
+    per_dst = cnt_all.view(R, R, L).sum(dim=2)  # [src, dst]
+    return per_dst[rank].tolist(), per_dst[:, rank].tolist()
+
+
 class DistributedRank:
     """This process's rank of a one-GPU-per-process job (torch.distributed,
-    NCCL). The workspace is symmetric memory, so every rank can store into and
-    load from every other rank's receive arrays.
+    NCCL). Every rank maps every other rank's workspace (IpcPeerMemory, or
+    torch symmetric memory when passed as `peer_mem`), so it can store into and
+    load from every rank's receive arrays.
 
-    Every call of a step runs on the current CUDA stream (or `stream`, made
-    current for the step), so the NCCL collectives (the count all-gather and
-    the barriers) are ordered after the kernels before them and before the
-    kernels after them.
+    Every call runs on the current CUDA stream (or `stream`, made current for
+    a step), and so do the NCCL collectives: the count all-gather and the
+    barriers. NCCL orders each collective after the kernels before it on
+    that stream and the kernels after it behind the collective, so a barrier
+    here is a one-int all-reduce that keeps the host free: a rank passes it
+    once every rank's earlier kernels have finished. Dispatch fences its
+    stores to peer memory at system scope before it ends.
 
-    `ep_lib` and `symm_mem_lib` default to the library binding and torch's
-    symmetric memory; the host logic (call order, count exchange, pointer
-    tables) is tested on CPU ranks with stand-ins for both. The repository has
-    no multi-GPU test of it."""
+    `ep_lib` and `peer_mem` default to the library binding and IpcPeerMemory;
+    the host logic (call order, count exchange, pointer tables) is tested on
+    CPU ranks with stand-ins for both."""
 
     def __init__(self, w: wl.Workload, device: torch.device, group=None, num_sms: int = 0, ep_lib=None,
-                 symm_mem_lib=None):
+                 peer_mem=None):
         import torch.distributed as dist
-        if symm_mem_lib is None:
-            from torch.distributed import _symmetric_memory as symm_mem_lib
+        peer_mem = IpcPeerMemory() if peer_mem is None else peer_mem
         self.ep = ep if ep_lib is None else ep_lib
         self.w = w
         self.group = group
@@ -186,35 +237,69 @@ class DistributedRank:
             raise ValueError(f"world size {dist.get_world_size(group)} != R={w.R}")
         cfg = shard_config(w, num_sms)
         nbytes = self.ep.ep_buffer_workspace_bytes(cfg)
-        self.workspace = symm_mem_lib.empty(nbytes, dtype=torch.uint8, device=device)
-        self.handle = symm_mem_lib.rendezvous(self.workspace,
+        self.workspace = peer_mem.empty(nbytes, dtype=torch.uint8, device=device)
+        self.handle = peer_mem.rendezvous(self.workspace,
                                               group=group if group is not None else dist.group.WORLD)
         self.buf = self.ep.ep_buffer_create(cfg, workspace=self.workspace)
         self.recv = self.ep.ep_buffer_recv(self.buf)
         self.sh = self.ep.ep_buffer_shard(self.buf, w.T)
         self.peers = peer_tables(self.workspace.data_ptr(), list(self.handle.buffer_ptrs),
                                  {k: self.recv[k] for k in ("recv_x", "recv_scale", "recv_src", "recv_w")})
+        self._flag = torch.zeros(1, dtype=torch.int32, device=device)
 
     def barrier(self):
+        """Stream-ordered barrier over the ranks (see the class notes)."""
         import torch.distributed as dist
-        dist.barrier(group=self.group)
+        dist.all_reduce(self._flag, group=self.group)
+
+    # --- the phases of one step, in order ----------------------------------
+    def layout(self, logits):
+        w = self.w
+        self.ep.ep_shard_layout(self.buf, self.rank, w.T, logits=logits, route=route_of(w),
+                                mask_seed=w.mask_seed, mask_frac=w.mask_frac)
+
+    def exchange(self):
+        exchange_counts(self.sh["cnt_row"], self.sh["cnt_all"], self.group)
+
+    def place(self):
+        self.ep.ep_shard_place(self.buf, self.rank, self.w.T)
+
+    def dispatch(self, x):
+        p = self.peers
+        self.ep.ep_shard_dispatch(self.buf, self.rank, self.w.T, x, p["recv_x"], p["recv_scale"], p["recv_src"],
+                                  p["recv_w"])
+
+    def combine(self, out):
+        """Bf16 rows are the expert output as they are; FP8 rows are read as
+        e4m3 + scales (fused dequantisation)."""
+        p = self.peers
+        self.ep.ep_shard_combine(self.buf, self.rank, self.w.T, p["recv_x"], p["recv_scale"] if self.w.fp8 else None,
+                                 out)
 
     def step(self, x: torch.Tensor, logits: torch.Tensor, out: torch.Tensor, expert=None, stream=None):
         """One step for this rank's T tokens. `expert(recv_x, recv_scale, rows)`
         may transform the received rows in place (identity when None)."""
         import contextlib
-        w, s, b, lib = self.w, self.rank, self.buf, self.ep
         ctx = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
         with ctx:
-            lib.ep_shard_layout(b, s, w.T, logits=logits, route=route_of(w), mask_seed=w.mask_seed,
-                                mask_frac=w.mask_frac)
-            exchange_counts(self.sh["cnt_row"], self.sh["cnt_all"], self.group)
-            lib.ep_shard_place(b, s, w.T)
+            self.layout(logits)
+            self.exchange()
+            self.place()
             self.barrier()  # every rank is done reading the previous step's rows
-            p = self.peers
-            lib.ep_shard_dispatch(b, s, w.T, x, p["recv_x"], p["recv_scale"], p["recv_src"], p["recv_w"])
+            self.dispatch(x)
             self.barrier()  # every rank's rows are written
             if expert is not None:
-                expert(self.recv["recv_x"], self.recv["recv_scale"], int(self.sh["recv_off"][-1].item()))
-            self.barrier()  # every expert output is ready
-            lib.ep_shard_combine(b, s, w.T, p["recv_x"], p["recv_scale"] if w.fp8 else None, out)
+                expert(self.recv["recv_x"], self.recv["recv_scale"], self.received_rows())
+                self.barrier()  # every expert output is ready
+            self.combine(out)
+
+    def received_rows(self) -> int:
+        return int(self.sh["recv_off"][-1].item())
+
+    def check_errors(self) -> int:
+        return self.ep.ep_check_errors(self.buf)
+
+    # --- NCCL baseline ----------------------------------------------------------
+    def alltoallv_splits(self) -> tuple[list[int], list[int]]:
+        """(send, receive) row counts per rank for this step (syncs the host)."""
+        return alltoallv_splits(self.sh["cnt_all"].cpu(), self.rank, self.w.L)

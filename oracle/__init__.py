@@ -351,3 +351,97 @@ def run_path(x: np.ndarray, logits: np.ndarray | None, w, topk_idx=None, topk_w=
     lap("combine")
     return dict(topk_idx=idx, topk_w=tw, margin=margin, M=M, recv_x=recv_x,
                 recv_scale=recv_scale, recv_src=recv_src, recv_w=recv_w, y=y, out=out, **lay)
+
+
+# ---- the whole path over token chunks on host threads -------------------------
+
+def _spans(n: int, parts: int):
+    step = max(1, -(-n // max(1, parts)))
+    return [(a, min(n, a + step)) for a in range(0, n, step)]
+
+
+def run_path_parallel(x: np.ndarray, logits: np.ndarray, w, threads: int, timings: dict | None = None):
+    """run_path over token chunks on `threads` host threads: the same C
+    functions, each token's arithmetic in the same order, so every output is
+    identical to run_path's. ctypes releases the GIL during each call.
+    Routing, dispatch, the identity expert and combine run per chunk; the
+    slot mask (it hashes global slot ids) and the layout (a scan over all
+    tokens) run once, serially. Returns the same dict as run_path."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    lib = _load()
+    clock = [time.perf_counter()]
+
+    def lap(name):
+        now = time.perf_counter()
+        if timings is not None:
+            timings[name] = timings.get(name, 0.0) + now - clock[0]
+        clock[0] = now
+
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    N, H = x.shape
+    E, K = logits.shape[1], w.K
+    spans = _spans(N, 4 * threads)
+    P = ctypes.c_void_p
+
+    def at(a: np.ndarray, row: int):  # pointer to row `row` of a C-contiguous array
+        return P(a.ctypes.data + row * a.strides[0])
+
+    with ThreadPoolExecutor(max_workers=threads) as pool:
+        idx = np.empty((N, K), dtype=np.int32)
+        tw = np.empty((N, K), dtype=np.float32)
+        margin = np.empty(N, dtype=np.float64) if w.route == 2 else None
+
+        def route_span(ab):
+            a, b = ab
+            if w.route == 2:
+                lib.orc_route_group_sigmoid(at(logits, a), b - a, E, K, w.G, w.KG, at(idx, a), at(tw, a),
+                                            at(margin, a))
+            else:
+                lib.orc_route_softmax(at(logits, a), b - a, E, K, 1 if w.route == 1 else 0, at(idx, a), at(tw, a))
+        list(pool.map(route_span, spans))
+        if w.mask_frac:
+            apply_mask(idx, tw, w.mask_seed, w.mask_frac)
+        lap("route")
+        lay = layout(idx, w.R, w.T, E)
+        M = int(lay["expert_off"][-1])
+        if getattr(w, "low_latency", False):
+            lay["dst_row"], _ = layout_ll(idx, w.R, w.T, w.T, E)
+            M = E * w.R * w.T
+        lap("layout")
+        dst = lay["dst_row"]
+        recv_x = np.zeros((M, H), dtype=np.uint8 if w.fp8 else np.uint16)
+        recv_scale = np.zeros((M, H // 128), dtype=np.float32) if w.fp8 else None
+        recv_src = np.full(M, -1, dtype=np.int32)
+        recv_w = np.zeros(M, dtype=np.float32)
+
+        def dispatch_span(ab):  # every span writes its own tokens' rows
+            a, b = ab
+            lib.orc_dispatch(at(x, a), at(dst, a), at(tw, a), b - a, H, K, 1 if w.fp8 else 0, _p(recv_x),
+                             _p(recv_scale), _p(recv_src), _p(recv_w))
+        list(pool.map(dispatch_span, spans))
+        # orc_dispatch numbers a span's tokens from 0: the source id of each
+        # row is its global token index
+        gs, ks = np.nonzero(dst >= 0)
+        recv_src[dst[gs, ks]] = gs
+        lap("dispatch")
+        if w.fp8:
+            y = np.empty((M, H), dtype=np.uint16)
+
+            def expert_span(ab):
+                a, b = ab
+                lib.orc_identity_expert_fp8(at(recv_x, a), at(recv_scale, a), b - a, H, at(y, a))
+            list(pool.map(expert_span, _spans(M, 4 * threads)))
+        else:
+            y = recv_x
+        lap("expert")
+        out = np.empty((N, H), dtype=np.uint16)
+
+        def combine_span(ab):
+            a, b = ab
+            lib.orc_combine(_p(y), None, at(dst, a), at(tw, a), b - a, H, K, None, b - a, at(out, a))
+        list(pool.map(combine_span, spans))
+        lap("combine")
+    return dict(topk_idx=idx, topk_w=tw, margin=margin, M=M, recv_x=recv_x, recv_scale=recv_scale,
+                recv_src=recv_src, recv_w=recv_w, y=y, out=out, **lay)

@@ -76,6 +76,11 @@ def test_max_over_ranks_gloo_world2():
     assert res[0] == res[1] == [2.0, 5.0]
 
 
+def bench_host_cores():
+    import bench
+    return bench.host_cores()
+
+
 def test_reference_arm_json_line():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "tiny",
                         "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=300)
@@ -83,7 +88,7 @@ def test_reference_arm_json_line():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "GB/s"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
-    assert line["cpu_baseline"]["cores"] == 1 and line["cpu_baseline"]["host"]["nproc"] >= 1
+    assert line["cpu_baseline"]["cores"] == bench_host_cores() and line["cpu_baseline"]["host"]["nproc"] >= 1
     # both arms print the same metric, so their values compare directly
     import bench
     assert line["metric"] == bench.METRIC and line["higher_is_better"] is True
@@ -133,9 +138,13 @@ def test_ncu_traffic_parse_and_hash(tmp_path, monkeypatch):
     c = tmp_path / "ncu.csv"
     c.write_text(NCU_CSV)
     monkeypatch.setattr(metrics, "TRAFFIC_FILE", str(f))
-    metrics.record_traffic(str(c), "prefill", "ncu ...", "test")
-    assert metrics.stored_traffic("dispatch", "prefill") == 472_184_064 + 3_698_034_176
+    # a capture at 1024 tokens per rank scales by 4096 / 1024 to the prefill workload
+    ent = metrics.record_traffic(str(c), "prefill", "dispatch", "ncu ... -k regex:dispatch -c 1 ...", 1024)
+    assert ent["scale_to_workload"] == 4.0
+    assert metrics.stored_traffic("dispatch", "prefill") == 4 * (472_184_064 + 3_698_034_176)
+    assert metrics.stored_traffic("combine", "prefill") is None  # not recorded
     assert metrics.stored_traffic("dispatch", "large") is None
+    metrics.record_traffic(str(c), "prefill", "combine", "ncu ...", 1024)
     data = json.loads(f.read_text())
     data["prefill"]["combine"]["source_hash"] = "0" * 16  # captured from other sources
     f.write_text(json.dumps(data))

@@ -151,3 +151,21 @@ def test_combine_fused_dequant_equals_identity_expert_fp8_path():
     b = oracle.run_path(x, logits, w, fp8_combine_fused=True)
     oa, ob = _bf16_f32(a["out"]).double(), _bf16_f32(b["out"]).double()
     assert ((oa - ob).abs() <= 2 ** -7 * ob.abs() + 1e-6).all()
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "decode_ll", "skewed", "prefill"])
+def test_parallel_runner_equals_serial_oracle(name):
+    """The oracle over token chunks on host threads (the multi-core CPU
+    baseline) returns exactly the serial oracle's outputs."""
+    w = wl.WORKLOADS[name]
+    w = w.with_tokens(min(w.T, 32))
+    x, logits = wl.make_x(w, 1), wl.make_logits(w, 1)
+    a = oracle.run_path(x, logits, w)
+    b = oracle.run_path_parallel(x, logits, w, threads=3)
+    for key in ("topk_idx", "topk_w", "dst_row", "expert_off", "recv_x", "recv_scale", "recv_src", "recv_w",
+                "y", "out"):
+        if a[key] is None:
+            assert b[key] is None
+            continue
+        assert np.array_equal(np.asarray(a[key]).view(np.uint8), np.asarray(b[key]).view(np.uint8)), key
+    assert a["M"] == b["M"]

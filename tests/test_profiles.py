@@ -1,7 +1,11 @@
 """The profile summaries under profiles/ stay runnable: every bench command they
-quote parses with the current bench.py flags, every ncu command leaves the
-GPU clocks alone (--clock-control none), and the stored traffic figures name
-a workload and kernels the bench knows."""
+quote parses with the current bench.py flags, and every ncu command leaves
+the GPU clocks alone (--clock-control none). An ncu command that collects
+more than the launch list (gpu__time_duration.sum alone) names one kernel
+(-k), at most three launches (-c) and a small case (--tokens, or a workload
+that is small already). The stored traffic figures name a workload and
+kernels the bench knows, each from such a capture, scaled to full size by
+tokens."""
 import glob
 import json
 import os
@@ -56,7 +60,6 @@ def _summaries():
 def test_summaries_exist():
     names = [os.path.basename(p) for p in _summaries()]
     assert any(n.startswith("launches_") for n in names)
-    assert any(n.startswith("dram_traffic_") for n in names)
     assert any(n.startswith("ncu_full_") for n in names)
 
 
@@ -71,21 +74,44 @@ def test_quoted_commands_are_current(path):
         stripped = line.strip()
         if stripped.startswith("ncu ") and ("--metrics" in stripped or "--set" in stripped):
             assert "--clock-control none" in stripped, stripped
+            _check_capture_is_small(stripped)
     assert n_bench > 0, "no bench command quoted"
+
+
+SMALL_WORKLOADS = {"tiny", "decode", "decode_ll"}
+
+
+def _check_capture_is_small(cmd: str):
+    """A capture beyond the one-pass launch list: one kernel, <= 3 launches,
+    a small case."""
+    launch_list = re.search(r"--metrics\s+gpu__time_duration\.sum(\s|$)", cmd) is not None
+    if launch_list:
+        return
+    assert re.search(r"\s-k\s+\S+", cmd), f"no -k kernel filter: {cmd}"
+    m = re.search(r"\s-c\s+(\d+)", cmd)
+    assert m and int(m.group(1)) <= 3, f"more than 3 launches: {cmd}"
+    for args in _bench_args(cmd):
+        import bench
+        a = bench.parse_args(args)
+        assert a.tokens or a.config in SMALL_WORKLOADS, f"not a small case: {cmd}"
 
 
 def test_stored_traffic_entries():
     with open(metrics.TRAFFIC_FILE) as f:
         data = json.load(f)
     assert set(data) <= set(wl.WORKLOADS)
+    import bench
     for wname, ent in data.items():
-        assert "--clock-control none" in ent["command"], wname
-        args = _bench_args(ent["command"])
-        assert len(args) == 1, wname
-        import bench
-        a = bench.parse_args(args[0])
-        assert a.config == wname
-        for kern in ("layout", "dispatch", "combine"):
-            k = ent[kern]
-            assert k["dram_bytes_per_launch"] == k["dram_read"] + k["dram_write"]
+        for kern, k in ent.items():
+            assert kern in ("layout", "dispatch", "combine"), (wname, kern)
+            cmd = k["command"]
+            assert "--clock-control none" in cmd, (wname, kern)
+            _check_capture_is_small(cmd)
+            args = _bench_args(cmd)
+            assert len(args) == 1, (wname, kern)
+            a = bench.parse_args(args[0])
+            assert a.config == wname and a.tokens == k["captured_tokens_per_rank"]
+            scale = wl.WORKLOADS[wname].T / k["captured_tokens_per_rank"]
+            assert k["scale_to_workload"] == scale
+            assert k["dram_bytes_per_launch"] == round((k["dram_read"] + k["dram_write"]) * scale)
             assert len(k["source_hash"]) == 16

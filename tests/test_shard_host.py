@@ -90,7 +90,7 @@ def test_peer_tables_keep_offsets():
 
 
 class _FakeSymmMem:
-    """Stand-in for torch symmetric memory on CPU ranks: a plain workspace,
+    """Stand-in for the peer-memory provider on CPU ranks: a plain workspace,
     and made-up per-rank base addresses as the peer mappings."""
 
     def __init__(self, R):
@@ -162,19 +162,23 @@ def _driver_rank_main(rank: int, world: int, port: int, q):
     try:
         from combine_top_group_b200 import shard
         fake = _FakeEp(W2)
-        drv = shard.DistributedRank(W2, torch.device("cpu"), ep_lib=fake, symm_mem_lib=_FakeSymmMem(world))
+        drv = shard.DistributedRank(W2, torch.device("cpu"), ep_lib=fake, peer_mem=_FakeSymmMem(world))
         real_barrier = drv.barrier
         drv.barrier = lambda: (fake.calls.append(("barrier",)), real_barrier())
         logits = torch.from_numpy(wl.make_logits(W2, 0)[rank * W2.T:(rank + 1) * W2.T].copy())
         drv.step(torch.zeros(W2.T, W2.H), logits, torch.zeros(W2.T, W2.H))
-        q.put((rank, fake.calls))
+        calls = list(fake.calls)
+        fake.calls.clear()
+        drv.step(torch.zeros(W2.T, W2.H), logits, torch.zeros(W2.T, W2.H),
+                 expert=lambda x, scale, rows: fake.calls.append(("expert", rows)))
+        q.put((rank, calls, [c[0] for c in fake.calls]))
     finally:
         dist.destroy_process_group()
 
 
 def test_distributed_driver_order_exchange_and_tables():
     """DistributedRank on 2 gloo ranks, with stand-ins for the kernels and for
-    symmetric memory: the calls come in the method's order, the count rows
+    peer memory: the calls come in the method's order, the count rows
     are exchanged before placement, and the peer tables point at the same
     offset inside every rank's (stand-in) workspace."""
     import oracle
@@ -184,10 +188,11 @@ def test_distributed_driver_order_exchange_and_tables():
     procs = [ctx.Process(target=_driver_rank_main, args=(r, W2.R, port, q)) for r in range(W2.R)]
     for p in procs:
         p.start()
-    res = {}
+    res, with_expert = {}, {}
     for _ in procs:
-        r, calls = q.get(timeout=120)
+        r, calls, kinds2 = q.get(timeout=120)
         res[r] = calls
+        with_expert[r] = kinds2
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
@@ -196,8 +201,10 @@ def test_distributed_driver_order_exchange_and_tables():
     bases = _FakeSymmMem(W2.R).bases
     for r, calls in res.items():
         kinds = [c[0] for c in calls]
-        # barriers: before dispatch (rows free), after it (rows written), after the experts
-        assert kinds == ["layout", "place", "barrier", "dispatch", "barrier", "barrier", "combine"]
+        # barriers: before dispatch (rows free), after it (rows written)
+        assert kinds == ["layout", "place", "barrier", "dispatch", "barrier", "combine"]
+        # an expert step that rewrites the rows gets its own barrier before the combine
+        assert with_expert[r] == ["layout", "place", "barrier", "dispatch", "barrier", "expert", "barrier", "combine"]
         layout, place, disp, comb = (c for c in calls if c[0] != "barrier")
         assert layout[1] == r and place[1] == r and disp[1] == r and comb[1] == r
         assert np.array_equal(place[3], want_cnt)  # all-gathered before placement
@@ -206,6 +213,18 @@ def test_distributed_driver_order_exchange_and_tables():
         assert disp[5] == [b + 4096 for b in bases] and disp[6] == [b + 8192 for b in bases]
         assert disp[4] is None and comb[4] is None  # bf16: no scale tables
         assert comb[3] == [b + 256 for b in bases]  # combine reads every rank's rows
+
+
+def test_alltoallv_splits_from_counts():
+    """Rows rank s sends to rank d = sum of cnt_all[s][e] over d's experts;
+    rows it receives from s' = the same sum over its own experts."""
+    from combine_top_group_b200.shard import alltoallv_splits
+    R, L = 3, 2
+    cnt = torch.arange(R * R * L, dtype=torch.int32).view(R, R * L)  # cnt[s][e] = s*6 + e
+    send, recv = alltoallv_splits(cnt, 1, L)
+    assert send == [6 + 7, 8 + 9, 10 + 11]
+    assert recv == [2 + 3, 8 + 9, 14 + 15]
+    assert sum(send) == int(cnt[1].sum())
 
 
 def test_shard_view_matches_hand_worked_example(golden):
