@@ -150,3 +150,22 @@ def test_ncu_traffic_parse_and_hash(tmp_path, monkeypatch):
     f.write_text(json.dumps(data))
     assert metrics.stored_traffic("combine", "prefill") is None
     assert metrics.stored_traffic("dispatch", "prefill") is not None
+
+
+def test_ep_workload_one_rank_per_gpu():
+    """--gpus N runs the workload with R = N ranks, each keeping the
+    workload's T tokens (weak scaling); E must split evenly over the ranks."""
+    import pytest
+
+    import bench
+    w = wl.WORKLOADS["prefill"]
+    for n in (1, 2, 4, 8):
+        e = bench.ep_workload(w, n)
+        assert (e.R, e.T, e.E, e.K, e.H, e.G, e.KG) == (n, w.T, w.E, w.K, w.H, w.G, w.KG)
+        assert e.L == w.E // n
+    with pytest.raises(SystemExit):
+        bench.ep_workload(w, 3)  # 256 experts do not split over 3 ranks
+    with pytest.raises(SystemExit):
+        bench.ep_workload(wl.WORKLOADS["decode_ll"], 2)  # the low-latency layout has no per-GPU path
+    a = bench.parse_args(["--gpus", "8", "--replicas"])
+    assert a.replicas and not a.one_rank_per_gpu
