@@ -164,9 +164,13 @@ __global__ void __launch_bounds__(512) dispatch_bf16_kernel(DispatchParams p, Re
         }
         __syncthreads();  // s_row is rewritten by the next token
     }
-    // stores into peer memory reach the other GPUs before the kernel ends, so
-    // a collective that follows it on the stream orders them for the readers
-    if constexpr (Recv::kPeer) __threadfence_system();
+    // Stores into peer memory reach the other GPUs before the kernel ends, so
+    // a collective that follows it on the stream orders them for the readers.
+    // The loop's last barrier orders every thread's stores before thread 0,
+    // whose system-scope fence (cumulative) then covers the whole CTA.
+    if constexpr (Recv::kPeer) {
+        if (threadIdx.x == 0) __threadfence_system();
+    }
 }
 
 template <int VPT, class Recv>
@@ -229,7 +233,9 @@ __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchParams p, Rec
         }
         __syncthreads();
     }
-    if constexpr (Recv::kPeer) __threadfence_system();  // as in dispatch_bf16_kernel
+    if constexpr (Recv::kPeer) {  // as in dispatch_bf16_kernel
+        if (threadIdx.x == 0) __threadfence_system();
+    }
 }
 
 template <class Recv>
