@@ -46,6 +46,7 @@ struct DispatchParams {
     const uint8_t* dst_rank;  // [N, K] destination rank of each slot (PeerRecv only)
     int num_peers;            // entries of the PeerRecv tables
     int64_t g_base;           // global id of local token 0 (recv_src)
+    int ordered;              // write a token's rows in (destination rank, row) order
     uint32_t* err;
 };
 
@@ -112,7 +113,11 @@ __device__ __forceinline__ void stage_rows(const DispatchParams& p, const Recv& 
 // in flight hold consecutive tokens, whose rows for one expert are adjacent,
 // so in this order their writes meet in fewer places at a time (measured on
 // B200: prefill dispatch 687 -> 678 us). Threads t < K, after s_row / s_rank
-// are visible.
+// are visible. With many CTAs in flight (a full grid, or a num_sms cap of at
+// least half the SMs) the CTAs write in this order. Under a smaller cap each
+// CTA loops over hundreds of tokens and pays the extra barrier on each, and
+// slot order is faster (measured on B200, prefill: 20 SMs 1318 against 1390
+// us, 37 SMs 847 against 881 us; at 74 SMs 779 ordered against 787).
 template <class Recv>
 __device__ __forceinline__ void order_rows(int K, const int32_t* s_row, const int32_t* s_rank, int32_t* s_ord) {
     const int t = threadIdx.x;
@@ -149,10 +154,12 @@ __global__ void __launch_bounds__(512) dispatch_bf16_kernel(DispatchParams p, Re
             if (c < nv) v[j] = ld256_stream(p.x + g * rb + (size_t)c * 32);
         }
         __syncthreads();
-        order_rows<Recv>(p.K, s_row, s_rank, s_ord);
-        __syncthreads();
+        if (p.ordered) {  // uniform over the grid
+            order_rows<Recv>(p.K, s_row, s_rank, s_ord);
+            __syncthreads();
+        }
         for (int i = 0; i < p.K; ++i) {
-            const int k = s_ord[i];
+            const int k = p.ordered ? s_ord[i] : i;
             const int32_t r = s_row[k];
             if (r < 0) continue;
             uint8_t* dst = rv.x_of(Recv::kPeer ? s_rank[k] : 0) + (size_t)r * rb;
@@ -213,10 +220,12 @@ __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchParams p, Rec
             sc[j] = __fdiv_rn(amax, 448.0f);
         }
         __syncthreads();
-        order_rows<Recv>(p.K, s_row, s_rank, s_ord);
-        __syncthreads();
+        if (p.ordered) {  // uniform over the grid
+            order_rows<Recv>(p.K, s_row, s_rank, s_ord);
+            __syncthreads();
+        }
         for (int i = 0; i < p.K; ++i) {
-            const int k = s_ord[i];
+            const int k = p.ordered ? s_ord[i] : i;
             const int32_t r = s_row[k];
             if (r < 0) continue;
             const int d = Recv::kPeer ? s_rank[k] : 0;
@@ -304,8 +313,10 @@ void (*fp8_kernel_of(int vpt))(DispatchParams, Recv) {
 }
 
 template <class Recv>
-cudaError_t launch_any(const DispatchParams& p, const Recv& rv, bool fp8, int sm_cap, int full_sms,
+cudaError_t launch_any(const DispatchParams& p0, const Recv& rv, bool fp8, int sm_cap, int full_sms,
                        cudaStream_t st) {
+    DispatchParams p = p0;
+    p.ordered = 2 * sm_cap >= full_sms ? 1 : 0;
     int threads, vpt;
     shape_of(p.H, fp8 ? 2 : 1, &threads, &vpt);
     if (!fp8) {

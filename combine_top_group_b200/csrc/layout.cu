@@ -82,21 +82,22 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
 }
 
 // Bounded grid-wide barrier (the grid is co-resident: cooperative launch).
+// The CTA barrier orders every thread's writes before thread 0, whose
+// release-add publishes them (cumulatively) at GPU scope; the acquire loads
+// of the spin order the CTA's later reads after every other CTA's arrival.
 __device__ void grid_barrier(uint32_t* arrive, uint32_t target, uint32_t* err,
                              unsigned long long limit_ns = kWaitLimitNs) {
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(arrive, 1u);
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(arrive) : "memory");
         const unsigned long long t0 = globaltimer_ns();
         while (ld_acquire(arrive) < target) {
             if (globaltimer_ns() - t0 > limit_ns) {
                 set_error(err, EP_DEVERR_TIMEOUT);
                 break;
             }
-            __nanosleep(64);
+            __nanosleep(32);
         }
-        __threadfence();
     }
     __syncthreads();
 }
@@ -629,15 +630,13 @@ __global__ void __launch_bounds__(kThreads, EPL >= 16 ? 2 : 4) layout_kernel(Lay
         }
     }
 
-    // the last CTA out resets the barrier words for the next launch
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        if (atomicAdd(p.bar + 1, 1u) == (uint32_t)p.nb - 1u) {
-            p.bar[0] = 0u;
-            p.bar[1] = 0u;
-            __threadfence();
-        }
+    // The last CTA out resets the barrier words for the next launch. Every
+    // CTA counts itself out after leaving the last grid barrier, so when the
+    // count is full no CTA reads the words again in this launch; the end of
+    // the kernel publishes the reset to the next one.
+    if (threadIdx.x == 0 && atomicAdd(p.bar + 1, 1u) == (uint32_t)p.nb - 1u) {
+        p.bar[0] = 0u;
+        p.bar[1] = 0u;
     }
 }
 
