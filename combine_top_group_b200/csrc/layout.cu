@@ -262,7 +262,6 @@ __device__ __forceinline__ void load_logits(const LayoutParams& p, int64_t g, in
 struct WarpStage {
     int32_t e[32];     // expert of each slot (-1: none)
     uint32_t key[32];  // order key of the slot's logit
-    uint32_t mx[32];   // per token: key of its largest logit
     double z[32];      // per token: sum over all experts of exp(l - max) (plain softmax)
     double s[32];      // per slot: unnormalised weight
     uint32_t rb[32];   // per slot: bit of its destination rank
@@ -302,13 +301,15 @@ __device__ __forceinline__ void select_token(const LayoutParams& p, int lane, co
     }
 
     // top-K: K rounds of warp max. Equal keys go to the lowest lane, which
-    // holds the lowest expert ids; within a lane top3_of keeps id order.
+    // holds the lowest expert ids; within a lane top3_of keeps id order. The
+    // winner is the lane holding the maximum with no lower lane holding it.
+    // Slot 0's key is the token's largest logit (the softmax max).
     const int base = j * p.K;
+    const unsigned below = (1u << lane) - 1u;
     for (int k = 0; k < p.K; ++k) {
         const uint32_t wk = __reduce_max_sync(FULL, a);
-        const int win = __ffs(__ballot_sync(FULL, a == wk)) - 1;
-        if (k == 0 && lane == 0) st.mx[j] = wk;
-        if (lane == win) {
+        const unsigned tie = __ballot_sync(FULL, a == wk);
+        if (a == wk && (tie & below) == 0u) {
             st.e[base + k] = (wk != 0u) ? e0 + pa : -1;
             st.key[base + k] = wk;
             if (wk != 0u) {  // pop this lane's head
@@ -326,7 +327,7 @@ __device__ __forceinline__ void select_token(const LayoutParams& p, int lane, co
     if (p.route == EP_ROUTE_SOFTMAX) {
         // the normaliser of the plain softmax: every expert, fp64
         __syncwarp();
-        const double mx = (double)key_value(st.mx[j]);
+        const double mx = (double)key_value(st.key[base]);
         double z = 0.0;
 #pragma unroll
         for (int i = 0; i < EPL; ++i)  // softmax routes never zero keys: key i is logit i
@@ -370,7 +371,7 @@ __device__ __forceinline__ void finish_group(const LayoutParams& p, int lane, in
         double sv = 0.0;
         if (e >= 0) {
             const double l = (double)key_value(st.key[lane]);
-            sv = (p.route == EP_ROUTE_GROUP_SIGMOID) ? sigmoid_d(l) : exp(l - (double)key_value(st.mx[jj]));
+            sv = (p.route == EP_ROUTE_GROUP_SIGMOID) ? sigmoid_d(l) : exp(l - (double)key_value(st.key[jj * K]));
         }
         st.s[lane] = sv;
         __syncwarp();
