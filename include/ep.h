@@ -353,7 +353,10 @@ ep_status_t ep_shard_place(ep_buffer_t *buf, int rank, int T, void *stream);
  * be usable from this GPU: peer access enabled, or IPC or symmetric-memory
  * mappings. Every entry is non-NULL. peer_recv_x entries are 32-byte aligned;
  * peer_recv_scale may be NULL without EP_FLAG_FP8. d_x: bf16 [T, H], 32-byte
- * aligned. Needs ep_shard_place first. Errors: EP_ERR_INVALID. */
+ * aligned. Needs ep_shard_place first. The kernel makes its stores complete
+ * at system scope before it ends, so a collective that follows it on
+ * `stream` (the barrier of step 6) orders them for the receiving ranks.
+ * Errors: EP_ERR_INVALID. */
 ep_status_t ep_shard_dispatch(ep_buffer_t *buf, int rank, int T, const void *d_x,
                               void *const *peer_recv_x, float *const *peer_recv_scale,
                               int32_t *const *peer_recv_src, float *const *peer_recv_w, void *stream);
