@@ -40,16 +40,35 @@ def _bf16_f64(bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).double().numpy()
 
 
-def _close(got, ref):
-    g, r = _bf16_f64(got), _bf16_f64(ref)
-    assert (np.abs(g - r) <= 2.0 ** -7 * np.abs(r) + 1e-3).all()
-    assert (got == ref).mean() >= 0.999
+def _close(got, ref, chunk=8192):
+    """Every element within the tolerance and >= 99.9% bit-exact, compared in
+    row chunks (full-size arrays would not fit as fp64)."""
+    exact = 0
+    for a in range(0, got.shape[0], chunk):
+        gb, rb = got[a:a + chunk], ref[a:a + chunk]
+        g, r = _bf16_f64(gb), _bf16_f64(rb)
+        assert (np.abs(g - r) <= 2.0 ** -7 * np.abs(r) + 1e-3).all(), f"rows {a}.."
+        exact += int((gb == rb).sum())
+    assert exact >= 0.999 * got.size
 
 
-CASES = [("tiny", None, 0), ("decode", None, 1), ("skewed", 512, 0), ("prefill", 256, 2)]
+def _equal_rows(dev, ref, what, chunk=32768):
+    """dev (device rows) equals ref (host rows) bit for bit, copied back in
+    chunks."""
+    assert dev.shape[0] == ref.shape[0]
+    for a in range(0, ref.shape[0], chunk):
+        got = _host(dev[a:a + chunk])
+        exp = ref[a:a + chunk]
+        if got.dtype == np.float32:
+            got, exp = got.view(np.uint32), exp.view(np.uint32)
+        assert np.array_equal(got, exp), f"{what}: rows {a}.."
 
 
-@pytest.mark.parametrize("name,T,seed", CASES, ids=[c[0] for c in CASES])
+# prefill at T = 4096 is the full-size workload: D = 129 866 dedup rows, M = 262 144 expert rows
+CASES = [("tiny", None, 0), ("decode", None, 1), ("skewed", 512, 0), ("prefill", 256, 2), ("prefill", None, 1)]
+
+
+@pytest.mark.parametrize("name,T,seed", CASES, ids=[f"{c[0]}-{c[1] or 'full'}" for c in CASES])
 @pytest.mark.parametrize("fused", [False, True], ids=["y_bf16", "y_fused"])
 def test_dedup_path_parity(cuda, name, T, seed, fused):
     ep, runner = cuda
@@ -98,17 +117,17 @@ def test_dedup_path_parity(cuda, name, T, seed, fused):
     assert np.array_equal(_host(dd["dd_topk_idx"][:D]), o_d["recv_topk_idx"])
     gw, ow = _host(dd["dd_topk_w"][:D]).astype(np.float64), o_d["recv_topk_w"]
     assert (np.abs(gw - ow) <= 2.0 ** -22 * np.abs(ow)).all()
-    assert np.array_equal(_host(dd["dd_x"][:D]), o_d["recv_x"])
+    _equal_rows(dd["dd_x"][:D], o_d["recv_x"], "dedup rows")
     if w.fp8:
-        assert np.array_equal(_host(dd["dd_scale"][:D]).view(np.uint32), o_d["recv_scale"].view(np.uint32))
+        _equal_rows(dd["dd_scale"][:D], o_d["recv_scale"], "dedup scales")
 
     # permute -> the standard expert-grouped receive buffers
     pipe.permute()
     assert pipe.check_errors() == 0
-    assert np.array_equal(_host(pipe.recv["recv_x"][:M]), o_rx)
+    _equal_rows(pipe.recv["recv_x"][:M], o_rx, "expert rows")
     assert np.array_equal(_host(pipe.recv["recv_src"][:M]), o_src)
     if w.fp8:
-        assert np.array_equal(_host(pipe.recv["recv_scale"][:M]).view(np.uint32), o_rs.view(np.uint32))
+        _equal_rows(pipe.recv["recv_scale"][:M], o_rs, "expert scales")
 
     # local reduce + cross-rank combine
     if w.fp8 and not fused:
@@ -117,6 +136,7 @@ def test_dedup_path_parity(cuda, name, T, seed, fused):
     pipe.combine_dedup()
     assert pipe.check_errors() == 0
     _close(_host(dd["partial"][:D]), o_part)
+    del o_rx, o_d
     _close(_host(pipe.out), o_out)
 
 
