@@ -31,6 +31,13 @@ namespace {
 // at 80 registers; 1715 -> 1604 us against 4 warps on the large shape.
 constexpr int kBf16Threads = 128;
 constexpr int kFp8Threads = 64;
+// Under a num_sms cap of n the grid is at most n CTAs, so that no more than n
+// SMs run the kernel (the block scheduler places CTAs breadth-first: 4n small
+// CTAs would occupy 4n SMs). Each CTA then holds as many of the token groups
+// above as one SM does: kSub groups of the same size, each looping over its
+// own tokens.
+constexpr int kBf16Sub = 4;   // 512 threads, 128 registers each: the register file
+constexpr int kFp8Sub = 12;   // 768 threads at 80 registers
 
 struct CombineParams {
     int64_t N;
@@ -76,22 +83,25 @@ __device__ __forceinline__ const uint8_t* peer_row(const CombineParams& p, const
 }
 
 template <class Y>
-__device__ __forceinline__ void report_rows(const CombineParams& p, int64_t g) {
-    if (threadIdx.x < p.K) {
-        const int32_t r = __ldg(p.dst_row + g * p.K + threadIdx.x);
+__device__ __forceinline__ void report_rows(const CombineParams& p, int64_t g, int tid) {
+    if (tid < p.K) {
+        const int32_t r = __ldg(p.dst_row + g * p.K + tid);
         bool bad = r >= p.m_max;
-        if constexpr (Y::kPeer) bad = bad || (r >= 0 && __ldg(p.dst_rank + g * p.K + threadIdx.x) >= p.num_peers);
+        if constexpr (Y::kPeer) bad = bad || (r >= 0 && __ldg(p.dst_rank + g * p.K + tid) >= p.num_peers);
         if (bad) set_error(p.err, EP_DEVERR_ROW_BOUNDS);
     }
 }
 
-template <class Y>
-__global__ void __launch_bounds__(kBf16Threads) combine_bf16_kernel(CombineParams p, Y py) {
+// SUB groups of kBf16Threads threads per CTA; group j of CTA b takes tokens
+// b * SUB + j, then strides by the grid's groups.
+template <class Y, int SUB>
+__global__ void __launch_bounds__(kBf16Threads * SUB) combine_bf16_kernel(CombineParams p, Y py) {
     const int nvec = p.H / 16;  // 32-byte vectors: 16 bf16 channels
     const size_t rb = (size_t)p.H * 2;
-    for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {  // grid-stride when num_sms caps the grid
-        report_rows<Y>(p, g);
-        for (int v = threadIdx.x; v < nvec; v += kBf16Threads) {
+    const int sub = threadIdx.x / kBf16Threads, tid = threadIdx.x - sub * kBf16Threads;
+    for (int64_t g = (int64_t)blockIdx.x * SUB + sub; g < p.N; g += (int64_t)gridDim.x * SUB) {
+        report_rows<Y>(p, g, tid);
+        for (int v = tid; v < nvec; v += kBf16Threads) {
             float acc[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
@@ -131,14 +141,16 @@ __global__ void __launch_bounds__(kBf16Threads) combine_bf16_kernel(CombineParam
     }
 }
 
-template <class Y>
-__global__ void __launch_bounds__(kFp8Threads) combine_fp8_kernel(CombineParams p, Y py) {
+// SUB groups of kFp8Threads threads per CTA, as in combine_bf16_kernel.
+template <class Y, int SUB>
+__global__ void __launch_bounds__(kFp8Threads * SUB) combine_fp8_kernel(CombineParams p, Y py) {
     const int nvec = p.H / 16;  // 16 e4m3 channels (16 B) per vector
     const int nb = p.H / 128;
     const size_t rb = (size_t)p.H;
-    for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {
-        report_rows<Y>(p, g);
-        for (int v = threadIdx.x; v < nvec; v += kFp8Threads) {
+    const int sub = threadIdx.x / kFp8Threads, tid = threadIdx.x - sub * kFp8Threads;
+    for (int64_t g = (int64_t)blockIdx.x * SUB + sub; g < p.N; g += (int64_t)gridDim.x * SUB) {
+        report_rows<Y>(p, g, tid);
+        for (int v = tid; v < nvec; v += kFp8Threads) {
             // acc[j] holds channels 2j and 2j+1 as an fp32 pair
             uint64_t acc[8];
 #pragma unroll
@@ -202,23 +214,276 @@ __global__ void __launch_bounds__(kFp8Threads) combine_fp8_kernel(CombineParams 
     }
 }
 
+// ---- bf16 combine under a num_sms cap: a TMA bulk-copy pipeline ------------
+//
+// Under a num_sms cap the grid is one CTA per SM, and the register gather
+// above keeps at most 128 KB per SM in flight (512 threads, 8 loads of 32 B
+// each). Here the bulk-copy (TMA) engine moves the rows into shared memory
+// instead: 4 stages, each K row segments of kTmaChunk channels (56 KB at
+// K = 8), so the threads issue only the arithmetic. Measured on B200 at the
+// prefill shape (8 x 4096 tokens, H = 7168, K = 8): 2.3-2.6 ms against 2.9 ms
+// for the register gather at 20 SMs, 0.69-0.72 against 0.88 ms at 74 SMs.
+// More and smaller stages (2-4 KB copies, 6-12 stages) and whole-row copies
+// (14 KB, 4 slots per stage) were slower.
+//
+// One CTA per SM: kTmaConsumers consumer threads and one producer warp. A
+// unit is one token and one block of kTmaChunk channels; CTA b takes a
+// contiguous range of tokens, all blocks of each. The producer warp reads the
+// (row, weight) pairs of kTmaBatch tokens at once, lane 8j + k holding slot k
+// of token j (one coalesced load of each table), a batch ahead of the copies
+// so that their latency overlaps the copies of the batch before. For a unit it
+// writes the token, the slot mask and the weights next to the stage, arms the
+// stage's "full" barrier with the bytes to come, and each lane of the token's
+// group with an unmasked slot issues that row's bulk copy. Every consumer
+// warp, after reading a stage, arrives on its "empty" barrier, which frees
+// the stage for the producer. The sum is the register kernel's: an fp32 fma
+// chain over k ascending, one bf16 rounding.
+//
+// Every wait is bounded (kWaitLimitNs): a wait that gives up sets
+// EP_DEVERR_TIMEOUT, and before the CTA returns the producer waits, bounded
+// again, for the copies it issued, so none lands in shared memory after the
+// CTA has left. A consumer arrives on "empty" only after its "full" wait
+// succeeded, so a stage is refilled only once its previous copies landed:
+// only the last kTmaStages units issued can still be in flight.
+constexpr int kTmaConsumers = 224;
+constexpr int kTmaThreads = kTmaConsumers + 32;
+constexpr int kTmaStages = 4;
+constexpr int kTmaMaxK = 8;
+constexpr int kTmaBatch = 32 / kTmaMaxK;  // tokens whose slots the producer warp reads at once
+constexpr int kTmaVec = 16;               // channels per consumer: 8 or 16
+constexpr int kTmaChunk = kTmaConsumers * kTmaVec;  // channels per unit
+constexpr size_t kTmaStageBytes = (size_t)kTmaMaxK * kTmaChunk * 2;
+// What the producer tells the consumers about the unit in a stage.
+struct TmaUnit {
+    int64_t g;          // token
+    int cb;             // channel block
+    uint32_t mask;      // bit k: slot k's row is in the stage
+    float w[kTmaMaxK];  // the slots' weights
+};
+constexpr size_t kTmaSmem =
+    kTmaStages * kTmaStageBytes + 2 * kTmaStages * sizeof(uint64_t) + kTmaStages * sizeof(TmaUnit);
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_arrive(uint64_t* bar, uint32_t tx) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(tx) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+                 : "=r"(ok)
+                 : "r"(smem_addr(bar)), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+// Waits for the phase of `bar` with this parity to complete; false if it
+// has not after kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    return true;
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+
+// One lane's slot (token g, slot k), as the producer warp reads it: every
+// load is issued without waiting on another, so a batch's loads overlap.
+struct TmaSlot {
+    const uint8_t* src;  // start of the row in y, nullptr when masked or refused
+    float w;
+    bool bad;  // a row the buffer cannot hold, or a rank the table lacks
+};
+
+template <class Y>
+__device__ __forceinline__ TmaSlot tma_slot(const CombineParams& p, const Y& py, int64_t g, int k, size_t rb) {
+    const int64_t at = g * p.K + k;
+    const int32_t r = __ldg(p.dst_row + at);
+    TmaSlot sl;
+    sl.w = __ldg(p.topk_w + at);
+    sl.bad = r >= p.m_max;
+    const bool use = r >= 0 && !sl.bad;
+    if constexpr (Y::kPeer) {
+        const int d = __ldg(p.dst_rank + at);
+        const bool known = d >= 0 && d < p.num_peers;
+        sl.bad = sl.bad || (r >= 0 && !known);
+        sl.src = (use && known) ? py.y[d] + (size_t)r * rb : nullptr;
+    } else {
+        sl.src = use ? p.y + (size_t)r * rb : nullptr;
+    }
+    return sl;
+}
+
+template <class Y>
+__global__ void __launch_bounds__(kTmaThreads, 1) combine_bf16_tma_kernel(CombineParams p, Y py) {
+    extern __shared__ __align__(128) uint8_t sm[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + kTmaStages * kTmaStageBytes);
+    uint64_t* empty = full + kTmaStages;
+    TmaUnit* meta = reinterpret_cast<TmaUnit*>(empty + kTmaStages);
+    const int t = threadIdx.x, lane = t & 31;
+    const int nblk = (p.H + kTmaChunk - 1) / kTmaChunk;
+    const size_t rb = (size_t)p.H * 2;
+    // this CTA's tokens [g0, g1)
+    const int64_t g0 = (int64_t)blockIdx.x * p.N / gridDim.x, g1 = (int64_t)(blockIdx.x + 1) * p.N / gridDim.x;
+    const int64_t mine = (g1 - g0) * nblk;
+    if (t == 0) {
+        for (int s = 0; s < kTmaStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kTmaConsumers / 32);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (t >= kTmaConsumers) {  // the producer warp
+        const int j = lane / kTmaMaxK, k = lane % kTmaMaxK;  // token j of a batch, slot k
+        const bool slot = k < p.K;
+        int64_t issued = 0;
+        bool ok = true;
+        // the batch at gb, and the next one, read while this one's copies go out
+        TmaSlot cur{nullptr, 0.0f, false};
+        if (slot && g0 + j < g1) cur = tma_slot<Y>(p, py, g0 + j, k, rb);
+        for (int64_t gb = g0; gb < g1 && ok; gb += kTmaBatch) {
+            TmaSlot next{nullptr, 0.0f, false};
+            if (slot && gb + kTmaBatch + j < g1) next = tma_slot<Y>(p, py, gb + kTmaBatch + j, k, rb);
+            if (cur.bad) set_error(p.err, EP_DEVERR_ROW_BOUNDS);
+            const uint32_t have = __ballot_sync(0xffffffffu, cur.src != nullptr);
+            for (int jj = 0; jj < kTmaBatch && gb + jj < g1 && ok; ++jj) {
+                const uint32_t mask = (have >> (jj * kTmaMaxK)) & ((1u << kTmaMaxK) - 1);
+                for (int cb = 0; cb < nblk; ++cb) {
+                    const int64_t i = issued;
+                    const int s = (int)(i % kTmaStages);
+                    if (i >= kTmaStages && lane == 0) ok = mbar_wait(&empty[s], (uint32_t)((i / kTmaStages - 1) & 1));
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) {
+                        if (lane == 0) set_error(p.err, EP_DEVERR_TIMEOUT);
+                        break;
+                    }
+                    const uint32_t bytes = (uint32_t)min(kTmaChunk, p.H - cb * kTmaChunk) * 2;
+                    TmaUnit& m = meta[s];
+                    if (j == jj) m.w[k] = cur.w;
+                    __syncwarp();
+                    if (lane == 0) {
+                        m.g = gb + jj;
+                        m.cb = cb;
+                        m.mask = mask;
+                        // releases the metadata with the arrival
+                        mbar_expect_arrive(&full[s], (uint32_t)__popc(mask) * bytes);
+                    }
+                    __syncwarp();
+                    if (j == jj && cur.src != nullptr)
+                        bulk_load(sm + (size_t)s * kTmaStageBytes + (size_t)k * kTmaChunk * 2,
+                                  cur.src + (size_t)cb * kTmaChunk * 2, bytes, &full[s]);
+                    issued = i + 1;
+                }
+            }
+            cur = next;
+        }
+        // copies issued and possibly not landed: only the last kTmaStages units
+        if (lane == 0)
+            for (int64_t i = (issued > kTmaStages ? issued - kTmaStages : 0); i < issued; ++i)
+                if (!mbar_wait(&full[i % kTmaStages], (uint32_t)((i / kTmaStages) & 1))) break;
+        return;
+    }
+
+    for (int64_t i = 0; i < mine; ++i) {
+        const int s = (int)(i % kTmaStages);
+        if (!mbar_wait(&full[s], (uint32_t)((i / kTmaStages) & 1))) {
+            set_error(p.err, EP_DEVERR_TIMEOUT);
+            break;
+        }
+        const TmaUnit& m = meta[s];
+        const int64_t g = m.g;
+        const uint32_t mask = m.mask;
+        const int v = m.cb * kTmaConsumers + t;  // this thread's kTmaVec channels
+        // the stage's rows into registers, then the stage goes back to the producer
+        const uint8_t* stage = sm + (size_t)s * kTmaStageBytes + (size_t)t * kTmaVec * 2;
+        uint32_t q[kTmaMaxK][kTmaVec / 2];
+        float w[kTmaMaxK];
+        const bool mine_v = v * kTmaVec < p.H;
+#pragma unroll
+        for (int k = 0; k < kTmaMaxK; ++k) {
+            w[k] = m.w[k];
+            if (mine_v && ((mask >> k) & 1u)) {
+#pragma unroll
+                for (int h = 0; h < kTmaVec / 8; ++h) {
+                    const uint4 a = *reinterpret_cast<const uint4*>(stage + (size_t)k * kTmaChunk * 2 + h * 16);
+                    q[k][4 * h] = a.x, q[k][4 * h + 1] = a.y, q[k][4 * h + 2] = a.z, q[k][4 * h + 3] = a.w;
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        if (mine_v) {
+            uint64_t acc[kTmaVec / 2];  // channel pairs (2j, 2j+1) as fp32 pairs
+#pragma unroll
+            for (int j = 0; j < kTmaVec / 2; ++j) acc[j] = 0ull;
+#pragma unroll
+            for (int k = 0; k < kTmaMaxK; ++k) {
+                if (!((mask >> k) & 1u)) continue;
+                const uint64_t w2 = f32x2_pack(w[k], w[k]);
+#pragma unroll
+                for (int j = 0; j < kTmaVec / 2; ++j)  // per channel: acc = fma(w, y, acc), rounded as the scalar chain
+                    acc[j] = f32x2_fma_rn(w2, f32x2_pack(bf16lo(q[k][j]), bf16hi(q[k][j])), acc[j]);
+            }
+            uint32_t o[kTmaVec / 2];
+#pragma unroll
+            for (int j = 0; j < kTmaVec / 2; ++j) {
+                const float2 a = f32x2_unpack(acc[j]);
+                o[j] = pack_bf16x2(a.x, a.y);
+            }
+            uint8_t* dst = p.out + (size_t)g * rb + (size_t)v * kTmaVec * 2;
+            if constexpr (kTmaVec == 16) {
+                u32x8 o8;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) o8.v[j] = o[j];
+                st256(dst, o8);
+            } else {
+                *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+        }
+    }
+}
+
+template <class Y>
+cudaError_t launch_tma(const CombineParams& p, const Y& py, int sm_cap, cudaStream_t st) {
+    // per launch: the attribute belongs to the current device
+    cudaError_t e = cudaFuncSetAttribute(combine_bf16_tma_kernel<Y>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kTmaSmem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = p.N < sm_cap ? p.N : sm_cap;  // one CTA per SM
+    combine_bf16_tma_kernel<Y><<<(unsigned)grid, kTmaThreads, kTmaSmem, st>>>(p, py);
+    return cudaGetLastError();
+}
+
 template <class Y>
 cudaError_t launch_y(const ep_buffer& b, const CombineParams& p, const Y& py, bool fp8, cudaStream_t st) {
-    auto kern = fp8 ? combine_fp8_kernel<Y> : combine_bf16_kernel<Y>;
-    const int threads = fp8 ? kFp8Threads : kBf16Threads;
-    int64_t grid = p.N;
     const ep_config_t& c = b.cfg;
     const int sm_cap = (c.num_sms > 0 && c.num_sms < b.sm_count) ? c.num_sms : b.sm_count;
-    if (sm_cap < b.sm_count) {
-        // num_sms cap (Buffer.set_num_sms): a resident grid on sm_cap SMs' worth of CTAs
-        int per_sm = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);
-        if (e != cudaSuccess) return e;
-        grid = (int64_t)sm_cap * (per_sm > 0 ? per_sm : 1);
-        if (grid > p.N) grid = p.N;
+    if (sm_cap == b.sm_count) {  // one CTA per token (a grid-stride loop past 2^31 - 1 tokens)
+        const unsigned grid = (unsigned)(p.N < 0x7fffffff ? p.N : 0x7fffffff);
+        if (fp8) combine_fp8_kernel<Y, 1><<<grid, kFp8Threads, 0, st>>>(p, py);
+        else combine_bf16_kernel<Y, 1><<<grid, kBf16Threads, 0, st>>>(p, py);
+        return cudaGetLastError();
     }
-    if (grid > 0x7fffffff) grid = 0x7fffffff;
-    kern<<<(unsigned)grid, threads, 0, st>>>(p, py);
+    // num_sms cap (Buffer.set_num_sms): at most sm_cap CTAs, each filling an SM
+    if (!fp8 && p.K <= kTmaMaxK) return launch_tma(p, py, sm_cap, st);
+    const int sub = fp8 ? kFp8Sub : kBf16Sub;
+    int64_t grid = (p.N + sub - 1) / sub;
+    if (grid > sm_cap) grid = sm_cap;
+    if (fp8) combine_fp8_kernel<Y, kFp8Sub><<<(unsigned)grid, kFp8Threads * kFp8Sub, 0, st>>>(p, py);
+    else combine_bf16_kernel<Y, kBf16Sub><<<(unsigned)grid, kBf16Threads * kBf16Sub, 0, st>>>(p, py);
     return cudaGetLastError();
 }
 

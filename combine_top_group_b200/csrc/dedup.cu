@@ -375,14 +375,12 @@ DedupParams params_of(const ep_buffer& b, int T) {
 template <typename KernelT>
 cudaError_t launch_tokens(KernelT kernel, int threads, const ep_buffer& b, const DedupParams& p, cudaStream_t st) {
     int64_t grid = p.N;
+    // num_sms cap (Buffer.set_num_sms): at most sm_cap CTAs, so that no more
+    // than sm_cap SMs run the kernel (the block scheduler places CTAs
+    // breadth-first); each loops over tokens. One CTA of the usual size per
+    // SM, not the several an SM could hold.
     const int sm_cap = (b.cfg.num_sms > 0 && b.cfg.num_sms < b.sm_count) ? b.cfg.num_sms : b.sm_count;
-    if (sm_cap < b.sm_count) {
-        int per_sm = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0);
-        if (e != cudaSuccess) return e;
-        grid = (int64_t)sm_cap * (per_sm > 0 ? per_sm : 1);
-        if (grid > p.N) grid = p.N;
-    }
+    if (sm_cap < b.sm_count && grid > sm_cap) grid = sm_cap;
     if (grid > 0x7fffffff) grid = 0x7fffffff;
     if (grid < 1) return cudaSuccess;
     kernel<<<(unsigned)grid, threads, 0, st>>>(p);

@@ -4,9 +4,10 @@
 // full all-to-all). The optional FP8 cast sends 1 byte per element instead of
 // 2 (same section) and adds one fp32 scale per 128 channels.
 //
-// One CTA per token (a grid-stride loop when num_sms caps the grid). The
-// threads read the token's row once into registers with 256-bit loads, then
-// write it to each of the K receive rows:
+// One CTA per token; under a num_sms cap, at most num_sms CTAs of several
+// token groups each, looping over tokens. The threads read the token's row
+// once into registers with 256-bit loads, then write it to each of the K
+// receive rows:
 //  - bf16: 256-bit stores, 16 channels per thread;
 //  - FP8: each thread reads 16 channels (32 B) and 8 threads reduce amax over
 //    one 128-channel block with xor shuffles. It casts with
@@ -47,6 +48,7 @@ struct DispatchParams {
     int num_peers;            // entries of the PeerRecv tables
     int64_t g_base;           // global id of local token 0 (recv_src)
     int ordered;              // write a token's rows in (destination rank, row) order
+    int sub_threads;          // threads per token group: blockDim.x, or a part of it under a num_sms cap
     uint32_t* err;
 };
 
@@ -78,13 +80,40 @@ struct PeerRecv {
 };
 
 constexpr int kMaxK = 32;
+constexpr int kMaxSub = 8;  // token groups per CTA under a num_sms cap
+
+// Token groups. Without a num_sms cap (G = false) a CTA is one group: one
+// token at a time, __syncthreads. Under a cap (G = true) a CTA holds
+// blockDim.x / p.sub_threads groups; group j of CTA b takes tokens
+// b * groups + j, then strides by the grid's groups, and waits only for
+// itself, on named barrier 1 + j.
+template <bool G>
+struct Group;
+template <>
+struct Group<false> {
+    static constexpr int sub = 0, n = 1;
+    int tid, threads;
+    __device__ __forceinline__ explicit Group(int) : tid(threadIdx.x), threads(blockDim.x) {}
+    __device__ __forceinline__ void sync() const { __syncthreads(); }
+};
+template <>
+struct Group<true> {
+    int sub, tid, n, threads;
+    __device__ __forceinline__ explicit Group(int sub_threads)
+        : sub(threadIdx.x / sub_threads),
+          tid(threadIdx.x - sub * sub_threads),
+          n(blockDim.x / sub_threads),
+          threads(sub_threads) {}
+    __device__ __forceinline__ void sync() const {
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + sub), "r"(threads) : "memory");
+    }
+};
 
 // Loads the token's K receive rows (checked) and destination ranks, and
 // writes recv_src / recv_w.
 template <class Recv>
 __device__ __forceinline__ void stage_rows(const DispatchParams& p, const Recv& rv, int64_t g, int32_t* s_row,
-                                           int32_t* s_rank) {
-    const int t = threadIdx.x;
+                                           int32_t* s_rank, int t) {
     if (t < p.K) {
         int32_t r = __ldg(p.dst_row + g * p.K + t);
         int d = 0;
@@ -113,14 +142,12 @@ __device__ __forceinline__ void stage_rows(const DispatchParams& p, const Recv& 
 // in flight hold consecutive tokens, whose rows for one expert are adjacent,
 // so in this order their writes meet in fewer places at a time (measured on
 // B200: prefill dispatch 687 -> 678 us). Threads t < K, after s_row / s_rank
-// are visible. With many CTAs in flight (a full grid, or a num_sms cap of at
-// least half the SMs) the CTAs write in this order. Under a smaller cap each
-// CTA loops over hundreds of tokens and pays the extra barrier on each, and
-// slot order is faster (measured on B200, prefill: 20 SMs 1318 against 1390
-// us, 37 SMs 847 against 881 us; at 74 SMs 779 ordered against 787).
+// are visible. With many tokens in flight (a full grid, or a num_sms cap of
+// at least half the SMs) the CTAs write in this order. Under a smaller cap
+// each group loops over hundreds of tokens and pays the extra barrier on
+// each, and slot order is faster.
 template <class Recv>
-__device__ __forceinline__ void order_rows(int K, const int32_t* s_row, const int32_t* s_rank, int32_t* s_ord) {
-    const int t = threadIdx.x;
+__device__ __forceinline__ void order_rows(int K, const int32_t* s_row, const int32_t* s_rank, int32_t* s_ord, int t) {
     if (t < K) {
         auto key = [&](int q) -> uint64_t {
             const int32_t r = s_row[q];
@@ -138,25 +165,29 @@ __device__ __forceinline__ void order_rows(int K, const int32_t* s_row, const in
     }
 }
 
-template <int VPT, class Recv>
-__global__ void __launch_bounds__(512) dispatch_bf16_kernel(DispatchParams p, Recv rv) {
-    __shared__ int32_t s_row[kMaxK];
-    __shared__ int32_t s_rank[Recv::kPeer ? kMaxK : 1];
-    __shared__ int32_t s_ord[kMaxK];
+template <int VPT, class Recv, bool G>
+__global__ void __launch_bounds__(G ? 1024 : 512) dispatch_bf16_kernel(DispatchParams p, Recv rv) {
+    __shared__ int32_t s_row_all[G ? kMaxSub : 1][kMaxK];
+    __shared__ int32_t s_rank_all[G ? kMaxSub : 1][Recv::kPeer ? kMaxK : 1];
+    __shared__ int32_t s_ord_all[G ? kMaxSub : 1][kMaxK];
+    const Group<G> grp(p.sub_threads);
+    int32_t* s_row = s_row_all[grp.sub];
+    int32_t* s_rank = s_rank_all[grp.sub];
+    int32_t* s_ord = s_ord_all[grp.sub];
     const int nv = p.H / 16;  // 32-byte vectors per bf16 row
     const size_t rb = (size_t)p.H * 2;
-    for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {
-        stage_rows(p, rv, g, s_row, s_rank);
+    for (int64_t g = (int64_t)blockIdx.x * grp.n + grp.sub; g < p.N; g += (int64_t)gridDim.x * grp.n) {
+        stage_rows(p, rv, g, s_row, s_rank, grp.tid);
         u32x8 v[VPT];
 #pragma unroll
         for (int j = 0; j < VPT; ++j) {
-            const int c = threadIdx.x + j * blockDim.x;
+            const int c = grp.tid + j * grp.threads;
             if (c < nv) v[j] = ld256_stream(p.x + g * rb + (size_t)c * 32);
         }
-        __syncthreads();
+        grp.sync();
         if (p.ordered) {  // uniform over the grid
-            order_rows<Recv>(p.K, s_row, s_rank, s_ord);
-            __syncthreads();
+            order_rows<Recv>(p.K, s_row, s_rank, s_ord, grp.tid);
+            grp.sync();
         }
         for (int i = 0; i < p.K; ++i) {
             const int k = p.ordered ? s_ord[i] : i;
@@ -165,37 +196,42 @@ __global__ void __launch_bounds__(512) dispatch_bf16_kernel(DispatchParams p, Re
             uint8_t* dst = rv.x_of(Recv::kPeer ? s_rank[k] : 0) + (size_t)r * rb;
 #pragma unroll
             for (int j = 0; j < VPT; ++j) {
-                const int c = threadIdx.x + j * blockDim.x;
+                const int c = grp.tid + j * grp.threads;
                 if (c < nv) st256(dst + (size_t)c * 32, v[j]);
             }
         }
-        __syncthreads();  // s_row is rewritten by the next token
+        grp.sync();  // s_row is rewritten by the next token
     }
     // Stores into peer memory reach the other GPUs before the kernel ends, so
     // a collective that follows it on the stream orders them for the readers.
-    // The loop's last barrier orders every thread's stores before thread 0,
-    // whose system-scope fence (cumulative) then covers the whole CTA.
+    // The loop's last barrier orders every thread's stores of a group before
+    // its thread 0, whose system-scope fence (cumulative) then covers the
+    // group.
     if constexpr (Recv::kPeer) {
-        if (threadIdx.x == 0) __threadfence_system();
+        if (grp.tid == 0) __threadfence_system();
     }
 }
 
-template <int VPT, class Recv>
-__global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchParams p, Recv rv) {
-    __shared__ int32_t s_row[kMaxK];
-    __shared__ int32_t s_rank[Recv::kPeer ? kMaxK : 1];
-    __shared__ int32_t s_ord[kMaxK];
+template <int VPT, class Recv, bool G>
+__global__ void __launch_bounds__(G ? 1024 : 512) dispatch_fp8_kernel(DispatchParams p, Recv rv) {
+    __shared__ int32_t s_row_all[G ? kMaxSub : 1][kMaxK];
+    __shared__ int32_t s_rank_all[G ? kMaxSub : 1][Recv::kPeer ? kMaxK : 1];
+    __shared__ int32_t s_ord_all[G ? kMaxSub : 1][kMaxK];
+    const Group<G> grp(p.sub_threads);
+    int32_t* s_row = s_row_all[grp.sub];
+    int32_t* s_rank = s_rank_all[grp.sub];
+    int32_t* s_ord = s_ord_all[grp.sub];
     const int nv = p.H / 16;  // 16-channel vectors per row: 32 B in, 16 B out
     const int nb = p.H / 128;
     const size_t rb_in = (size_t)p.H * 2;
     const int lane = threadIdx.x & 31;
-    for (int64_t g = blockIdx.x; g < p.N; g += gridDim.x) {
-        stage_rows(p, rv, g, s_row, s_rank);
+    for (int64_t g = (int64_t)blockIdx.x * grp.n + grp.sub; g < p.N; g += (int64_t)gridDim.x * grp.n) {
+        stage_rows(p, rv, g, s_row, s_rank, grp.tid);
         uint4 q[VPT];
         float sc[VPT];
 #pragma unroll
         for (int j = 0; j < VPT; ++j) {
-            const int c = threadIdx.x + j * blockDim.x;
+            const int c = grp.tid + j * grp.threads;
             const bool act = c < nv;  // uniform over each aligned group of 8 lanes
             u32x8 x = act ? ld256_stream(p.x + g * rb_in + (size_t)c * 32) : u32x8{};
             float f[16];
@@ -219,10 +255,10 @@ __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchParams p, Rec
             q[j] = make_uint4(w[0], w[1], w[2], w[3]);
             sc[j] = __fdiv_rn(amax, 448.0f);
         }
-        __syncthreads();
+        grp.sync();
         if (p.ordered) {  // uniform over the grid
-            order_rows<Recv>(p.K, s_row, s_rank, s_ord);
-            __syncthreads();
+            order_rows<Recv>(p.K, s_row, s_rank, s_ord, grp.tid);
+            grp.sync();
         }
         for (int i = 0; i < p.K; ++i) {
             const int k = p.ordered ? s_ord[i] : i;
@@ -233,34 +269,27 @@ __global__ void __launch_bounds__(512) dispatch_fp8_kernel(DispatchParams p, Rec
             float* scale = rv.scale_of(d);
 #pragma unroll
             for (int j = 0; j < VPT; ++j) {
-                const int c = threadIdx.x + j * blockDim.x;
+                const int c = grp.tid + j * grp.threads;
                 if (c < nv) {
                     __stcs(reinterpret_cast<uint4*>(dst) + c, q[j]);
                     if ((lane & 7) == 0) scale[(size_t)r * nb + c / 8] = sc[j];
                 }
             }
         }
-        __syncthreads();
+        grp.sync();
     }
     if constexpr (Recv::kPeer) {  // as in dispatch_bf16_kernel
-        if (threadIdx.x == 0) __threadfence_system();
+        if (grp.tid == 0) __threadfence_system();
     }
 }
 
+// One CTA per token (a grid-stride loop past 2^31 - 1 tokens).
 template <class Recv>
-cudaError_t launch_rows(void (*kernel)(DispatchParams, Recv), int threads, int sm_cap, int full_sms,
-                        const DispatchParams& p, const Recv& rv, cudaStream_t st) {
-    int64_t grid = p.N;
-    if (sm_cap < full_sms) {
-        // num_sms cap (Buffer.set_num_sms): a resident grid on sm_cap SMs' worth of CTAs
-        int per_sm = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0);
-        if (e != cudaSuccess) return e;
-        grid = (int64_t)sm_cap * (per_sm > 0 ? per_sm : 1);
-        if (grid > p.N) grid = p.N;
-    }
-    if (grid > 0x7fffffff) grid = 0x7fffffff;
-    kernel<<<(unsigned)grid, threads, 0, st>>>(p, rv);
+cudaError_t launch_rows(void (*kernel)(DispatchParams, Recv), int threads, DispatchParams p, const Recv& rv,
+                        cudaStream_t st) {
+    p.sub_threads = threads;
+    const unsigned grid = (unsigned)(p.N < 0x7fffffff ? p.N : 0x7fffffff);
+    kernel<<<grid, threads, 0, st>>>(p, rv);
     return cudaGetLastError();
 }
 
@@ -304,12 +333,44 @@ cudaError_t per_sm_of(const void* fn, int threads, int* per_sm) {
     return cudaSuccess;
 }
 
-template <class Recv>
+template <class Recv, bool G>
 void (*fp8_kernel_of(int vpt))(DispatchParams, Recv) {
-    if (vpt <= 1) return dispatch_fp8_kernel<1, Recv>;
-    if (vpt <= 2) return dispatch_fp8_kernel<2, Recv>;
-    if (vpt <= 4) return dispatch_fp8_kernel<4, Recv>;
-    return dispatch_fp8_kernel<8, Recv>;
+    if (vpt <= 1) return dispatch_fp8_kernel<1, Recv, G>;
+    if (vpt <= 2) return dispatch_fp8_kernel<2, Recv, G>;
+    if (vpt <= 4) return dispatch_fp8_kernel<4, Recv, G>;
+    return dispatch_fp8_kernel<8, Recv, G>;
+}
+
+template <class Recv, bool G>
+void (*bf16_kernel_of(int vpt))(DispatchParams, Recv) {
+    if (vpt <= 1) return dispatch_bf16_kernel<1, Recv, G>;
+    if (vpt <= 2) return dispatch_bf16_kernel<2, Recv, G>;
+    if (vpt <= 4) return dispatch_bf16_kernel<4, Recv, G>;
+    return dispatch_bf16_kernel<8, Recv, G>;
+}
+
+// num_sms cap (Buffer.set_num_sms): at most sm_cap CTAs, so that no more than
+// sm_cap SMs run the kernel (the block scheduler places CTAs breadth-first:
+// 4 * sm_cap small CTAs would occupy 4 * sm_cap SMs). Each CTA holds as many
+// token groups as fit one SM (up to 1024 threads), each group two 16-channel
+// vectors per thread, so that an SM keeps as many bytes in flight as it
+// would with several one-vector CTAs.
+template <class Recv>
+cudaError_t launch_capped(DispatchParams p, const Recv& rv, bool fp8, int sm_cap, cudaStream_t st) {
+    int threads, vpt;
+    shape_of(p.H, 2, &threads, &vpt);
+    auto kern = fp8 ? fp8_kernel_of<Recv, true>(vpt) : bf16_kernel_of<Recv, true>(vpt);
+    int per_sm = 0;
+    cudaError_t e = per_sm_of((const void*)kern, threads, &per_sm);
+    if (e != cudaSuccess) return e;
+    int subs = per_sm < 1024 / threads ? per_sm : 1024 / threads;
+    subs = subs < kMaxSub ? subs : kMaxSub;
+    subs = subs > 1 ? subs : 1;
+    int64_t grid = (p.N + subs - 1) / subs;
+    grid = grid < sm_cap ? grid : sm_cap;
+    p.sub_threads = threads;
+    kern<<<(unsigned)grid, threads * subs, 0, st>>>(p, rv);
+    return cudaGetLastError();
 }
 
 template <class Recv>
@@ -317,35 +378,29 @@ cudaError_t launch_any(const DispatchParams& p0, const Recv& rv, bool fp8, int s
                        cudaStream_t st) {
     DispatchParams p = p0;
     p.ordered = 2 * sm_cap >= full_sms ? 1 : 0;
+    if (sm_cap < full_sms) return launch_capped(p, rv, fp8, sm_cap, st);
     int threads, vpt;
     shape_of(p.H, fp8 ? 2 : 1, &threads, &vpt);
-    if (!fp8) {
-        if (vpt <= 1) return launch_rows(dispatch_bf16_kernel<1, Recv>, threads, sm_cap, full_sms, p, rv, st);
-        if (vpt <= 2) return launch_rows(dispatch_bf16_kernel<2, Recv>, threads, sm_cap, full_sms, p, rv, st);
-        if (vpt <= 4) return launch_rows(dispatch_bf16_kernel<4, Recv>, threads, sm_cap, full_sms, p, rv, st);
-        return launch_rows(dispatch_bf16_kernel<8, Recv>, threads, sm_cap, full_sms, p, rv, st);
-    }
-    auto kern = fp8_kernel_of<Recv>(vpt);
-    if (sm_cap == full_sms) {
-        // A batch a little over one wave of CTAs (decode: 1024 tokens against
-        // 888 resident CTAs of 224 threads) would leave a short second wave
-        // running alone. Half as many threads with twice the vectors each fit
-        // it in one wave when they can.
-        int per_sm = 0;
-        cudaError_t e = per_sm_of((const void*)kern, threads, &per_sm);
+    if (!fp8) return launch_rows(bf16_kernel_of<Recv, false>(vpt), threads, p, rv, st);
+    auto kern = fp8_kernel_of<Recv, false>(vpt);
+    // A batch a little over one wave of CTAs (decode: 1024 tokens against
+    // 888 resident CTAs of 224 threads) would leave a short second wave
+    // running alone. Half as many threads with twice the vectors each fit it
+    // in one wave when they can.
+    int per_sm = 0;
+    cudaError_t e = per_sm_of((const void*)kern, threads, &per_sm);
+    if (e != cudaSuccess) return e;
+    const int64_t wave = (int64_t)per_sm * full_sms;
+    if (p.N > wave && p.N <= 2 * wave) {
+        int t4, v4;
+        shape_of(p.H, 4, &t4, &v4);
+        auto k4 = fp8_kernel_of<Recv, false>(v4);
+        int per4 = 0;
+        e = per_sm_of((const void*)k4, t4, &per4);
         if (e != cudaSuccess) return e;
-        const int64_t wave = (int64_t)per_sm * full_sms;
-        if (p.N > wave && p.N <= 2 * wave) {
-            int t4, v4;
-            shape_of(p.H, 4, &t4, &v4);
-            auto k4 = fp8_kernel_of<Recv>(v4);
-            int per4 = 0;
-            e = per_sm_of((const void*)k4, t4, &per4);
-            if (e != cudaSuccess) return e;
-            if (p.N <= (int64_t)per4 * full_sms) return launch_rows(k4, t4, sm_cap, full_sms, p, rv, st);
-        }
+        if (p.N <= (int64_t)per4 * full_sms) return launch_rows(k4, t4, p, rv, st);
     }
-    return launch_rows(kern, threads, sm_cap, full_sms, p, rv, st);
+    return launch_rows(kern, threads, p, rv, st);
 }
 
 DispatchParams params_of(const ep_buffer& b, int64_t N, const void* x) {

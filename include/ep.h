@@ -151,12 +151,18 @@ ep_status_t ep_buffer_create(const ep_config_t *cfg, void *d_workspace, size_t b
 /* Frees the host struct only. NULL is a no-op. */
 ep_status_t ep_buffer_destroy(ep_buffer_t *buf);
 
-/* Sets the SM budget of the buffer's dispatch and combine kernels: at most
- * num_sms SMs' worth of resident CTAs, each looping over tokens; 0 = all SMs.
- * This is the analogue of DeepEP's Buffer.set_num_sms (DeepEP summary,
- * "如何调优 Buffer.set_num_sms"; DeepEP overlap notes, §节点内通信: 20
- * communication SMs, the rest for compute). It takes effect from the next
- * call. Results are identical under any budget.
+/* Sets the SM budget of the buffer's dispatch and combine kernels (the
+ * standard, shard and deduplicated ones; not ep_get_layout): with
+ * 0 < num_sms < the device's SM count, each such kernel launches at most
+ * num_sms CTAs, so it occupies at most num_sms SMs, and each CTA loops over
+ * tokens. A CTA is made as large as one SM holds where the kernel allows it
+ * (several token groups per CTA in dispatch and the register combines; a
+ * bulk-copy pipeline of one CTA per SM in the bf16 combine). 0, or a count
+ * at or above the SM count, = all SMs. This is the analogue of DeepEP's
+ * Buffer.set_num_sms (DeepEP summary, "如何调优 Buffer.set_num_sms"; DeepEP
+ * overlap notes, §节点内通信: 20 communication SMs, the rest for compute).
+ * It takes effect from the next call. Results are identical under any
+ * budget.
  * Errors: EP_ERR_INVALID for num_sms < 0. */
 ep_status_t ep_buffer_set_num_sms(ep_buffer_t *buf, int num_sms);
 

@@ -150,3 +150,37 @@ def test_dedup_calls_need_the_flag(cuda):
         with pytest.raises(ep.EpError) as ei:
             call()
         assert ei.value.status == ep.EP_ERR_INVALID
+
+
+@pytest.mark.parametrize("num_sms", [1, 20])
+def test_dedup_path_under_sm_budget(cuda, num_sms):
+    """Every dedup stage under a num_sms cap (one CTA per SM, looping over
+    tokens) gives the uncapped run's bytes: dedup rows, expert rows, partials
+    and output; bf16 and FP8 rows, the fused dequant included."""
+    ep, runner = cuda
+    for name, fused in (("tiny", False), ("decode", True), ("skewed", False)):
+        w = wl.WORKLOADS[name]
+        if name == "skewed":
+            w = w.with_tokens(64)
+        pipe = runner.Pipeline(w, 3, dedup=True)
+        dd = pipe.dd
+
+        def run():
+            pipe.layout()
+            pipe.dispatch_dedup()
+            pipe.permute()
+            if w.fp8 and not fused:
+                pipe.identity_expert()
+            pipe.local_reduce(fused=fused)
+            pipe.combine_dedup()
+            assert pipe.check_errors() == 0
+            D, M = pipe.dedup_rows(), pipe.num_rows()
+            return [t.clone() for t in (dd["dd_x"][:D], pipe.recv["recv_x"][:M], dd["partial"][:D], pipe.out)]
+
+        ref = run()
+        ep.ep_buffer_set_num_sms(pipe.buf, num_sms)
+        for t in (dd["dd_x"], pipe.recv["recv_x"], dd["partial"], pipe.out):
+            t.zero_()
+        got = run()
+        for a, b in zip(got, ref):
+            assert torch.equal(a.view(torch.int8), b.view(torch.int8))

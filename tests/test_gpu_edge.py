@@ -148,23 +148,38 @@ def test_num_sms_cap_gives_identical_bytes(cuda):
     assert torch.equal(a.out, b.out)
 
 
+def _step(pipe, fused):
+    """One step; an FP8 receive combined unfused goes through bf16 y."""
+    if pipe.w.fp8 and not fused:
+        pipe.layout()
+        pipe.dispatch()
+        pipe.identity_expert()
+        pipe.combine()
+    else:
+        pipe.step(fused=fused)
+
+
 @pytest.mark.parametrize("num_sms", [1, 7, 37, 74])
 def test_set_num_sms_changes_nothing_but_the_grid(cuda, num_sms):
     """Buffer.set_num_sms analogue: dispatch and combine (bf16 and fused FP8)
-    under an SM budget loop over tokens and give the same bytes."""
+    under an SM budget loop over tokens and give the same bytes; token counts
+    that the budget does not divide, K below 8 and masked slots included."""
     ep, runner = cuda
-    for name in ("tiny", "decode"):
+    for name, fused in (("tiny", True), ("decode", True), ("tiny", False), ("decode", False), ("skewed", False)):
         w = wl.WORKLOADS[name]
+        if name == "skewed":
+            w = w.with_tokens(37)
         pipe = runner.Pipeline(w, 4)
-        pipe.step(fused=True)
+        _step(pipe, fused)
         M = pipe.num_rows()
         ref = (pipe.recv["recv_x"][:M].clone(), pipe.out.clone())
         ep.ep_buffer_set_num_sms(pipe.buf, num_sms)
         pipe.recv["recv_x"][:M].zero_()
         pipe.out.zero_()
-        pipe.step(fused=True)
+        _step(pipe, fused)
         assert pipe.check_errors() == 0
-        assert torch.equal(pipe.recv["recv_x"][:M], ref[0]) and torch.equal(pipe.out, ref[1])
+        assert torch.equal(pipe.recv["recv_x"][:M].view(torch.int8), ref[0].view(torch.int8))
+        assert torch.equal(pipe.out.view(torch.int16), ref[1].view(torch.int16))
     with pytest.raises(ep.EpError):
         ep.ep_buffer_set_num_sms(pipe.buf, -1)
 
