@@ -216,15 +216,19 @@ __global__ void __launch_bounds__(kFp8Threads * SUB) combine_fp8_kernel(CombineP
 
 // ---- bf16 combine under a num_sms cap: a TMA bulk-copy pipeline ------------
 //
-// Under a num_sms cap the grid is one CTA per SM, and the register gather
-// above keeps at most 128 KB per SM in flight (512 threads, 8 loads of 32 B
+// Under a num_sms cap the grid is one CTA per SM. The register gather above
+// then keeps at most 128 KB per SM in flight (512 threads, 8 loads of 32 B
 // each). Here the bulk-copy (TMA) engine moves the rows into shared memory
 // instead: 4 stages, each K row segments of kTmaChunk channels (56 KB at
 // K = 8), so the threads issue only the arithmetic. Measured on B200 at the
-// prefill shape (8 x 4096 tokens, H = 7168, K = 8): 2.3-2.6 ms against 2.9 ms
-// for the register gather at 20 SMs, 0.69-0.72 against 0.88 ms at 74 SMs.
-// More and smaller stages (2-4 KB copies, 6-12 stages) and whole-row copies
-// (14 KB, 4 slots per stage) were slower.
+// prefill shape (8 x 4096 tokens, H = 7168, K = 8): 2.2 ms at 20 SMs and
+// 0.66 ms at 74 SMs, against 2.9 and 0.88 ms for the register gather. Every
+// byte crosses shared memory twice (the copy, then the consumers' reads),
+// which bounds this design at about half the shared-memory bandwidth.
+// Slower, as measured:
+//  - more and smaller stages (2-4 KB copies, 6-12 stages);
+//  - whole-row copies (14 KB, 4 slots per stage);
+//  - 448 consumers of 8 channels with a sleep hint in the waits.
 //
 // One CTA per SM: kTmaConsumers consumer threads and one producer warp. A
 // unit is one token and one block of kTmaChunk channels; CTA b takes a
@@ -234,10 +238,12 @@ __global__ void __launch_bounds__(kFp8Threads * SUB) combine_fp8_kernel(CombineP
 // so that their latency overlaps the copies of the batch before. For a unit it
 // writes the token, the slot mask and the weights next to the stage, arms the
 // stage's "full" barrier with the bytes to come, and each lane of the token's
-// group with an unmasked slot issues that row's bulk copy. Every consumer
-// warp, after reading a stage, arrives on its "empty" barrier, which frees
-// the stage for the producer. The sum is the register kernel's: an fp32 fma
-// chain over k ascending, one bf16 rounding.
+// group with an unmasked slot issues that row's bulk copy. A consumer thread
+// t owns channels 8t.. and kTmaChunk/2 + 8t.. of the block (16-byte reads,
+// contiguous across a warp: no bank conflicts). It moves them to registers
+// for all K rows, and every consumer warp then arrives on the stage's "empty"
+// barrier, which frees the stage for the producer. The sum is the register
+// kernel's: an fp32 fma chain over k ascending, one bf16 rounding.
 //
 // Every wait is bounded (kWaitLimitNs): a wait that gives up sets
 // EP_DEVERR_TIMEOUT, and before the CTA returns the producer waits, bounded
@@ -250,7 +256,7 @@ constexpr int kTmaThreads = kTmaConsumers + 32;
 constexpr int kTmaStages = 4;
 constexpr int kTmaMaxK = 8;
 constexpr int kTmaBatch = 32 / kTmaMaxK;  // tokens whose slots the producer warp reads at once
-constexpr int kTmaVec = 16;               // channels per consumer: 8 or 16
+constexpr int kTmaVec = 16;               // channels per consumer
 constexpr int kTmaChunk = kTmaConsumers * kTmaVec;  // channels per unit
 constexpr size_t kTmaStageBytes = (size_t)kTmaMaxK * kTmaChunk * 2;
 // What the producer tells the consumers about the unit in a stage.
@@ -406,52 +412,53 @@ __global__ void __launch_bounds__(kTmaThreads, 1) combine_bf16_tma_kernel(Combin
         const TmaUnit& m = meta[s];
         const int64_t g = m.g;
         const uint32_t mask = m.mask;
-        const int v = m.cb * kTmaConsumers + t;  // this thread's kTmaVec channels
+        // This thread's channels of the block: 8 at c0 and 8 at c1, so that a
+        // warp's 16-byte shared-memory reads are contiguous (no bank conflict).
+        const int wb = min(kTmaChunk, p.H - m.cb * kTmaChunk);  // channels in the block
+        const int c0 = 8 * t, c1 = kTmaChunk / 2 + 8 * t;
+        const bool h0 = c0 < wb, h1 = c1 < wb;
         // the stage's rows into registers, then the stage goes back to the producer
-        const uint8_t* stage = sm + (size_t)s * kTmaStageBytes + (size_t)t * kTmaVec * 2;
-        uint32_t q[kTmaMaxK][kTmaVec / 2];
+        const uint8_t* stage = sm + (size_t)s * kTmaStageBytes;
+        uint32_t q[kTmaMaxK][8];
         float w[kTmaMaxK];
-        const bool mine_v = v * kTmaVec < p.H;
 #pragma unroll
         for (int k = 0; k < kTmaMaxK; ++k) {
             w[k] = m.w[k];
-            if (mine_v && ((mask >> k) & 1u)) {
-#pragma unroll
-                for (int h = 0; h < kTmaVec / 8; ++h) {
-                    const uint4 a = *reinterpret_cast<const uint4*>(stage + (size_t)k * kTmaChunk * 2 + h * 16);
-                    q[k][4 * h] = a.x, q[k][4 * h + 1] = a.y, q[k][4 * h + 2] = a.z, q[k][4 * h + 3] = a.w;
+            if ((mask >> k) & 1u) {
+                const uint8_t* row = stage + (size_t)k * kTmaChunk * 2;
+                if (h0) {
+                    const uint4 a = *reinterpret_cast<const uint4*>(row + c0 * 2);
+                    q[k][0] = a.x, q[k][1] = a.y, q[k][2] = a.z, q[k][3] = a.w;
+                }
+                if (h1) {
+                    const uint4 a = *reinterpret_cast<const uint4*>(row + c1 * 2);
+                    q[k][4] = a.x, q[k][5] = a.y, q[k][6] = a.z, q[k][7] = a.w;
                 }
             }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
-        if (mine_v) {
-            uint64_t acc[kTmaVec / 2];  // channel pairs (2j, 2j+1) as fp32 pairs
+        if (h0) {  // h1 implies h0
+            uint64_t acc[8];  // channel pairs as fp32 pairs: 0-3 at c0, 4-7 at c1
 #pragma unroll
-            for (int j = 0; j < kTmaVec / 2; ++j) acc[j] = 0ull;
+            for (int j = 0; j < 8; ++j) acc[j] = 0ull;
 #pragma unroll
             for (int k = 0; k < kTmaMaxK; ++k) {
                 if (!((mask >> k) & 1u)) continue;
                 const uint64_t w2 = f32x2_pack(w[k], w[k]);
 #pragma unroll
-                for (int j = 0; j < kTmaVec / 2; ++j)  // per channel: acc = fma(w, y, acc), rounded as the scalar chain
-                    acc[j] = f32x2_fma_rn(w2, f32x2_pack(bf16lo(q[k][j]), bf16hi(q[k][j])), acc[j]);
+                for (int j = 0; j < 8; ++j)  // per channel: acc = fma(w, y, acc), rounded as the scalar chain
+                    if (j < 4 || h1) acc[j] = f32x2_fma_rn(w2, f32x2_pack(bf16lo(q[k][j]), bf16hi(q[k][j])), acc[j]);
             }
-            uint32_t o[kTmaVec / 2];
+            uint32_t o[8];
 #pragma unroll
-            for (int j = 0; j < kTmaVec / 2; ++j) {
+            for (int j = 0; j < 8; ++j) {
                 const float2 a = f32x2_unpack(acc[j]);
                 o[j] = pack_bf16x2(a.x, a.y);
             }
-            uint8_t* dst = p.out + (size_t)g * rb + (size_t)v * kTmaVec * 2;
-            if constexpr (kTmaVec == 16) {
-                u32x8 o8;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) o8.v[j] = o[j];
-                st256(dst, o8);
-            } else {
-                *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
-            }
+            uint8_t* dst = p.out + (size_t)g * rb + (size_t)m.cb * kTmaChunk * 2;
+            *reinterpret_cast<uint4*>(dst + c0 * 2) = make_uint4(o[0], o[1], o[2], o[3]);
+            if (h1) *reinterpret_cast<uint4*>(dst + c1 * 2) = make_uint4(o[4], o[5], o[6], o[7]);
         }
     }
 }
