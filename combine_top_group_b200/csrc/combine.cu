@@ -67,6 +67,7 @@ struct PeerY {
 };
 
 constexpr int kChunk = 8;  // slots gathered per pass: kChunk loads in flight per thread
+constexpr int kMaxKFp8 = 8;  // slots held in registers by combine_fp8_k8_kernel
 
 // Receive row of slot k, read by every thread (broadcast, L1 after the first
 // warp) so that no warp waits on another; -1 for masked or out-of-range rows.
@@ -200,6 +201,88 @@ __global__ void __launch_bounds__(kFp8Threads * SUB) combine_fp8_kernel(CombineP
                             acc[2 * j + 1] =
                                 f32x2_fma_rn(w2, f32x2_mul_rn(f32x2_pack(b.x, b.y), s2), acc[2 * j + 1]);
                         }
+                    }
+                }
+            }
+            u32x8 o;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float2 a = f32x2_unpack(acc[j]);
+                o.v[j] = pack_bf16x2(a.x, a.y);
+            }
+            st256(p.out + (size_t)g * p.H * 2 + (size_t)v * 32, o);
+        }
+    }
+}
+
+// The same for K <= kMaxKFp8: the token's K row and scale-row addresses and
+// weights are read once per token into registers (masked and refused slots
+// are skipped), then each thread walks its 16-channel vectors.
+template <class Y, int SUB>
+__global__ void __launch_bounds__(kFp8Threads * SUB) combine_fp8_k8_kernel(CombineParams p, Y py) {
+    const int nvec = p.H / 16;  // 16 e4m3 channels (16 B) per vector
+    const int nb = p.H / 128;
+    const size_t rb = (size_t)p.H;
+    const int sub = threadIdx.x / kFp8Threads, tid = threadIdx.x - sub * kFp8Threads;
+    for (int64_t g = (int64_t)blockIdx.x * SUB + sub; g < p.N; g += (int64_t)gridDim.x * SUB) {
+        report_rows<Y>(p, g, tid);
+        const uint8_t* base[kMaxKFp8];
+        const float* sbase[kMaxKFp8];
+        float w[kMaxKFp8];
+        uint32_t live = 0;  // bit i: slot i is read
+#pragma unroll
+        for (int i = 0; i < kMaxKFp8; ++i) {
+            base[i] = nullptr;
+            sbase[i] = nullptr;
+            w[i] = 0.0f;
+            if (i < p.K) {
+                const int32_t r = row_of(p, g, i);
+                if (r >= 0) {
+                    if constexpr (Y::kPeer) {
+                        const int d = __ldg(p.dst_rank + g * p.K + i);
+                        if (d < p.num_peers) {
+                            base[i] = py.y[d] + (size_t)r * rb;
+                            sbase[i] = py.scale[d] + (size_t)r * nb;
+                        }
+                    } else {
+                        base[i] = p.y + (size_t)r * rb;
+                        sbase[i] = p.y_scale + (size_t)r * nb;
+                    }
+                    if (base[i] != nullptr) {
+                        w[i] = __ldg(p.topk_w + g * p.K + i);
+                        live |= 1u << i;
+                    }
+                }
+            }
+        }
+        for (int v = tid; v < nvec; v += kFp8Threads) {
+            // acc[j] holds channels 2j and 2j+1 as an fp32 pair
+            uint64_t acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = 0ull;
+            uint4 q[kMaxKFp8];
+            float sc[kMaxKFp8];
+#pragma unroll
+            for (int i = 0; i < kMaxKFp8; ++i) {
+                if ((live >> i) & 1u) {
+                    q[i] = __ldcs(reinterpret_cast<const uint4*>(base[i]) + v);
+                    sc[i] = __ldg(sbase[i] + v / 8);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kMaxKFp8; ++i) {
+                if ((live >> i) & 1u) {
+                    // per channel: acc = fma(w, e4m3 * scale, acc), each step rounded
+                    // as in the scalar chain, two channels per instruction
+                    const uint64_t w2 = f32x2_pack(w[i], w[i]);
+                    const uint64_t s2 = f32x2_pack(sc[i], sc[i]);
+                    const uint32_t u[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 a = unpack_e4m3x2(u[j] & 0xffffu);
+                        const float2 b = unpack_e4m3x2(u[j] >> 16);
+                        acc[2 * j] = f32x2_fma_rn(w2, f32x2_mul_rn(f32x2_pack(a.x, a.y), s2), acc[2 * j]);
+                        acc[2 * j + 1] = f32x2_fma_rn(w2, f32x2_mul_rn(f32x2_pack(b.x, b.y), s2), acc[2 * j + 1]);
                     }
                 }
             }
@@ -480,7 +563,8 @@ cudaError_t launch_y(const ep_buffer& b, const CombineParams& p, const Y& py, bo
     const int sm_cap = (c.num_sms > 0 && c.num_sms < b.sm_count) ? c.num_sms : b.sm_count;
     if (sm_cap == b.sm_count) {  // one CTA per token (a grid-stride loop past 2^31 - 1 tokens)
         const unsigned grid = (unsigned)(p.N < 0x7fffffff ? p.N : 0x7fffffff);
-        if (fp8) combine_fp8_kernel<Y, 1><<<grid, kFp8Threads, 0, st>>>(p, py);
+        if (fp8 && p.K <= kMaxKFp8) combine_fp8_k8_kernel<Y, 1><<<grid, kFp8Threads, 0, st>>>(p, py);
+        else if (fp8) combine_fp8_kernel<Y, 1><<<grid, kFp8Threads, 0, st>>>(p, py);
         else combine_bf16_kernel<Y, 1><<<grid, kBf16Threads, 0, st>>>(p, py);
         return cudaGetLastError();
     }
