@@ -372,13 +372,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 // Waits for the phase of `bar` with this parity to complete; false if it
-// has not after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// has not after limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity))
-        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
     return true;
+}
+
+// Self-test of the bounded mbarrier wait: a barrier that expects one arrival
+// nobody makes. The wait must give up after limit_ns; thread 0 then records
+// that in gave_up and sets EP_DEVERR_TIMEOUT. No copy is in flight.
+__global__ void mbarrier_timeout_selftest_kernel(uint32_t* err, uint32_t* gave_up, unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait(&bar, 0, limit_ns)) {
+        *gave_up = 1u;
+        set_error(err, EP_DEVERR_TIMEOUT);
+    }
 }
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
     asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -595,6 +612,12 @@ CombineParams params_of(const ep_buffer& b, int64_t N, const void* y, const floa
 }
 
 }  // namespace
+
+cudaError_t launch_mbarrier_timeout_selftest(uint32_t* err, uint32_t* gave_up, unsigned long long limit_ns,
+                                             cudaStream_t st) {
+    mbarrier_timeout_selftest_kernel<<<1, 32, 0, st>>>(err, gave_up, limit_ns);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_combine(const ep_buffer& b, int T, const void* y, const float* y_scale, void* out,
                            cudaStream_t st) {

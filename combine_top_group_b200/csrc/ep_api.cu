@@ -585,6 +585,7 @@ ep_status_t ep_selftest_wait_timeout(uint32_t* d_words, uint64_t limit_ns, uint3
     if (limit_ns < 1000 || limit_ns > 2000000000ull) return fail(EP_ERR_INVALID, "limit_ns must be in [1 us, 2 s]");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = ep::launch_barrier_timeout_selftest(d_words, limit_ns, s);
+    if (e == cudaSuccess) e = ep::launch_mbarrier_timeout_selftest(d_words + 2, d_words + 3, limit_ns, s);
     uint32_t v = 0;
     if (e == cudaSuccess) e = cudaMemcpyAsync(&v, d_words + 2, sizeof v, cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);

@@ -98,6 +98,10 @@ cudaError_t launch_layout(const ep_buffer& b, const LayoutArgs& a, cudaStream_t 
 // Runs the layout's grid barrier with an unreachable target on 2 CTAs
 // (words: 4 device uint32; [2] receives the error bits).
 cudaError_t launch_barrier_timeout_selftest(uint32_t* words, unsigned long long limit_ns, cudaStream_t stream);
+// The combine pipeline's mbarrier wait on a phase that never completes; sets
+// *gave_up = 1 and EP_DEVERR_TIMEOUT in *err when the wait ends unmet.
+cudaError_t launch_mbarrier_timeout_selftest(uint32_t* err, uint32_t* gave_up, unsigned long long limit_ns,
+                                             cudaStream_t stream);
 cudaError_t launch_dispatch(const ep_buffer& b, int T, const void* x, cudaStream_t stream);
 cudaError_t launch_dispatch_dedup(const ep_buffer& b, int T, const void* x, cudaStream_t stream);
 cudaError_t launch_permute(const ep_buffer& b, int T, cudaStream_t stream);

@@ -378,9 +378,13 @@ ep_status_t ep_shard_dispatch(ep_buffer_t *buf, int rank, int T, const void *d_x
 ep_status_t ep_shard_combine(ep_buffer_t *buf, int rank, int T, const void *const *peer_y,
                              const float *const *peer_y_scale, void *d_out, void *stream);
 
-/* Diagnostic: proves that the library's bounded waits end. Runs the layout's
- * grid barrier on 2 CTAs with a target that can never be reached, and a limit
- * of limit_ns (1 us .. 2 s). Every CTA must give up and set EP_DEVERR_TIMEOUT.
+/* Diagnostic: proves that the library's bounded waits end. Runs, each with a
+ * limit of limit_ns (1 us .. 2 s):
+ *  - the layout's grid barrier on 2 CTAs with a target that can never be
+ *    reached: every CTA must give up and set EP_DEVERR_TIMEOUT;
+ *  - the capped combine pipeline's mbarrier wait on a phase that never
+ *    completes: it must give up, set EP_DEVERR_TIMEOUT and write 1 to
+ *    d_words[3].
  * d_words: 4 device uint32 of scratch, owned by the caller. The call
  * synchronises `stream` and returns the error bits in *word. It never traps,
  * and the CUDA context stays usable. (The pages have no counterpart: it checks

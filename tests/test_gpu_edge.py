@@ -322,17 +322,18 @@ def test_guard_bands_and_rows_beyond_M_untouched(cuda):
 
 
 def test_bounded_wait_gives_up_and_context_survives(cuda):
-    """A grid barrier whose target nothing can reach must end after its limit
-    with EP_DEVERR_TIMEOUT (no trap, no hang), and the next path call must
-    work."""
+    """A grid barrier whose target nothing can reach, and an mbarrier phase
+    that never completes, must each end after the limit with
+    EP_DEVERR_TIMEOUT (no trap, no hang), and the next path call must work."""
     import time
     ep, runner = cuda
     words = torch.zeros(4, dtype=torch.int32, device="cuda")
     t0 = time.perf_counter()
-    bits = ep.ep_selftest_wait_timeout(words, 50_000_000)  # 50 ms
+    bits = ep.ep_selftest_wait_timeout(words, 50_000_000)  # 50 ms each
     dt = time.perf_counter() - t0
     assert bits & ep.EP_DEVERR_TIMEOUT
-    assert 0.04 < dt < 5.0
+    assert int(words[3].item()) == 1  # the mbarrier wait gave up
+    assert 0.09 < dt < 5.0
     w = wl.WORKLOADS["tiny"]
     x, logits = wl.make_x(w, 1), wl.make_logits(w, 1)
     pipe = runner.Pipeline(w, 1, x=x, logits=logits)
