@@ -358,3 +358,57 @@ def test_low_latency_region_overflow_flagged(cuda):
     ref, ref_err = oracle.layout_ll(idx, 2, 2, 2, 4)
     assert ref_err & 2
     assert np.array_equal(ep.ep_buffer_layout(pipe.buf, 2)["dst_row"].cpu().numpy(), ref)
+
+
+def _kernel_grids(fn):
+    """(kernel name, grid x) of every CUDA kernel launched by fn(), from the
+    profiler's trace."""
+    import json
+    import tempfile
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    with tempfile.NamedTemporaryFile(suffix=".json") as f:
+        prof.export_chrome_trace(f.name)
+        trace = json.load(open(f.name))
+    return [(e["name"], int(e["args"]["grid"][0])) for e in trace["traceEvents"]
+            if e.get("cat") == "kernel" and "grid" in e.get("args", {})]
+
+
+@pytest.mark.parametrize("num_sms", [7, 20])
+def test_capped_kernels_launch_at_most_num_sms_ctas(cuda, num_sms):
+    """Under a num_sms cap every dispatch and combine kernel (bf16, FP8, the
+    fused FP8 combine, the bulk-copy combine, the dedup kernels) launches at
+    most num_sms CTAs, so it can occupy at most num_sms SMs; without a cap the
+    grid is one CTA per token."""
+    ep, runner = cuda
+    capped = ("dispatch", "combine", "permute", "local_reduce")
+    seen = set()
+    for name, fused, dedup in (("tiny", False, False), ("decode", True, False), ("skewed", False, False),
+                               ("decode", True, True)):
+        w = wl.WORKLOADS[name]
+        if name == "skewed":
+            w = w.with_tokens(64)
+        pipe = runner.Pipeline(w, 2, dedup=dedup)
+
+        def run():
+            if dedup:
+                pipe.step_dedup(fused=fused)
+            elif w.fp8 and not fused:
+                _step(pipe, fused)
+            else:
+                pipe.step(fused=fused)
+
+        run()  # warm-up outside the trace
+        full = _kernel_grids(run)
+        ep.ep_buffer_set_num_sms(pipe.buf, num_sms)
+        grids = _kernel_grids(run)
+        assert pipe.check_errors() == 0
+        ours = [(k, g) for k, g in grids if any(c in k for c in capped)]
+        assert ours, grids
+        for k, g in ours:
+            assert g <= num_sms, (name, k, g)
+            seen.add(k)
+        assert any(g == w.N for k, g in full if "dispatch" in k and "dedup" not in k) or dedup
+    assert any("tma" in k for k in seen) and any("fp8" in k for k in seen)
