@@ -6,12 +6,15 @@
 // slots. FP8 expert outputs are dequantised in the same pass: e4m3 * scale
 // in fp32.
 //
-// One CTA per token (a grid-stride loop when num_sms caps the grid). Each
-// thread owns 16 channels of y at a time: a 32-byte vector of
-// bf16 (256-bit load) or a 16-byte vector of e4m3. It issues the K gathers of
-// that column before any arithmetic, so K loads are in flight per thread.
-// Loads use the streaming cache hint (y is read once). The 32 output bytes
-// go out in one 256-bit store.
+// One CTA per token; under a num_sms cap, at most num_sms CTAs of several
+// token groups each, looping over tokens, or for bf16 y the bulk-copy
+// pipeline further down. Each thread owns 16 channels of y at a time: a
+// 32-byte vector of bf16 (256-bit load) or a 16-byte vector of e4m3. It
+// issues the K gathers of that column before any arithmetic, so K loads are
+// in flight per thread. For K <= 8 (the *_k8 kernels) a thread reads the
+// token's K row addresses and weights once, not once per vector. Loads use
+// the streaming cache hint (y is read once). The 32 output bytes go out in
+// one 256-bit store.
 //
 // The same kernels serve one rank of a one-process-per-GPU deployment (PeerY):
 // each slot's row is then read from the expert output of its destination
@@ -67,7 +70,7 @@ struct PeerY {
 };
 
 constexpr int kChunk = 8;  // slots gathered per pass: kChunk loads in flight per thread
-constexpr int kMaxKFp8 = 8;  // slots held in registers by combine_fp8_k8_kernel
+constexpr int kMaxKFp8 = 8;  // slots held in registers by the *_k8 kernels
 
 // Receive row of slot k, read by every thread (broadcast, L1 after the first
 // warp) so that no warp waits on another; -1 for masked or out-of-range rows.
@@ -137,6 +140,63 @@ __global__ void __launch_bounds__(kBf16Threads * SUB) combine_bf16_kernel(Combin
             u32x8 o;
 #pragma unroll
             for (int j = 0; j < 8; ++j) o.v[j] = pack_bf16x2(acc[2 * j], acc[2 * j + 1]);
+            st256(p.out + (size_t)g * rb + (size_t)v * 32, o);
+        }
+    }
+}
+
+// combine_bf16_kernel for K <= kMaxKFp8: the token's K row addresses and
+// weights are read once per token into registers (masked and refused slots
+// are skipped), then each thread walks its 32-byte vectors.
+template <class Y, int SUB>
+__global__ void __launch_bounds__(kBf16Threads * SUB) combine_bf16_k8_kernel(CombineParams p, Y py) {
+    const int nvec = p.H / 16;  // 32-byte vectors: 16 bf16 channels
+    const size_t rb = (size_t)p.H * 2;
+    const int sub = threadIdx.x / kBf16Threads, tid = threadIdx.x - sub * kBf16Threads;
+    for (int64_t g = (int64_t)blockIdx.x * SUB + sub; g < p.N; g += (int64_t)gridDim.x * SUB) {
+        report_rows<Y>(p, g, tid);
+        const uint8_t* base[kMaxKFp8];
+        float w[kMaxKFp8];
+        uint32_t live = 0;  // bit i: slot i is read
+#pragma unroll
+        for (int i = 0; i < kMaxKFp8; ++i) {
+            base[i] = nullptr;
+            w[i] = 0.0f;
+            if (i < p.K) {
+                const int32_t r = row_of(p, g, i);
+                if (r >= 0) {
+                    if constexpr (Y::kPeer) base[i] = peer_row(p, py, g, i, r, rb);
+                    else base[i] = p.y + (size_t)r * rb;
+                    if (base[i] != nullptr) {
+                        w[i] = __ldg(p.topk_w + g * p.K + i);
+                        live |= 1u << i;
+                    }
+                }
+            }
+        }
+        for (int v = tid; v < nvec; v += kBf16Threads) {
+            u32x8 q[kMaxKFp8];
+#pragma unroll
+            for (int i = 0; i < kMaxKFp8; ++i)
+                if ((live >> i) & 1u) q[i] = ld256_stream(base[i] + (size_t)v * 32);
+            uint64_t acc[8];  // channel pairs (2j, 2j+1) as fp32 pairs
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = 0ull;
+#pragma unroll
+            for (int i = 0; i < kMaxKFp8; ++i) {
+                if ((live >> i) & 1u) {
+                    const uint64_t w2 = f32x2_pack(w[i], w[i]);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)  // per channel: acc = fma(w, y, acc), rounded as the scalar chain
+                        acc[j] = f32x2_fma_rn(w2, f32x2_pack(bf16lo(q[i].v[j]), bf16hi(q[i].v[j])), acc[j]);
+                }
+            }
+            u32x8 o;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float2 a = f32x2_unpack(acc[j]);
+                o.v[j] = pack_bf16x2(a.x, a.y);
+            }
             st256(p.out + (size_t)g * rb + (size_t)v * 32, o);
         }
     }
@@ -578,19 +638,26 @@ template <class Y>
 cudaError_t launch_y(const ep_buffer& b, const CombineParams& p, const Y& py, bool fp8, cudaStream_t st) {
     const ep_config_t& c = b.cfg;
     const int sm_cap = (c.num_sms > 0 && c.num_sms < b.sm_count) ? c.num_sms : b.sm_count;
+    const bool k8 = p.K <= kMaxKFp8;
     if (sm_cap == b.sm_count) {  // one CTA per token (a grid-stride loop past 2^31 - 1 tokens)
         const unsigned grid = (unsigned)(p.N < 0x7fffffff ? p.N : 0x7fffffff);
-        if (fp8 && p.K <= kMaxKFp8) combine_fp8_k8_kernel<Y, 1><<<grid, kFp8Threads, 0, st>>>(p, py);
+        if (fp8 && k8) combine_fp8_k8_kernel<Y, 1><<<grid, kFp8Threads, 0, st>>>(p, py);
         else if (fp8) combine_fp8_kernel<Y, 1><<<grid, kFp8Threads, 0, st>>>(p, py);
+        else if (k8) combine_bf16_k8_kernel<Y, 1><<<grid, kBf16Threads, 0, st>>>(p, py);
         else combine_bf16_kernel<Y, 1><<<grid, kBf16Threads, 0, st>>>(p, py);
         return cudaGetLastError();
     }
-    // num_sms cap (Buffer.set_num_sms): at most sm_cap CTAs, each filling an SM
-    if (!fp8 && p.K <= kTmaMaxK) return launch_tma(p, py, sm_cap, st);
+    // num_sms cap (Buffer.set_num_sms): at most sm_cap CTAs, each filling an
+    // SM. bf16 y: the bulk-copy pipeline where the rows split into whole
+    // units (measured on B200, 20 SMs: prefill H = 7168 2.2 ms against 2.4
+    // for the register gather below; skewed H = 4096, whose 512-channel tail
+    // unit would hold a whole stage, 1.66 against 1.24 ms).
+    if (!fp8 && p.K <= kTmaMaxK && p.H % kTmaChunk == 0) return launch_tma(p, py, sm_cap, st);
     const int sub = fp8 ? kFp8Sub : kBf16Sub;
     int64_t grid = (p.N + sub - 1) / sub;
     if (grid > sm_cap) grid = sm_cap;
     if (fp8) combine_fp8_kernel<Y, kFp8Sub><<<(unsigned)grid, kFp8Threads * kFp8Sub, 0, st>>>(p, py);
+    else if (k8) combine_bf16_k8_kernel<Y, kBf16Sub><<<(unsigned)grid, kBf16Threads * kBf16Sub, 0, st>>>(p, py);
     else combine_bf16_kernel<Y, kBf16Sub><<<(unsigned)grid, kBf16Threads * kBf16Sub, 0, st>>>(p, py);
     return cudaGetLastError();
 }

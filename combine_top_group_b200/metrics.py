@@ -107,7 +107,8 @@ SHARED_SOURCES = ("common.cuh", "internal.h")
 NCU_NAMES = {
     "layout": "layout_kernel",
     "dispatch": ("dispatch_bf16_kernel", "dispatch_fp8_kernel"),
-    "combine": ("combine_bf16_kernel", "combine_fp8_kernel"),
+    "combine": ("combine_bf16_kernel", "combine_fp8_kernel", "combine_bf16_k8_kernel", "combine_fp8_k8_kernel",
+                "combine_bf16_tma_kernel"),
 }
 
 

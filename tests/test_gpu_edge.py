@@ -379,17 +379,17 @@ def _kernel_grids(fn):
 @pytest.mark.parametrize("num_sms", [7, 20])
 def test_capped_kernels_launch_at_most_num_sms_ctas(cuda, num_sms):
     """Under a num_sms cap every dispatch and combine kernel (bf16, FP8, the
-    fused FP8 combine, the bulk-copy combine, the dedup kernels) launches at
-    most num_sms CTAs, so it can occupy at most num_sms SMs; without a cap the
-    grid is one CTA per token."""
+    fused FP8 combine, the bulk-copy combine at H = 7168, the register combine
+    elsewhere, the dedup kernels) launches at most num_sms CTAs, so it can
+    occupy at most num_sms SMs; without a cap the grid is one CTA per token."""
     ep, runner = cuda
     capped = ("dispatch", "combine", "permute", "local_reduce")
     seen = set()
     for name, fused, dedup in (("tiny", False, False), ("decode", True, False), ("skewed", False, False),
-                               ("decode", True, True)):
+                               ("prefill", False, False), ("decode", True, True)):
         w = wl.WORKLOADS[name]
-        if name == "skewed":
-            w = w.with_tokens(64)
+        if name in ("skewed", "prefill"):
+            w = w.with_tokens(64 if name == "skewed" else 32)
         pipe = runner.Pipeline(w, 2, dedup=dedup)
 
         def run():
