@@ -362,9 +362,10 @@ __global__ void __launch_bounds__(kFp8Threads * SUB) combine_fp8_k8_kernel(Combi
 // then keeps at most 128 KB per SM in flight (512 threads, 8 loads of 32 B
 // each). Here the bulk-copy (TMA) engine moves the rows into shared memory
 // instead: 4 stages, each K row segments of kTmaChunk channels (56 KB at
-// K = 8), so the threads issue only the arithmetic. Measured on B200 at the
-// prefill shape (8 x 4096 tokens, H = 7168, K = 8): 2.2 ms at 20 SMs and
-// 0.66 ms at 74 SMs, against 2.9 and 0.88 ms for the register gather. Every
+// K = 8), so the threads issue only the arithmetic. Used where H is a
+// multiple of kTmaChunk. Measured on B200 at the prefill shape (8 x 4096
+// tokens, H = 7168, K = 8): 2.2 ms at 20 SMs and 0.66 ms at 74 SMs, against
+// 2.4 and 0.79 ms for the register gather (combine_bf16_k8_kernel). Every
 // byte crosses shared memory twice (the copy, then the consumers' reads),
 // which bounds this design at about half the shared-memory bandwidth.
 // Slower, as measured:

@@ -4,6 +4,7 @@ from __future__ import annotations
 
 import csv
 import hashlib
+import re
 import io
 import json
 import os
@@ -112,19 +113,29 @@ NCU_NAMES = {
 }
 
 
+_COMMENT = re.compile(r"//[^\n]*|/\*.*?\*/", re.S)
+
+
+def code_of(text: str) -> str:
+    """Source text without its comments and with every run of whitespace
+    collapsed to one space: what the compiler sees. (The kernel sources hold
+    no string literal with a comment marker in it.)"""
+    return " ".join(_COMMENT.sub(" ", text).split())
+
+
 def source_hash(kernel: str | None = None) -> str:
-    """Hash of the sources a kernel is built from (all kernel sources when
-    `kernel` is None); a stored ncu traffic figure is only valid for the
-    sources it was captured from."""
+    """Hash of the code a kernel is built from (all kernel sources when
+    `kernel` is None); a stored ncu traffic figure is only valid for the code
+    it was captured from. Comments and layout do not count."""
     if kernel is None:
         names = sorted(n for n in os.listdir(CSRC) if n.endswith((".cu", ".cuh", ".h")))
     else:
         names = sorted(set(KERNEL_SOURCES[kernel]) | set(SHARED_SOURCES))
     h = hashlib.sha256()
     for name in names:
-        with open(os.path.join(CSRC, name), "rb") as f:
+        with open(os.path.join(CSRC, name), encoding="utf-8") as f:
             h.update(name.encode())
-            h.update(f.read())
+            h.update(code_of(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -115,3 +115,21 @@ def test_stored_traffic_entries():
             assert k["scale_to_workload"] == scale
             assert k["dram_bytes_per_launch"] == round((k["dram_read"] + k["dram_write"]) * scale)
             assert len(k["source_hash"]) == 16
+
+
+def test_source_hash_ignores_comments_not_code(tmp_path, monkeypatch):
+    """A stored traffic figure stays valid across comment-only edits of its
+    kernel's sources, and not across a code change."""
+    import shutil
+    from combine_top_group_b200 import metrics
+    for name in set(metrics.KERNEL_SOURCES["combine"]) | set(metrics.SHARED_SOURCES):
+        shutil.copy(os.path.join(metrics.CSRC, name), tmp_path / name)
+    monkeypatch.setattr(metrics, "CSRC", str(tmp_path))
+    base = metrics.source_hash("combine")
+    src = (tmp_path / "combine.cu").read_text()
+    edited = "// a new note\n/* and a block\n   note */\n" + src.replace("\n", "\n\n", 3)
+    assert edited != src
+    (tmp_path / "combine.cu").write_text(edited)
+    assert metrics.source_hash("combine") == base
+    (tmp_path / "combine.cu").write_text(src.replace("kTmaStages = 4", "kTmaStages = 3", 1))
+    assert metrics.source_hash("combine") != base
