@@ -73,7 +73,14 @@ struct LayoutParams {
 };
 
 __device__ __forceinline__ double sigmoid_d(double x) { return 1.0 / (1.0 + exp(-x)); }
-__device__ __forceinline__ float sigmoid_f(float x) { return __frcp_rn(1.0f + expf(-x)); }
+// fp32 sigmoid from the fast intrinsics, whose published maximum errors are
+// 2 + floor(|1.173 x|) ulp for __expf(x) and 2 ulp for __fdividef(x, y) with
+// 2^-126 <= |y| <= 2^126 (0 above, where the true value is below 2^-126).
+// With e = __expf(-x) off by |d| <= (2 + 1.2|x|) 2^-23 relative, the add and
+// the divide by 2^-24 and 2^-22 relative:
+//   |s - sigmoid(x)| <= s(1-s)|d| + s(2^-24 + 2^-22) <= (0.63 + 0.5 + 2) 2^-23 < 3.8e-7,
+// as s(1-s)(2 + 1.2|x|) <= 0.63 for every x.
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
     uint32_t v;
@@ -158,7 +165,15 @@ __device__ __forceinline__ uint32_t kept_groups(const LayoutParams& p, const uin
         // group g's fp32 score sits on lane g * lpg. A group's rank is the
         // number of groups ahead of it: higher score, or equal score and lower
         // id. Kept = rank < KG.
-        const float s32 = sigmoid_f(key_value(a)) + sigmoid_f(key_value(b));
+        // group score: lane pairs (2i, 2i+1) inside a group take one sigmoid
+        // each, of a and of b, and add them (either order: the sum is exact)
+        float s32;
+        if (lpg >= 2) {
+            const float sg1 = sigmoid_f(key_value((lane & 1) ? b : a));
+            s32 = sg1 + __shfl_xor_sync(FULL, sg1, 1);
+        } else {
+            s32 = sigmoid_f(key_value(a)) + sigmoid_f(key_value(b));
+        }
         float sg;   // score of group gq
         int gq, rk;  // rank of group gq, on the lanes that report it
         bool lead;  // this lane reports group gq
@@ -187,8 +202,9 @@ __device__ __forceinline__ uint32_t kept_groups(const LayoutParams& p, const uin
         const uint32_t kept = __reduce_or_sync(FULL, (lead && rk < p.KG) ? 1u << gq : 0u);  // gq < G <= 32
         bool certain = true;
         if (p.KG < p.G) {
-            // fp32 sigmoid error <= 3*2^-23 (expf <= 2 ulp, add and rcp 0.5 ulp each),
-            // so a score errs by < 1e-6. A gap over 4e-6 decides as fp64 would.
+            // A score (two sigmoids < 3.8e-7 each, then an add rounding
+            // < 1.2e-7) errs by < 9e-7, a gap between two by < 1.8e-6. A gap
+            // over 4e-6 decides as fp64 would.
             const uint32_t m_last = __ballot_sync(FULL, lead && rk == p.KG - 1);
             const uint32_t m_next = __ballot_sync(FULL, lead && rk == p.KG);
             const float s_last = __shfl_sync(FULL, sg, __ffs(m_last) - 1);

@@ -113,3 +113,46 @@ def test_group_score_ties_decide_by_lower_id(cuda):
     assert (np.abs(g_w - o_w) <= 2.0 ** -22 * np.abs(o_w)).all()
     # all-equal tokens keep groups 0..3 only
     assert (o_idx[:half] < 128).all()
+
+
+def test_group_scores_within_fp32_error_decide_as_fp64(cuda):
+    """Groups 2 and 5 compete for the last kept group with fp64 scores a few
+    1e-8 apart (either sign, or equal), far below what fp32 sigmoids resolve:
+    the kernel's certainty test must send these tokens to the fp64 path, and
+    the selection must equal the oracle's fp64 decision for every token."""
+    ep, runner = cuda
+    w = wl.Workload("near_ties", R=2, T=64, H=128, E=256, K=8, G=8, KG=4, route=G)
+    rng = np.random.default_rng(11)
+    N = w.N
+    logits = np.empty((N, 256), np.float32)
+    for g in range(8):  # everything else well below each group's top two
+        logits[:, 32 * g:32 * g + 32] = rng.uniform(-6.0, -5.0, (N, 32))
+    for g in (0, 1, 3):  # clearly kept
+        logits[:, 32 * g] = 3.0
+        logits[:, 32 * g + 1] = 2.9
+    x1 = rng.uniform(-0.5, 1.5, N).astype(np.float32)
+    x2 = (x1 - rng.uniform(0.05, 0.5, N)).astype(np.float32)
+    logits[:, 64], logits[:, 65] = x1, x2  # group 2
+    k1 = rng.integers(-3, 4, N)
+    k2 = rng.integers(-3, 4, N)
+    y1 = x1.copy()
+    y2 = x2.copy()
+    for i in range(N):  # group 5: each of its top two a few ulps from group 2's
+        for _ in range(abs(k1[i])):
+            y1[i] = np.nextafter(y1[i], np.float32(np.inf if k1[i] > 0 else -np.inf))
+        for _ in range(abs(k2[i])):
+            y2[i] = np.nextafter(y2[i], np.float32(np.inf if k2[i] > 0 else -np.inf))
+    logits[:, 160], logits[:, 161] = y1, y2
+    x = wl.make_x(w, 11)
+    pipe = runner.Pipeline(w, 11, x=x, logits=logits)
+    pipe.layout()
+    assert pipe.check_errors() == 0
+    lay = ep.ep_buffer_layout(pipe.buf, w.T)
+    o_idx, o_w, margin = oracle_route(w, logits)
+    assert (margin < 1e-6).mean() > 0.9  # the decision really is within fp32 error
+    g_idx = to_host(lay["topk_idx"])
+    assert np.array_equal(g_idx, o_idx)
+    kept5 = (o_idx >= 160) & (o_idx < 192)
+    assert kept5.any(axis=1).any() and (~kept5.any(axis=1)).any()  # both outcomes occur
+    g_w = to_host(lay["topk_w"]).astype(np.float64)
+    assert (np.abs(g_w - o_w) <= 2.0 ** -22 * np.abs(o_w)).all()
