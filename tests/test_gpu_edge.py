@@ -208,6 +208,28 @@ def test_capped_combine_prefill_shape(cuda, num_sms):
     check_combine(to_host(pipe.out), combine_expected(w, x, o_idx, o_w, np.arange(w.N), "bf16"))
 
 
+@pytest.mark.parametrize("num_sms", [3, 20])
+def test_capped_bulk_copy_combine_k6_masked(cuda, num_sms):
+    """The bulk-copy combine (bf16 y, H = 7168) with K = 6 and 5% of the slots
+    masked, on a token count that the CTAs share unevenly: the output equals
+    the uncapped run's bit for bit and the oracle's within the tolerance."""
+    ep, runner = cuda
+    from parity_util import check_combine, combine_expected, oracle_route, to_host
+    w = wl.Workload("k6_masked", R=4, T=97, H=7168, E=64, K=6, mask_frac=0.05)
+    x, logits = wl.make_x(w, 8), wl.make_logits(w, 8)
+    pipe = runner.Pipeline(w, 8, x=x, logits=logits)
+    pipe.step()
+    ref = pipe.out.clone()
+    ep.ep_buffer_set_num_sms(pipe.buf, num_sms)
+    pipe.out.zero_()
+    pipe.step()
+    assert pipe.check_errors() == 0
+    assert torch.equal(pipe.out.view(torch.int16), ref.view(torch.int16))
+    o_idx, o_w, _ = oracle_route(w, logits)
+    assert (o_idx == -1).any()
+    check_combine(to_host(pipe.out), combine_expected(w, x, o_idx, o_w, np.arange(w.N), "bf16"))
+
+
 def test_capped_shard_combine_through_peer_tables(cuda):
     """The one-rank-per-GPU combine (peer pointer tables) under an SM budget
     gives the uncapped bytes."""
