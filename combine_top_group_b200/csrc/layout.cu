@@ -41,6 +41,7 @@ namespace ep {
 namespace {
 
 constexpr int kWarps = 8;  // warps per CTA
+constexpr int kPrePlace = 2;  // placement rounds (32 slots each) whose experts are loaded ahead
 constexpr int kThreads = kWarps * 32;
 
 struct LayoutParams {
@@ -555,7 +556,19 @@ __global__ void __launch_bounds__(kThreads, EPL >= 16 ? 2 : 4) layout_kernel(Lay
     }
     grid_barrier(p.bar, 2u * (uint32_t)p.nb, p.err);
 
-    // ---- phase 3: expert offsets, per-warp bases, row placement
+    // ---- phase 3: expert offsets, per-warp bases, row placement. The warp's
+    // first kPrePlace * 32 slot experts and this thread's chunk prefix are
+    // loaded before the scan, so their latency overlaps it.
+    const unsigned lt = (1u << lane) - 1u;
+    const int64_t slot0 = ((int64_t)s * p.T + w0) * p.K;
+    const int nslots = has_chunk ? (w1 - w0) * p.K : 0;
+    int pre_e[kPrePlace];
+#pragma unroll
+    for (int q = 0; q < kPrePlace; ++q) {
+        const int j = q * 32 + lane;
+        pre_e[q] = (j < nslots) ? p.topk_idx[slot0 + j] : -1;
+    }
+    const int pre_chunk = (has_chunk && (int)threadIdx.x < p.E) ? p.chunk[(int64_t)threadIdx.x * p.nc + c] : 0;
     block_exclusive_scan(p.tot, 1, p.E, eoff, warp_tot);
     if (blockIdx.x == 0) {
         for (int e = threadIdx.x; e <= p.E; e += kThreads) p.expert_off[e] = eoff[e];
@@ -594,9 +607,9 @@ __global__ void __launch_bounds__(kThreads, EPL >= 16 ? 2 : 4) layout_kernel(Lay
         for (int e = threadIdx.x; e < p.E; e += kThreads) {
             // standard: expert block + chunk prefix. Low-latency: fixed region of
             // (e, s) + this rank's part of the chunk prefix
-            int run = p.ll ? (int)(((int64_t)e * p.R + s) * p.T_max) + p.chunk[(int64_t)e * p.nc + c] -
-                                 p.src_off[(int64_t)e * p.R + s]
-                           : eoff[e] + p.chunk[(int64_t)e * p.nc + c];
+            const int cpre = (e == (int)threadIdx.x) ? pre_chunk : p.chunk[(int64_t)e * p.nc + c];
+            int run = p.ll ? (int)(((int64_t)e * p.R + s) * p.T_max) + cpre - p.src_off[(int64_t)e * p.R + s]
+                           : eoff[e] + cpre;
 #pragma unroll
             for (int w = 0; w < kWarps; ++w) {
                 const int x = hist[w * p.J + e];
@@ -605,13 +618,14 @@ __global__ void __launch_bounds__(kThreads, EPL >= 16 ? 2 : 4) layout_kernel(Lay
             }
         }
         __syncthreads();
-        const unsigned lt = (1u << lane) - 1u;
-        const int64_t slot0 = ((int64_t)s * p.T + w0) * p.K;
-        const int nslots = (w1 - w0) * p.K;
         for (int i0 = 0; i0 < nslots; i0 += 32) {
             const int j = i0 + lane;
             const bool active = j < nslots;
-            const int e = active ? p.topk_idx[slot0 + j] : -1;
+            int e = -1;
+#pragma unroll
+            for (int q = 0; q < kPrePlace; ++q)
+                if (i0 == q * 32) e = pre_e[q];
+            if (i0 >= kPrePlace * 32) e = active ? p.topk_idx[slot0 + j] : -1;
             const bool valid = e >= 0;
             const unsigned peers = __match_any_sync(FULL, valid ? e : -1);
             if (active) {
