@@ -230,6 +230,30 @@ def test_capped_bulk_copy_combine_k6_masked(cuda, num_sms):
     check_combine(to_host(pipe.out), combine_expected(w, x, o_idx, o_w, np.arange(w.N), "bf16"))
 
 
+@pytest.mark.parametrize("num_sms", [1, 5])
+def test_capped_top16(cuda, num_sms):
+    """K = 16 (above the kernels that hold 8 slots in registers): grouped
+    dispatch and the general combine under a num_sms cap give the uncapped
+    bytes, and the output is the oracle's."""
+    ep, runner = cuda
+    from parity_util import check_combine, combine_expected, oracle_route, to_host
+    w = wl.Workload("top16", R=2, T=75, H=512, E=32, K=16)
+    x, logits = wl.make_x(w, 9), wl.make_logits(w, 9)
+    pipe = runner.Pipeline(w, 9, x=x, logits=logits)
+    pipe.step()
+    M = pipe.num_rows()
+    ref = (pipe.recv["recv_x"][:M].clone(), pipe.out.clone())
+    ep.ep_buffer_set_num_sms(pipe.buf, num_sms)
+    pipe.recv["recv_x"][:M].zero_()
+    pipe.out.zero_()
+    pipe.step()
+    assert pipe.check_errors() == 0
+    assert torch.equal(pipe.recv["recv_x"][:M].view(torch.int16), ref[0].view(torch.int16))
+    assert torch.equal(pipe.out.view(torch.int16), ref[1].view(torch.int16))
+    o_idx, o_w, _ = oracle_route(w, logits)
+    check_combine(to_host(pipe.out), combine_expected(w, x, o_idx, o_w, np.arange(w.N), "bf16"))
+
+
 def test_capped_shard_combine_through_peer_tables(cuda):
     """The one-rank-per-GPU combine (peer pointer tables) under an SM budget
     gives the uncapped bytes."""
